@@ -1,0 +1,124 @@
+"""Seeded synthetic inputs for the nanochat forward pass.
+
+This module only draws random numbers and converts storage formats.  It holds
+none of the forward pass's arithmetic, so both the CUDA path and the CPU oracle
+can take their inputs from it without sharing any of the method.
+
+The pages train on ClimbMix text with a 32 768-token BPE vocabulary ("nanochat
+depth sweep" model card, Training).  That corpus is not available here, so
+token ids are drawn uniformly from [0, V): the worst case for gather locality,
+and FLOP-neutral.
+
+Weights follow the synthetic recipe: every Linear weight ~ N(0, 1/fan_in),
+the token and value-embedding tables ~ N(0, 1), the gate weights ~ N(0, 1/12)
+(gate logits ~ N(0, 1) on unit-RMS input), lambda = 1, mu = 0.1, beta = 0.5.
+
+Every tensor has its own PCG64 stream keyed by (seed, tensor id), so a subset
+of the tensors (one layer, one row) can be regenerated without drawing the
+rest.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+SEED_BASE = 20260  # seed of workload i is SEED_BASE + i
+
+# tensor ids for the per-tensor streams
+_ID_TOKENS, _ID_TARGETS, _ID_WTE, _ID_HEAD, _ID_SMEAR = 1, 2, 3, 4, 5
+_ID_Q, _ID_K, _ID_V = 11, 12, 13
+_LAYER_BASE = 1000  # layer l uses ids _LAYER_BASE + 16*l + j
+
+
+def _gen(seed: int, tid: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64([int(seed), int(tid)]))
+
+
+def normal(seed: int, tid: int, shape, std: float) -> np.ndarray:
+    """float32 N(0, std^2) array from the stream (seed, tid)."""
+    a = _gen(seed, tid).standard_normal(size=shape, dtype=np.float32)
+    if std != 1.0:
+        a *= np.float32(std)
+    return a
+
+
+def round_bf16(a: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest bfloat16 (ties to even); the result
+    is float32 holding bf16-representable values."""
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    u = a.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + lsb) >> 16) << 16
+    nan = np.isnan(a)
+    out = r.astype(np.uint32).view(np.float32).copy()
+    out[nan] = np.float32("nan")
+    return out.reshape(a.shape)
+
+
+def bf16_bits(a: np.ndarray) -> np.ndarray:
+    """uint16 bit patterns of float32 values that are already bf16-exact."""
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    return (a.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def tokens(seed: int, B: int, T: int, V: int) -> np.ndarray:
+    return _gen(seed, _ID_TOKENS).integers(0, V, size=(B, T), dtype=np.int64).astype(np.int32)
+
+
+def targets(seed: int, B: int, T: int, V: int) -> np.ndarray:
+    return _gen(seed, _ID_TARGETS).integers(0, V, size=(B, T), dtype=np.int64).astype(np.int32)
+
+
+def params(seed: int, *, n_layer: int, n_embd: int, n_head: int, n_kv_head: int,
+           head_dim: int, vocab: int, vocab_padded: int, ve_layers, gate_channels: int = 12,
+           bf16: bool = True, layers=None) -> dict:
+    """Synthetic parameter set.
+
+    Shapes follow the nn.Linear [out, in] convention.  `ve_layers` lists the
+    layers that carry a value embedding; `layers` optionally restricts which
+    layers are drawn (the others are None).  With bf16=True every matrix and
+    table is rounded to bf16 values (still stored as float32); gates and
+    scalars stay float32.
+    """
+    C, Hq, Hkv, D, V = n_embd, n_head, n_kv_head, head_dim, vocab
+    ve_layers = set(int(l) for l in ve_layers)
+    rnd = round_bf16 if bf16 else (lambda a: a)
+    p = {
+        "wte": rnd(normal(seed, _ID_WTE, (V, C), 1.0)),
+        "lm_head": rnd(normal(seed, _ID_HEAD, (vocab_padded, C), C ** -0.5)),
+        "smear_gate": normal(seed, _ID_SMEAR, (gate_channels,), gate_channels ** -0.5),
+        "resid_lambdas": np.ones(n_layer, np.float32),
+        "x0_lambdas": np.full(n_layer, 0.1, np.float32),
+        "backout_lambda": np.float32(0.5),
+        "layers": [],
+    }
+    want = range(n_layer) if layers is None else set(layers)
+    for l in range(n_layer):
+        if l not in want:
+            p["layers"].append(None)
+            continue
+        b = _LAYER_BASE + 16 * l
+        nqkv = (Hq + 2 * Hkv) * D
+        lp = {
+            "w_qkv": rnd(normal(seed, b + 0, (nqkv, C), C ** -0.5)),
+            "w_o": rnd(normal(seed, b + 1, (C, Hq * D), (Hq * D) ** -0.5)),
+            "w_fc1": rnd(normal(seed, b + 2, (4 * C, C), C ** -0.5)),
+            "w_fc2": rnd(normal(seed, b + 3, (C, 4 * C), (4 * C) ** -0.5)),
+            "ve": None,
+            "ve_gate": None,
+        }
+        if l in ve_layers:
+            lp["ve"] = rnd(normal(seed, b + 4, (V, Hkv * D), 1.0))
+            lp["ve_gate"] = normal(seed, b + 5, (Hkv, gate_channels), gate_channels ** -0.5)
+        p["layers"].append(lp)
+    return p
+
+
+def attention_inputs(seed: int, B: int, T: int, H: int, D: int, Hkv: int | None = None,
+                     bf16: bool = True):
+    """q, k, v ~ N(0, 1) shaped (B, T, H, D) / (B, T, Hkv, D)."""
+    Hkv = H if Hkv is None else Hkv
+    rnd = round_bf16 if bf16 else (lambda a: a)
+    q = rnd(normal(seed, _ID_Q, (B, T, H, D), 1.0))
+    k = rnd(normal(seed, _ID_K, (B, T, Hkv, D), 1.0))
+    v = rnd(normal(seed, _ID_V, (B, T, Hkv, D), 1.0))
+    return q, k, v
