@@ -1,0 +1,469 @@
+// C ABI of libnc.so (declared in include/nc.h): configuration, workspace
+// layout, argument checks and the launch sequence of the forward pass.
+//
+// The launch sequence follows "The Mathematics of Karpathy's nanochat",
+// §High-Level Forward Pass: embedding + RMSNorm (+ smear, "nanochat depth
+// sweep" card), then per block the x0 re-injection (fused into the previous
+// block's last GEMM epilogue), RMSNorm, the QKV projection, RoPE + QK-norm
+// (+ value embedding), windowed attention, the output projection with the
+// residual add, RMSNorm, FC1 + ReLU^2, FC2 with the residual add; then backout,
+// the final RMSNorm, the head with softcap and the cross-entropy.
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "nc_internal.cuh"
+
+__device__ int g_nc_status;  // OR of 1 << NC_ERR_* bits set by kernels
+
+namespace nc {
+
+static thread_local int t_launches = 0;
+static thread_local char t_err[256] = {0};
+
+void count_launch() { ++t_launches; }
+
+static void set_err(const char* where, cudaError_t e) {
+  snprintf(t_err, sizeof(t_err), "%s: %s", where, cudaGetErrorString(e));
+}
+
+namespace {
+
+constexpr int kMaxDev = 64;
+
+struct DevInfo {
+  int* status = nullptr;
+  int num_sms = 0;
+  bool ok = false;
+};
+DevInfo g_dev[kMaxDev];
+std::mutex g_dev_mu;
+
+// Per-device set-up: the status word's device address and the SM count.
+bool dev_info(DevInfo* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    set_err("cudaGetDevice", e);
+    return false;
+  }
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.ok) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_nc_status);
+    if (e != cudaSuccess) {
+      set_err("cudaGetSymbolAddress", e);
+      return false;
+    }
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) {
+      set_err("cudaDeviceGetAttribute", e);
+      return false;
+    }
+    d.status = static_cast<int*>(p);
+    d.num_sms = sms;
+    d.ok = true;
+  }
+  *out = d;
+  return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+struct Layout {
+  size_t x, x0, xbo, xn, qkv, o, h, gate, rcos, rsin, ce_sum, ce_tgt, logits, tok, tgt, loss;
+  size_t total;
+  int ce_tiles;
+};
+
+bool config_ok(const nc_config& c) {
+  if (c.n_layer <= 0 || c.n_layer > NC_MAX_LAYERS) return false;
+  if (c.n_embd <= 0 || c.n_embd % 128 != 0) return false;
+  if (c.head_dim != 128 || c.n_head <= 0 || c.n_kv_head != c.n_head) return false;
+  if (c.vocab <= 0 || c.vocab_padded < c.vocab || c.vocab_padded % 64 != 0) return false;
+  if (c.mlp_hidden <= 0 || c.mlp_hidden % 128 != 0) return false;
+  if (c.max_T <= 0 || (c.dtype != NC_BF16 && c.dtype != NC_FP32)) return false;
+  if (c.gate_channels < 0 || c.gate_channels > c.n_embd) return false;
+  if (c.backout_layer >= c.n_layer) return false;
+  for (int l = 0; l < c.n_layer; ++l)
+    if (c.window[l] <= 0) return false;
+  return true;
+}
+
+Layout layout(const nc_config& c, int max_tokens) {
+  Layout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t M = (size_t)max_tokens;
+  const size_t C = c.n_embd, D = c.head_dim;
+  const size_t esz = c.dtype == NC_BF16 ? 2 : 4;
+  const size_t nqkv = (size_t)(c.n_head + 2 * c.n_kv_head) * D;
+  L.x = take(M * C * 4);
+  L.x0 = take(M * C * 4);
+  L.xbo = take(M * C * 4);
+  L.xn = take(M * C * esz);
+  L.qkv = take(M * nqkv * esz);
+  L.o = take(M * c.n_head * D * esz);
+  L.h = take(M * (size_t)c.mlp_hidden * esz);
+  L.gate = take(M * c.n_kv_head * 4);
+  L.rcos = take((size_t)c.max_T * D / 2 * 4);
+  L.rsin = take((size_t)c.max_T * D / 2 * 4);
+  L.ce_tiles = (c.vocab_padded + 127) / 128;
+  L.ce_sum = take(M * L.ce_tiles * 4);
+  L.ce_tgt = take(M * 4);
+  const bool simt_head = c.dtype == NC_FP32 || c.gemm_impl != 0;
+  L.logits = take(simt_head ? M * (size_t)c.vocab * 4 : 0);
+  L.tok = take(M * 4);
+  L.tgt = take(M * 4);
+  L.loss = take(M * 4);
+  L.total = off;
+  return L;
+}
+
+template <typename T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(base) + off);
+}
+
+// C = A B^T with the given epilogue, on tensor cores (bf16) or CUDA cores.
+bool gemm(const nc_config& c, const DevInfo& d, const void* A, int lda, const void* B, int ldb, int M,
+          int N, int K, const EpiParams& ep, cudaStream_t st) {
+  if (c.dtype == NC_BF16 && c.gemm_impl == 0)
+    return launch_gemm_tc((const bf16*)A, lda, (const bf16*)B, ldb, M, N, K, ep, d.status, d.num_sms, st);
+  launch_gemm_simt(A, lda, B, ldb, M, N, K, c.dtype == NC_BF16, ep, st);
+  return true;
+}
+
+EpiParams epi(int mode) {
+  EpiParams e;
+  memset(&e, 0, sizeof(e));
+  e.mode = mode;
+  return e;
+}
+
+int check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_err(what, e);
+    return NC_ERR_CUDA;
+  }
+  return NC_OK;
+}
+
+}  // namespace
+}  // namespace nc
+
+using namespace nc;
+
+extern "C" {
+
+int nc_init_config(nc_config* cfg, int depth, int max_T, int dtype, const char* window_pattern,
+                   int short_window, int backout_layer) {
+  if (cfg == nullptr || window_pattern == nullptr) return NC_ERR_ARG;
+  if (depth <= 0 || depth > NC_MAX_LAYERS || max_T <= 0 || short_window <= 0) return NC_ERR_ARG;
+  if (dtype != NC_BF16 && dtype != NC_FP32) return NC_ERR_ARG;
+  const size_t plen = strlen(window_pattern);
+  if (plen == 0) return NC_ERR_ARG;
+  for (size_t i = 0; i < plen; ++i)
+    if (window_pattern[i] != 'S' && window_pattern[i] != 'L') return NC_ERR_ARG;
+  if (backout_layer >= depth) return NC_ERR_ARG;
+  memset(cfg, 0, sizeof(*cfg));
+  const int head_dim = 128, aspect = 64;
+  cfg->n_layer = depth;
+  cfg->n_embd = ((depth * aspect + head_dim - 1) / head_dim) * head_dim;
+  cfg->n_head = cfg->n_embd / head_dim;
+  cfg->n_kv_head = cfg->n_head;
+  cfg->head_dim = head_dim;
+  cfg->vocab = 32768;
+  cfg->vocab_padded = ((cfg->vocab + 63) / 64) * 64;
+  cfg->mlp_hidden = 4 * cfg->n_embd;
+  cfg->max_T = max_T;
+  cfg->dtype = dtype;
+  for (int l = 0; l < depth; ++l) {
+    const char ch = window_pattern[l % plen];
+    cfg->window[l] = (ch == 'L' || l == depth - 1) ? max_T : short_window;
+    cfg->has_ve[l] = (l % 2) == ((depth - 1) % 2);
+  }
+  cfg->backout_layer = backout_layer < 0 ? depth / 2 : backout_layer;
+  cfg->gate_channels = 12;
+  cfg->smear = 1;
+  cfg->gemm_impl = 0;
+  cfg->attn_impl = 1;
+  cfg->qk_alpha = 1.15f;
+  cfg->softmax_scale = 1.0f / sqrtf((float)head_dim);
+  cfg->rope_base = 100000.0f;
+  cfg->eps = 1e-6f;
+  cfg->softcap = 15.0f;
+  cfg->ve_gate_scale = 3.0f;
+  return NC_OK;
+}
+
+size_t nc_workspace_bytes(const nc_config* cfg, int max_tokens) {
+  if (cfg == nullptr || max_tokens <= 0 || !config_ok(*cfg)) return 0;
+  return layout(*cfg, max_tokens).total;
+}
+
+int nc_params_init(nc_params* p, const nc_config* cfg) {
+  if (p == nullptr || cfg == nullptr) return NC_ERR_ARG;
+  memset(p, 0, sizeof(*p));
+  p->cfg = *cfg;
+  return NC_OK;
+}
+
+int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets, int B, int T,
+               float* out_loss, float* out_logits, void* stream) {
+  t_launches = 0;
+  if (p == nullptr || tokens == nullptr || targets == nullptr || out_loss == nullptr) return NC_ERR_ARG;
+  const nc_config& c = p->cfg;
+  if (!config_ok(c)) return NC_ERR_SHAPE;
+  if (B <= 0 || T <= 0 || T > c.max_T || (long long)B * T > (long long)p->max_tokens) return NC_ERR_SHAPE;
+  if (p->wte == nullptr || p->lm_head == nullptr || p->resid_lambdas == nullptr ||
+      p->x0_lambdas == nullptr || (c.smear && c.gate_channels > 0 && p->smear_gate == nullptr))
+    return NC_ERR_ARG;
+  for (int l = 0; l < c.n_layer; ++l) {
+    const nc_layer_params& lp = p->layer[l];
+    if (!lp.w_qkv || !lp.w_o || !lp.w_fc1 || !lp.w_fc2) return NC_ERR_ARG;
+    if (c.has_ve[l] && (!lp.ve || !lp.ve_gate)) return NC_ERR_ARG;
+    if (!aligned16(lp.w_qkv) || !aligned16(lp.w_o) || !aligned16(lp.w_fc1) || !aligned16(lp.w_fc2) ||
+        (lp.ve && !aligned16(lp.ve)))
+      return NC_ERR_ALIGN;
+  }
+  if (!aligned16(p->wte) || !aligned16(p->lm_head) || !aligned16(tokens) || !aligned16(targets) ||
+      !aligned16(out_loss) || (out_logits && !aligned16(out_logits)) || !aligned16(p->workspace))
+    return NC_ERR_ALIGN;
+  const Layout Lw = layout(c, p->max_tokens);
+  if (p->workspace == nullptr || p->workspace_bytes < Lw.total) return NC_ERR_WORKSPACE;
+  if (c.dtype == NC_BF16 && c.gemm_impl == 0 && c.vocab_padded % 128 != 0) return NC_ERR_SHAPE;
+  DevInfo d;
+  if (!dev_info(&d)) return NC_ERR_CUDA;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int M = B * T;
+  const int C = c.n_embd, H = c.n_head, Hkv = c.n_kv_head, D = c.head_dim, V = c.vocab;
+  const int nqkv = (H + 2 * Hkv) * D;
+  const int bf = c.dtype == NC_BF16;
+  void* ws = p->workspace;
+  float* x = at<float>(ws, Lw.x);
+  float* x0 = at<float>(ws, Lw.x0);
+  float* xbo = at<float>(ws, Lw.xbo);
+  void* xn = at<char>(ws, Lw.xn);
+  char* qkv = at<char>(ws, Lw.qkv);
+  void* o = at<char>(ws, Lw.o);
+  void* h = at<char>(ws, Lw.h);
+  float* gate = at<float>(ws, Lw.gate);
+  float* rcos = at<float>(ws, Lw.rcos);
+  float* rsin = at<float>(ws, Lw.rsin);
+  const size_t esz = bf ? 2 : 4;
+
+  launch_rope_table(rcos, rsin, T, D, c.rope_base, st);
+  launch_embed(p->wte, tokens, p->smear_gate, c.smear && c.gate_channels > 0, c.gate_channels,
+               p->resid_lambdas, p->x0_lambdas, c.eps, B, T, C, V, bf, x, x0, d.status, st);
+
+  for (int l = 0; l < c.n_layer; ++l) {
+    const nc_layer_params& lp = p->layer[l];
+    const bool ve = c.has_ve[l] != 0;
+    // attention sub-block
+    launch_rmsnorm(x, xn, M, C, c.eps, bf, ve ? lp.ve_gate : nullptr, Hkv, c.gate_channels,
+                   c.ve_gate_scale, ve ? gate : nullptr, st);
+    EpiParams e = epi(EPI_STORE);
+    e.out = qkv;
+    e.ldo = nqkv;
+    if (!gemm(c, d, xn, C, lp.w_qkv, C, M, nqkv, C, e, st)) return NC_ERR_CUDA;
+    launch_rope_qknorm_ve(qkv, nqkv, B, T, H, Hkv, D, rcos, rsin, c.qk_alpha, c.eps, tokens,
+                          ve ? lp.ve : nullptr, gate, V, bf, d.status, st);
+    const int w = c.window[l] >= T ? T : c.window[l];
+    launch_attn_simt(qkv, qkv + (size_t)H * D * esz, qkv + (size_t)(H + Hkv) * D * esz, nqkv, nqkv, nqkv,
+                     o, H * D, B, T, H, Hkv, w, c.softmax_scale, bf, st);
+    e = epi(EPI_RESID);
+    e.x = x;
+    e.ldx = C;
+    if (!gemm(c, d, o, H * D, lp.w_o, H * D, M, C, H * D, e, st)) return NC_ERR_CUDA;
+    // MLP sub-block
+    launch_rmsnorm(x, xn, M, C, c.eps, bf, nullptr, 0, 0, 0.f, nullptr, st);
+    e = epi(EPI_RELU2);
+    e.out = h;
+    e.ldo = c.mlp_hidden;
+    if (!gemm(c, d, xn, C, lp.w_fc1, C, M, c.mlp_hidden, C, e, st)) return NC_ERR_CUDA;
+    e = epi(EPI_BLOCK_END);
+    e.x = x;
+    e.x0 = x0;
+    e.xbo = xbo;
+    e.ldx = C;
+    e.capture_bo = (l == c.backout_layer);
+    if (l + 1 < c.n_layer) {
+      e.end_kind = 1;
+      e.lam = p->resid_lambdas + l + 1;
+      e.mu = p->x0_lambdas + l + 1;
+    } else {
+      e.end_kind = c.backout_layer >= 0 ? 2 : 0;
+      e.beta = p->backout_lambda;
+    }
+    if (!gemm(c, d, h, c.mlp_hidden, lp.w_fc2, c.mlp_hidden, M, C, c.mlp_hidden, e, st)) return NC_ERR_CUDA;
+  }
+
+  // final norm, head, softcap, cross-entropy
+  launch_rmsnorm(x, xn, M, C, c.eps, bf, nullptr, 0, 0, 0.f, nullptr, st);
+  if (bf && c.gemm_impl == 0) {
+    const int bn = gemm_tc_bn(c.vocab_padded);
+    const int tiles = (c.vocab_padded + bn - 1) / bn;
+    EpiParams e = epi(EPI_CE);
+    e.cap = c.softcap;
+    e.vocab = V;
+    e.logits = out_logits;
+    e.ldl = V;
+    e.targets = targets;
+    e.ce_sum = at<float>(ws, Lw.ce_sum);
+    e.ce_tgt = at<float>(ws, Lw.ce_tgt);
+    e.ce_tiles = tiles;
+    if (!gemm(c, d, xn, C, p->lm_head, C, M, c.vocab_padded, C, e, st)) return NC_ERR_CUDA;
+    launch_ce_combine(e.ce_sum, e.ce_tgt, tiles, c.softcap, targets, M, V, out_loss, d.status, st);
+  } else {
+    float* logits = out_logits ? out_logits : at<float>(ws, Lw.logits);
+    EpiParams e = epi(EPI_SOFTCAP);
+    e.cap = c.softcap;
+    e.vocab = V;
+    e.logits = logits;
+    e.ldl = V;
+    launch_gemm_simt(xn, C, p->lm_head, C, M, c.vocab_padded, C, bf, e, st);
+    launch_ce_rows(logits, V, targets, M, V, out_loss, d.status, st);
+  }
+  return check_launch("nc_forward");
+}
+
+int nc_forward_host(const nc_params* p, const int32_t* h_tokens, const int32_t* h_targets, int B,
+                    int T, float* h_out_loss, void* stream) {
+  if (p == nullptr || h_tokens == nullptr || h_targets == nullptr || h_out_loss == nullptr)
+    return NC_ERR_ARG;
+  if (!config_ok(p->cfg)) return NC_ERR_SHAPE;
+  if (B <= 0 || T <= 0 || (long long)B * T > (long long)p->max_tokens) return NC_ERR_SHAPE;
+  const Layout Lw = layout(p->cfg, p->max_tokens);
+  if (p->workspace == nullptr || p->workspace_bytes < Lw.total) return NC_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t n = (size_t)B * T;
+  int32_t* dtok = at<int32_t>(p->workspace, Lw.tok);
+  int32_t* dtgt = at<int32_t>(p->workspace, Lw.tgt);
+  float* dloss = at<float>(p->workspace, Lw.loss);
+  cudaError_t e = cudaMemcpyAsync(dtok, h_tokens, n * 4, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dtgt, h_targets, n * 4, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) {
+    set_err("nc_forward_host H2D", e);
+    return NC_ERR_CUDA;
+  }
+  const int rc = nc_forward(p, dtok, dtgt, B, T, dloss, nullptr, stream);
+  if (rc != NC_OK) return rc;
+  e = cudaMemcpyAsync(h_out_loss, dloss, n * 4, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) {
+    set_err("nc_forward_host D2H", e);
+    return NC_ERR_CUDA;
+  }
+  return NC_OK;
+}
+
+int nc_loss_mean(const float* loss, const int32_t* targets, int n, float* out_mean, void* stream) {
+  if (loss == nullptr || targets == nullptr || out_mean == nullptr || n < 0) return NC_ERR_ARG;
+  launch_loss_mean(loss, targets, n, out_mean, static_cast<cudaStream_t>(stream));
+  return check_launch("nc_loss_mean");
+}
+
+size_t nc_attention_workspace_bytes(int B, int T, int H, int Hkv, int D, int dtype, int rope_qknorm) {
+  if (B <= 0 || T <= 0 || H <= 0 || Hkv <= 0 || D <= 0) return 0;
+  if (!rope_qknorm) return 0;
+  const size_t esz = dtype == NC_BF16 ? 2 : 4;
+  const size_t M = (size_t)B * T;
+  return align256(M * H * D * esz) + align256(M * Hkv * D * esz) + 2 * align256((size_t)T * D / 2 * 4);
+}
+
+int nc_attention(const void* q, const void* k, const void* v, void* out, int B, int T, int H,
+                 int Hkv, int D, int window, int rope_qknorm, float alpha, float softmax_scale,
+                 float rope_base, float eps, int dtype, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  t_launches = 0;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return NC_ERR_ARG;
+  if (dtype != NC_BF16 && dtype != NC_FP32) return NC_ERR_ARG;
+  if (B <= 0 || T <= 0 || H <= 0 || Hkv <= 0) return NC_ERR_SHAPE;
+  if (D != 128 || Hkv != H) return NC_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return NC_ERR_ALIGN;
+  const size_t need = nc_attention_workspace_bytes(B, T, H, Hkv, D, dtype, rope_qknorm);
+  if (rope_qknorm && (workspace == nullptr || workspace_bytes < need)) return NC_ERR_WORKSPACE;
+  if (rope_qknorm && !aligned16(workspace)) return NC_ERR_ALIGN;
+  DevInfo d;
+  if (!dev_info(&d)) return NC_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int bf = dtype == NC_BF16;
+  const size_t esz = bf ? 2 : 4;
+  const size_t M = (size_t)B * T;
+  const int w = (window <= 0 || window >= T) ? T : window;
+  const void* qa = q;
+  const void* ka = k;
+  if (rope_qknorm) {
+    char* base = static_cast<char*>(workspace);
+    void* qo = base;
+    void* ko = base + align256(M * H * D * esz);
+    float* rc = reinterpret_cast<float*>(base + align256(M * H * D * esz) + align256(M * Hkv * D * esz));
+    float* rs = rc + align256((size_t)T * D / 2 * 4) / 4;
+    launch_rope_table(rc, rs, T, D, rope_base, st);
+    launch_rope_qknorm_copy(q, k, qo, ko, B, T, H, Hkv, D, rc, rs, alpha, eps, bf, st);
+    qa = qo;
+    ka = ko;
+  }
+  launch_attn_simt(qa, ka, v, H * D, Hkv * D, Hkv * D, out, H * D, B, T, H, Hkv, w, softmax_scale, bf, st);
+  return check_launch("nc_attention");
+}
+
+int nc_get_status(void* stream, int* out_bits) {
+  DevInfo d;
+  if (!dev_info(&d)) return NC_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  int bits = 0;
+  if (e == cudaSuccess) e = cudaMemcpy(&bits, d.status, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(d.status, 0, sizeof(int));
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    set_err("nc_get_status", e);
+    return NC_ERR_CUDA;
+  }
+  if (out_bits) *out_bits = bits;
+  if (bits & kStatusTimeout) return NC_ERR_TIMEOUT;
+  if (bits & kStatusData) return NC_ERR_DATA;
+  return NC_OK;
+}
+
+const char* nc_status_string(int s) {
+  switch (s) {
+    case NC_OK: return "ok";
+    case NC_ERR_ARG: return "invalid argument";
+    case NC_ERR_SHAPE: return "unsupported or inconsistent shape";
+    case NC_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case NC_ERR_CUDA: return "CUDA runtime error";
+    case NC_ERR_DATA: return "token or target id out of range (clamped on the device)";
+    case NC_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    case NC_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+const char* nc_last_error(void) { return t_err; }
+
+int nc_last_launch_count(void) { return t_launches; }
+
+size_t nc_sizeof(int which) {
+  switch (which) {
+    case 0: return sizeof(nc_config);
+    case 1: return sizeof(nc_layer_params);
+    case 2: return sizeof(nc_params);
+    default: return 0;
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,124 @@
+// Internal declarations shared by the CUDA translation units of libnc.so.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/nc.h"
+
+namespace nc {
+
+// bits of the device status word
+constexpr int kStatusData = 1 << NC_ERR_DATA;
+constexpr int kStatusTimeout = 1 << NC_ERR_TIMEOUT;
+
+// one second: upper bound of any wait inside a kernel
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+
+using bf16 = __nv_bfloat16;
+
+template <typename T> struct Act;
+template <> struct Act<float> {
+  static __device__ __forceinline__ float ld(const float* p) { return *p; }
+  static __device__ __forceinline__ void st(float* p, float v) { *p = v; }
+  static __device__ __forceinline__ float from(float v) { return v; }
+};
+template <> struct Act<bf16> {
+  static __device__ __forceinline__ float ld(const bf16* p) { return __bfloat162float(*p); }
+  static __device__ __forceinline__ void st(bf16* p, float v) { *p = __float2bfloat16_rn(v); }
+};
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + expf(-z)); }
+
+// ---------------------------------------------------------------------------
+// Epilogue description shared by the GEMM kernels (CUDA-core and tcgen05).
+// C = A B^T is computed in fp32; the epilogue decides what happens to it.
+// ---------------------------------------------------------------------------
+enum EpiMode : int {
+  EPI_STORE = 0,     // out[m, n] = acc                       (act dtype)
+  EPI_RELU2 = 1,     // out[m, n] = max(acc, 0)^2             (act dtype)
+  EPI_RESID = 2,     // x[m, n] += acc                        (fp32 residual)
+  EPI_BLOCK_END = 3, // x += acc; capture x_bo; then re-inject for the next block or apply backout
+  EPI_SOFTCAP = 4,   // logits[m, n] = cap tanh(acc / cap)    (fp32; CUDA-core path)
+  EPI_CE = 5         // softcap + per-(row, tile) log-sum-exp partials (+ optional logits)
+};
+
+struct EpiParams {
+  int mode;
+  void* out;          // EPI_STORE / EPI_RELU2: act [M, ldo]
+  int ldo;
+  float* x;           // residual [M, ldx] fp32
+  const float* x0;    // [M, ldx]
+  float* xbo;         // [M, ldx]
+  int ldx;
+  int capture_bo;     // EPI_BLOCK_END: store x_bo = x + acc
+  int end_kind;       // EPI_BLOCK_END: 0 = nothing after, 1 = x = lam x + mu x0, 2 = x -= beta x_bo
+  const float* lam;   // device scalars of the next block: lambda_{l+1}, mu_{l+1}
+  const float* mu;
+  float beta;
+  // EPI_SOFTCAP / EPI_CE
+  float cap;
+  int vocab;          // columns >= vocab are padding: not written, not in the LSE
+  float* logits;      // [M, ldl] fp32 or NULL
+  int ldl;
+  const int32_t* targets;  // [M]
+  float* ce_sum;      // [M, n_tiles]: sum over the tile's columns of exp(zhat - cap)
+  float* ce_tgt;      // [M]
+  int ce_tiles;
+};
+
+// launchers (host functions), all asynchronous on `st`
+void launch_embed(const void* wte, const int32_t* tokens, const float* smear_gate, int smear,
+                  int gate_channels, const float* lam0, const float* mu0, float eps, int B, int T, int C, int V,
+                  int act_bf16, float* x, float* x0, int* status, cudaStream_t st);
+void launch_rmsnorm(const float* x, void* xn, int M, int C, float eps, int act_bf16,
+                    const float* ve_gate, int Hkv, int gate_channels, float gate_scale, float* gate_out,
+                    cudaStream_t st);
+void launch_rope_table(float* cos_t, float* sin_t, int T, int D, float base, cudaStream_t st);
+void launch_rope_qknorm_ve(void* qkv, int ld, int B, int T, int H, int Hkv, int D,
+                           const float* cos_t, const float* sin_t, float alpha, float eps,
+                           const int32_t* tokens, const void* ve, const float* gate, int V,
+                           int act_bf16, int* status, cudaStream_t st);
+void launch_rope_qknorm_copy(const void* q, const void* k, void* qo, void* ko, int B, int T, int H,
+                             int Hkv, int D, const float* cos_t, const float* sin_t, float alpha,
+                             float eps, int act_bf16, cudaStream_t st);
+void launch_ce_rows(const float* logits, int ldl, const int32_t* targets, int M, int V, float* loss,
+                    int* status, cudaStream_t st);
+void launch_ce_combine(const float* ce_sum, const float* ce_tgt, int n_tiles, float offset,
+                       const int32_t* targets, int M, int V, float* loss, int* status, cudaStream_t st);
+void launch_loss_mean(const float* loss, const int32_t* targets, int n, float* out, cudaStream_t st);
+
+// CUDA-core GEMM: C[M, N] = A[M, K] B[N, K]^T, fp32 accumulate
+void launch_gemm_simt(const void* A, int lda, const void* Bm, int ldb, int M, int N, int K,
+                      int act_bf16, const EpiParams& ep, cudaStream_t st);
+// CUDA-core attention over q/k/v with row strides (in elements)
+void launch_attn_simt(const void* q, const void* k, const void* v, int ldq, int ldk, int ldv,
+                      void* o, int ldo, int B, int T, int H, int Hkv, int window, float scale,
+                      int act_bf16, cudaStream_t st);
+
+// tcgen05 GEMM (bf16 only).  Returns false if the tensor maps cannot be built.
+int gemm_tc_bn(int N);  // output tile width the tcgen05 GEMM uses for N columns
+bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int N, int K,
+                    const EpiParams& ep, int* status, int num_sms, cudaStream_t st);
+// tcgen05 attention (bf16 only)
+bool launch_attn_tc(const bf16* q, const bf16* k, const bf16* v, int ldq, int ldk, int ldv, bf16* o,
+                    int ldo, int B, int T, int H, int Hkv, int window, float scale, int* status,
+                    int num_sms, cudaStream_t st);
+
+// launch counter (per host thread), incremented by every launcher
+void count_launch();
+
+}  // namespace nc

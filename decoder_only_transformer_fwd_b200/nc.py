@@ -1,0 +1,234 @@
+"""ctypes binding of libnc.so (include/nc.h).
+
+Argument marshalling only: device buffers are torch tensors (PyTorch is used
+for allocation and streams), every step of the forward pass runs in the
+library's CUDA kernels.  The library is loaded on first use and a missing
+build raises immediately; there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+NC_MAX_LAYERS = 64
+NC_BF16, NC_FP32 = 0, 1
+STATUS = {0: "NC_OK", 1: "NC_ERR_ARG", 2: "NC_ERR_SHAPE", 3: "NC_ERR_ALIGN", 4: "NC_ERR_CUDA",
+          5: "NC_ERR_DATA", 6: "NC_ERR_TIMEOUT", 7: "NC_ERR_WORKSPACE"}
+STATUS_CODES = {v: k for k, v in STATUS.items()}
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnc.so")
+
+
+class nc_config(C.Structure):
+    _fields_ = [("n_layer", C.c_int), ("n_embd", C.c_int), ("n_head", C.c_int),
+                ("n_kv_head", C.c_int), ("head_dim", C.c_int), ("vocab", C.c_int),
+                ("vocab_padded", C.c_int), ("mlp_hidden", C.c_int), ("max_T", C.c_int),
+                ("dtype", C.c_int), ("window", C.c_int * NC_MAX_LAYERS),
+                ("has_ve", C.c_int * NC_MAX_LAYERS), ("backout_layer", C.c_int),
+                ("gate_channels", C.c_int), ("smear", C.c_int), ("gemm_impl", C.c_int),
+                ("attn_impl", C.c_int), ("qk_alpha", C.c_float), ("softmax_scale", C.c_float),
+                ("rope_base", C.c_float), ("eps", C.c_float), ("softcap", C.c_float),
+                ("ve_gate_scale", C.c_float)]
+
+
+class nc_layer_params(C.Structure):
+    _fields_ = [("w_qkv", C.c_void_p), ("w_o", C.c_void_p), ("w_fc1", C.c_void_p),
+                ("w_fc2", C.c_void_p), ("ve", C.c_void_p), ("ve_gate", C.c_void_p)]
+
+
+class nc_params(C.Structure):
+    _fields_ = [("cfg", nc_config), ("wte", C.c_void_p), ("lm_head", C.c_void_p),
+                ("smear_gate", C.c_void_p), ("resid_lambdas", C.c_void_p),
+                ("x0_lambdas", C.c_void_p), ("backout_lambda", C.c_float),
+                ("layer", nc_layer_params * NC_MAX_LAYERS), ("workspace", C.c_void_p),
+                ("workspace_bytes", C.c_size_t), ("max_tokens", C.c_int)]
+
+
+class NcError(RuntimeError):
+    pass
+
+
+_lib = None
+
+_SIGS = {
+    "nc_init_config": (C.c_int, [C.POINTER(nc_config), C.c_int, C.c_int, C.c_int, C.c_char_p, C.c_int, C.c_int]),
+    "nc_workspace_bytes": (C.c_size_t, [C.POINTER(nc_config), C.c_int]),
+    "nc_params_init": (C.c_int, [C.POINTER(nc_params), C.POINTER(nc_config)]),
+    "nc_forward": (C.c_int, [C.POINTER(nc_params), C.c_void_p, C.c_void_p, C.c_int, C.c_int,
+                             C.c_void_p, C.c_void_p, C.c_void_p]),
+    "nc_forward_host": (C.c_int, [C.POINTER(nc_params), C.c_void_p, C.c_void_p, C.c_int, C.c_int,
+                                  C.c_void_p, C.c_void_p]),
+    "nc_loss_mean": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
+    "nc_attention_workspace_bytes": (C.c_size_t, [C.c_int] * 7),
+    "nc_attention": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int,
+                               C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_float, C.c_float,
+                               C.c_float, C.c_float, C.c_int, C.c_void_p, C.c_size_t, C.c_void_p]),
+    "nc_get_status": (C.c_int, [C.c_void_p, C.POINTER(C.c_int)]),
+    "nc_status_string": (C.c_char_p, [C.c_int]),
+    "nc_last_error": (C.c_char_p, []),
+    "nc_last_launch_count": (C.c_int, []),
+    "nc_sizeof": (C.c_size_t, [C.c_int]),
+}
+
+
+def lib():
+    """Load libnc.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise NcError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m decoder_only_transformer_fwd_b200.build`")
+        h = C.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(h, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = h
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        err = lib().nc_last_error().decode()
+        raise NcError(f"{what}: {STATUS.get(rc, rc)} ({lib().nc_status_string(rc).decode()}) {err}")
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return C.c_void_p(s.cuda_stream)
+
+
+# --------------------------------------------------------------------------
+# the C calls, same names
+# --------------------------------------------------------------------------
+
+def nc_init_config(depth: int, max_T: int, dtype: str = "bf16", window_pattern: str = "SSSL",
+                   short_window: int | None = None, backout_layer: int = -1) -> nc_config:
+    cfg = nc_config()
+    dt = NC_BF16 if dtype == "bf16" else NC_FP32
+    sw = max_T // 2 if short_window is None else short_window
+    _check(lib().nc_init_config(C.byref(cfg), depth, max_T, dt, window_pattern.encode(), sw,
+                                backout_layer), "nc_init_config")
+    return cfg
+
+
+def nc_workspace_bytes(cfg: nc_config, max_tokens: int) -> int:
+    return int(lib().nc_workspace_bytes(C.byref(cfg), max_tokens))
+
+
+def nc_forward(params: nc_params, tokens, targets, out_loss, out_logits=None, stream=None):
+    B, T = tokens.shape
+    _check(lib().nc_forward(C.byref(params), _ptr(tokens), _ptr(targets), B, T, _ptr(out_loss),
+                            _ptr(out_logits), _stream(stream)), "nc_forward")
+
+
+def nc_forward_host(params: nc_params, tokens: np.ndarray, targets: np.ndarray, out_loss: np.ndarray,
+                    stream=None):
+    """tokens/targets/out_loss are host arrays (pinned torch tensors or numpy)."""
+    B, T = tokens.shape
+    ptr = lambda a: C.c_void_p(a.data_ptr() if hasattr(a, "data_ptr") else a.ctypes.data)
+    _check(lib().nc_forward_host(C.byref(params), ptr(tokens), ptr(targets), B, T, ptr(out_loss),
+                                 _stream(stream)), "nc_forward_host")
+
+
+def nc_loss_mean(loss, targets, out_mean, stream=None):
+    _check(lib().nc_loss_mean(_ptr(loss), _ptr(targets), loss.numel(), _ptr(out_mean),
+                              _stream(stream)), "nc_loss_mean")
+
+
+def nc_attention_workspace_bytes(B, T, H, Hkv, D, dtype="bf16", rope_qknorm=1) -> int:
+    dt = NC_BF16 if dtype == "bf16" else NC_FP32
+    return int(lib().nc_attention_workspace_bytes(B, T, H, Hkv, D, dt, rope_qknorm))
+
+
+def nc_attention(q, k, v, out, window: int, rope_qknorm: int = 1, alpha: float = 1.15,
+                 softmax_scale: float | None = None, rope_base: float = 100000.0, eps: float = 1e-6,
+                 workspace=None, stream=None):
+    import torch
+    B, T, H, D = q.shape
+    Hkv = k.shape[2]
+    dt = NC_BF16 if q.dtype == torch.bfloat16 else NC_FP32
+    scale = D ** -0.5 if softmax_scale is None else softmax_scale
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().nc_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, T, H, Hkv, D, window,
+                              rope_qknorm, alpha, scale, rope_base, eps, dt, _ptr(workspace),
+                              nbytes, _stream(stream)), "nc_attention")
+
+
+def nc_get_status(stream=None) -> tuple[int, int]:
+    bits = C.c_int(0)
+    rc = lib().nc_get_status(_stream(stream), C.byref(bits))
+    return rc, bits.value
+
+
+def nc_last_launch_count() -> int:
+    return int(lib().nc_last_launch_count())
+
+
+# --------------------------------------------------------------------------
+# parameter marshalling (allocation through torch)
+# --------------------------------------------------------------------------
+
+class NcModel:
+    """Device copies of a parameter set (as produced by `synth.params`) plus a
+    workspace, and the nc_params struct pointing at them."""
+
+    def __init__(self, cfg: nc_config, host_params: dict, max_tokens: int, device="cuda"):
+        import torch
+        self.cfg = cfg
+        self.device = torch.device(device)
+        act = torch.bfloat16 if cfg.dtype == NC_BF16 else torch.float32
+        keep = []
+
+        def dev(a, dtype=act):
+            t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(self.device).to(dtype)
+            keep.append(t)
+            return t
+
+        p = nc_params()
+        _check(lib().nc_params_init(C.byref(p), C.byref(cfg)), "nc_params_init")
+        self.wte = dev(host_params["wte"])
+        self.lm_head = dev(host_params["lm_head"])
+        self.smear_gate = dev(host_params["smear_gate"], torch.float32)
+        self.resid_lambdas = dev(host_params["resid_lambdas"], torch.float32)
+        self.x0_lambdas = dev(host_params["x0_lambdas"], torch.float32)
+        p.wte, p.lm_head = self.wte.data_ptr(), self.lm_head.data_ptr()
+        p.smear_gate = self.smear_gate.data_ptr()
+        p.resid_lambdas, p.x0_lambdas = self.resid_lambdas.data_ptr(), self.x0_lambdas.data_ptr()
+        p.backout_lambda = float(host_params["backout_lambda"])
+        for l, lp in enumerate(host_params["layers"]):
+            if lp is None:
+                raise ValueError(f"layer {l} missing from the parameter set")
+            L = p.layer[l]
+            L.w_qkv = dev(lp["w_qkv"]).data_ptr()
+            L.w_o = dev(lp["w_o"]).data_ptr()
+            L.w_fc1 = dev(lp["w_fc1"]).data_ptr()
+            L.w_fc2 = dev(lp["w_fc2"]).data_ptr()
+            if lp.get("ve") is not None:
+                L.ve = dev(lp["ve"]).data_ptr()
+                L.ve_gate = dev(lp["ve_gate"], torch.float32).data_ptr()
+        nbytes = nc_workspace_bytes(cfg, max_tokens)
+        if nbytes == 0:
+            raise NcError("invalid configuration (nc_workspace_bytes returned 0)")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        p.workspace = self.workspace.data_ptr()
+        p.workspace_bytes = nbytes
+        p.max_tokens = max_tokens
+        self._keep = keep
+        self.params = p
+
+    def forward(self, tokens, targets, want_logits: bool = False, stream=None):
+        import torch
+        B, T = tokens.shape
+        loss = torch.empty(B * T, dtype=torch.float32, device=self.device)
+        logits = (torch.empty(B * T, self.cfg.vocab, dtype=torch.float32, device=self.device)
+                  if want_logits else None)
+        nc_forward(self.params, tokens, targets, loss, logits, stream)
+        return loss, logits

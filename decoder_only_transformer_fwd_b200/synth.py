@@ -122,3 +122,15 @@ def attention_inputs(seed: int, B: int, T: int, H: int, D: int, Hkv: int | None 
     k = rnd(normal(seed, _ID_K, (B, T, Hkv, D), 1.0))
     v = rnd(normal(seed, _ID_V, (B, T, Hkv, D), 1.0))
     return q, k, v
+
+
+# Workload shapes (model depth, batch, sequence length, short window, dtype).
+# Workload i draws its inputs from seed SEED_BASE + i.
+WORKLOADS = {
+    "d1": dict(index=0, depth=1, B=1, T=256, short=256, dtype="fp32"),
+    "d4": dict(index=1, depth=4, B=4, T=1024, short=512, dtype="bf16"),
+    "d12": dict(index=2, depth=12, B=8, T=2048, short=1024, dtype="bf16"),
+    "d24": dict(index=3, depth=24, B=4, T=2048, short=1024, dtype="bf16"),
+}
+# single attention layer sweep: 12 heads x 128, batch 8, T x window
+ATTN_SWEEP = dict(index=4, H=12, D=128, B=8, cases=[(2048, 1024), (2048, 0), (8192, 1024), (8192, 0)])

@@ -1,0 +1,186 @@
+/*
+ * nc.h -- C ABI of libnc.so: the nanochat GPT forward pass, from token ids to
+ * per-token softcapped cross-entropy, on one B200 (sm_100a).
+ *
+ * The operation is the forward pass of "The Mathematics of Karpathy's
+ * nanochat" (§High-Level Forward Pass and the sections it links), extended by
+ * the smear gate and backout of the "nanochat depth sweep" model card
+ * (Architecture list) and "Reading nanochat Source" (§5, Forward pass, shape
+ * by shape).
+ *
+ * Conventions for every call:
+ *  - Pointers are DEVICE pointers unless the argument says "host".
+ *  - The library never allocates and never frees device memory: parameters
+ *    are borrowed, scratch comes from a caller-provided workspace.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream) unless stated otherwise.
+ *  - Arguments are validated on the host before any launch; a failed check
+ *    returns a non-zero nc_status and launches nothing.  No call throws,
+ *    exits or traps.
+ *  - Data errors found on the device (token or target id out of range, a
+ *    bounded wait that ran out) are clamped or skipped so that every access
+ *    stays in bounds, and are recorded in a device status word that
+ *    nc_get_status() returns.
+ *  - Calls are thread-compatible: concurrent calls must not share a
+ *    workspace.
+ */
+#ifndef NC_H_
+#define NC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define NC_MAX_LAYERS 64
+
+typedef enum {
+  NC_OK = 0,
+  NC_ERR_ARG = 1,        /* null pointer or invalid scalar argument          */
+  NC_ERR_SHAPE = 2,      /* unsupported or inconsistent sizes                */
+  NC_ERR_ALIGN = 3,      /* pointer or stride not 16-byte aligned            */
+  NC_ERR_CUDA = 4,       /* a CUDA runtime call failed (see nc_last_error)   */
+  NC_ERR_DATA = 5,       /* device-side: token/target id out of range        */
+  NC_ERR_TIMEOUT = 6,    /* device-side: a bounded wait inside a kernel ran out */
+  NC_ERR_WORKSPACE = 7   /* workspace missing or smaller than required       */
+} nc_status;
+
+typedef enum { NC_BF16 = 0, NC_FP32 = 1 } nc_dtype;
+
+/* Model configuration.  Filled by nc_init_config(); every field may be
+ * overridden by the caller before use. */
+typedef struct nc_config {
+  int n_layer;            /* L, the depth                                       */
+  int n_embd;             /* C = ceil(64 L / 128) * 128 ([Math] §Architecture Overview) */
+  int n_head;             /* H = C / 128                                        */
+  int n_kv_head;          /* H_kv (= H; the kernels require H_kv == H)          */
+  int head_dim;           /* D = 128 (the kernels require 128)                  */
+  int vocab;              /* V = 32768                                          */
+  int vocab_padded;       /* V rounded up to a multiple of 64 ([Source] §5.4)   */
+  int mlp_hidden;         /* 4 C                                                */
+  int max_T;              /* sequence length the windows are derived from      */
+  int dtype;              /* nc_dtype: NC_BF16 (bf16 storage, fp32 accumulate) or NC_FP32 */
+  int window[NC_MAX_LAYERS];  /* per-layer window w: key j visible to query i iff j <= i and i - j < w */
+  int has_ve[NC_MAX_LAYERS];  /* value embedding on layer l iff l % 2 == (L - 1) % 2 */
+  int backout_layer;      /* block whose output is subtracted before the head; -1 = none */
+  int gate_channels;      /* 12: input channels of the VE and smear gates       */
+  int smear;              /* 1 = smear gate on                                  */
+  int gemm_impl;          /* 0 = tensor cores (tcgen05) in bf16 mode, 1 = CUDA-core GEMM */
+  int attn_impl;          /* 0 = tensor cores (tcgen05) in bf16 mode, 1 = CUDA-core attention */
+  float qk_alpha;         /* 1.15 ([Math] §QK-Norm with Sharpening)              */
+  float softmax_scale;    /* 1/sqrt(D)                                          */
+  float rope_base;        /* 100000                                             */
+  float eps;              /* 1e-6, inside every RMSNorm's square root           */
+  float softcap;          /* 15 ([Math] §Logit Softcap)                          */
+  float ve_gate_scale;    /* 3 ([Math] §Value Embeddings)                        */
+} nc_config;
+
+/* Parameters of one block.  Matrices use the nn.Linear [out, in] row-major
+ * layout (y = x W^T) in the config's dtype (bf16 or fp32). */
+typedef struct nc_layer_params {
+  const void* w_qkv;      /* [(H + 2 H_kv) D, C]: rows of W_Q, then W_K, then W_V */
+  const void* w_o;        /* [C, H D]                                           */
+  const void* w_fc1;      /* [4C, C]                                            */
+  const void* w_fc2;      /* [C, 4C]                                            */
+  const void* ve;         /* [V, H_kv D] value-embedding table, or NULL when has_ve == 0 */
+  const float* ve_gate;   /* [H_kv, gate_channels] fp32, or NULL when has_ve == 0 */
+} nc_layer_params;
+
+typedef struct nc_params {
+  nc_config cfg;
+  const void* wte;            /* [V, C] token embedding                         */
+  const void* lm_head;        /* [V_pad, C] untied head                         */
+  const float* smear_gate;    /* [gate_channels] fp32                           */
+  const float* resid_lambdas; /* [L] fp32, lambda_l                              */
+  const float* x0_lambdas;    /* [L] fp32, mu_l                                  */
+  float backout_lambda;       /* beta (host scalar)                             */
+  nc_layer_params layer[NC_MAX_LAYERS];
+  void* workspace;            /* device scratch of >= nc_workspace_bytes(cfg, max_tokens) */
+  size_t workspace_bytes;
+  int max_tokens;             /* B*T capacity the workspace was sized for       */
+} nc_params;
+
+/* Fill `cfg` (host out) for a model of depth `depth`, following [Math]
+ * §Architecture Overview and §Sliding Window Pattern: the pattern string
+ * ("SSSL", "L", ...) is tiled over the layers, 'L' -> window max_T, 'S' ->
+ * short_window, and the last layer is always max_T.  backout_layer < 0 picks
+ * L/2.  Pure host function.  Returns NC_ERR_ARG on a null pointer, a
+ * non-positive size, a depth above NC_MAX_LAYERS or a pattern with characters
+ * other than 'S'/'L'. */
+int nc_init_config(nc_config* cfg, int depth, int max_T, int dtype, const char* window_pattern,
+                   int short_window, int backout_layer);
+
+/* Bytes of workspace nc_forward() needs for up to `max_tokens` = B*T tokens
+ * (256-byte aligned sub-buffers).  Host function; 0 on invalid config. */
+size_t nc_workspace_bytes(const nc_config* cfg, int max_tokens);
+
+/* Zero `p` (host) and copy `cfg` into it.  The caller then sets the pointers. */
+int nc_params_init(nc_params* p, const nc_config* cfg);
+
+/* Forward pass ([Math] §High-Level Forward Pass, §Cross-Entropy Loss).
+ *   tokens   [B, T] int32, ids in [0, V)
+ *   targets  [B, T] int32, ids in [0, V) or -1 (= ignored)
+ *   out_loss [B*T] fp32 per-token loss: logsumexp(zhat_t) - zhat_t[y_t], 0 where y_t == -1
+ *   out_logits_opt [B*T, V] fp32 softcapped logits 15 tanh(z/15), or NULL
+ *     (when NULL the logits are never written to memory in bf16 mode).
+ * Requires B*T <= p->max_tokens, T <= cfg.max_T, C % 128 == 0, D == 128,
+ * H_kv == H, all pointers 16-byte aligned. */
+int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets, int B, int T,
+               float* out_loss, float* out_logits_opt, void* stream);
+
+/* The same pass from HOST buffers: copies h_tokens/h_targets ([B, T] int32,
+ * host) into the workspace, runs nc_forward() and copies the per-token loss
+ * back into h_out_loss ([B*T] fp32, host).  Synchronous: returns after the
+ * loss is on the host.  Pinned host memory gives asynchronous-capable copies. */
+int nc_forward_host(const nc_params* p, const int32_t* h_tokens, const int32_t* h_targets, int B,
+                    int T, float* h_out_loss, void* stream);
+
+/* Mean of loss[i] over i with targets[i] != -1 ([Math] §Cross-Entropy Loss),
+ * written to *out_mean (device fp32); NaN when no target is valid.  n >= 0. */
+int nc_loss_mean(const float* loss, const int32_t* targets, int n, float* out_mean, void* stream);
+
+/* Workspace bytes nc_attention() needs (0 when rope_qknorm == 0). */
+size_t nc_attention_workspace_bytes(int B, int T, int H, int Hkv, int D, int dtype, int rope_qknorm);
+
+/* One attention layer ([Math] §QK-Norm with Sharpening, §Scaled Dot-Product
+ * Attention with Sliding Window):
+ *   q [B, T, H, D], k and v [B, T, H_kv, D] contiguous, in `dtype`;
+ *   out [B, T, H, D] in `dtype`.
+ *   With rope_qknorm = 1, q and k first get RoPE (base rope_base, position t
+ *   within the row) and qhat = alpha * RMSNorm_D(RoPE(q)) (likewise k), written
+ *   to the workspace; with 0 they are used as given.
+ *   o_i = sum_j softmax_j(softmax_scale * qhat_i . khat_j) v_j over j <= i,
+ *   i - j < window; window <= 0 or >= T means plain causal.
+ * Requires D == 128, H_kv == H, 16-byte aligned pointers. */
+int nc_attention(const void* q, const void* k, const void* v, void* out, int B, int T, int H,
+                 int Hkv, int D, int window, int rope_qknorm, float alpha, float softmax_scale,
+                 float rope_base, float eps, int dtype, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
+/* Synchronise `stream`, read the device status word (an OR of
+ * 1 << NC_ERR_DATA and 1 << NC_ERR_TIMEOUT bits set by kernels since the last
+ * read), clear it, and return NC_OK, NC_ERR_DATA or NC_ERR_TIMEOUT (timeout
+ * wins).  *out_bits (host, may be NULL) receives the raw bits. */
+int nc_get_status(void* stream, int* out_bits);
+
+/* Static description of a status code. */
+const char* nc_status_string(int status);
+
+/* Text of the last CUDA error seen by this thread (empty if none). */
+const char* nc_last_error(void);
+
+/* Number of kernel launches issued by the last nc_forward() / nc_attention()
+ * on this thread. */
+int nc_last_launch_count(void);
+
+/* sizeof of the ABI structs, for bindings to check their mirrors:
+ * which = 0 -> nc_config, 1 -> nc_layer_params, 2 -> nc_params; 0 otherwise. */
+size_t nc_sizeof(int which);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NC_H_ */

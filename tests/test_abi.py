@@ -1,0 +1,145 @@
+"""The C ABI without a GPU: the library loads, exports every symbol declared in
+include/nc.h, its struct layouts match the ctypes mirrors, and the host-side
+logic (configuration, workspace sizing, argument checks) behaves as declared.
+No test here launches a kernel."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from decoder_only_transformer_fwd_b200 import nc
+from oracle import nanochat_fwd as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "nc.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(nc_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = nc.lib()
+    names = _declared_functions()
+    assert "nc_forward" in names and "nc_attention" in names and "nc_init_config" in names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_struct_sizes_match_mirrors():
+    lib = nc.lib()
+    assert lib.nc_sizeof(0) == C.sizeof(nc.nc_config)
+    assert lib.nc_sizeof(1) == C.sizeof(nc.nc_layer_params)
+    assert lib.nc_sizeof(2) == C.sizeof(nc.nc_params)
+    assert lib.nc_sizeof(9) == 0
+
+
+@pytest.mark.parametrize("depth,T,short", [(1, 256, 256), (4, 1024, 512), (12, 2048, 1024),
+                                           (24, 2048, 1024), (7, 333, 100)])
+def test_init_config_matches_pages(depth, T, short):
+    cfg = nc.nc_init_config(depth, T, "bf16", "SSSL", short, -1)
+    ref = O.make_config(depth, T, short)
+    assert (cfg.n_layer, cfg.n_embd, cfg.n_head, cfg.n_kv_head, cfg.head_dim) == (
+        ref["n_layer"], ref["n_embd"], ref["n_head"], ref["n_kv_head"], ref["head_dim"])
+    assert cfg.vocab == ref["vocab"] and cfg.vocab_padded == ref["vocab_padded"]
+    assert cfg.mlp_hidden == 4 * ref["n_embd"]
+    assert list(cfg.window[:depth]) == ref["windows"]
+    assert [l for l in range(depth) if cfg.has_ve[l]] == ref["ve_layers"]
+    assert cfg.backout_layer == ref["backout_layer"]
+    assert cfg.gate_channels == ref["gate_channels"] and cfg.smear == 1
+    assert abs(cfg.qk_alpha - ref["qk_alpha"]) < 1e-7
+    assert abs(cfg.softmax_scale - ref["softmax_scale"]) < 1e-7
+    assert cfg.rope_base == ref["rope_base"] and abs(cfg.eps - ref["eps"]) < 1e-12
+    assert cfg.softcap == ref["softcap"] and cfg.ve_gate_scale == ref["ve_gate_scale"]
+
+
+def test_init_config_rejects_bad_arguments():
+    lib = nc.lib()
+    cfg = nc.nc_config()
+    assert lib.nc_init_config(None, 4, 1024, 0, b"SSSL", 512, -1) == 1
+    assert lib.nc_init_config(C.byref(cfg), 0, 1024, 0, b"SSSL", 512, -1) == 1
+    assert lib.nc_init_config(C.byref(cfg), 65, 1024, 0, b"SSSL", 512, -1) == 1
+    assert lib.nc_init_config(C.byref(cfg), 4, 1024, 7, b"SSSL", 512, -1) == 1
+    assert lib.nc_init_config(C.byref(cfg), 4, 1024, 0, b"SSXL", 512, -1) == 1
+    assert lib.nc_init_config(C.byref(cfg), 4, 1024, 0, b"", 512, -1) == 1
+    assert lib.nc_init_config(C.byref(cfg), 4, 1024, 0, b"SSSL", 512, 4) == 1
+    assert lib.nc_init_config(C.byref(cfg), 4, 1024, 0, b"L", 512, 1) == 0
+    assert list(cfg.window[:4]) == [1024] * 4 and cfg.backout_layer == 1
+
+
+def test_workspace_bytes():
+    cfg = nc.nc_init_config(24, 2048, "bf16", "SSSL", 1024)
+    w1 = nc.nc_workspace_bytes(cfg, 8192)
+    w2 = nc.nc_workspace_bytes(cfg, 4096)
+    assert w1 > w2 > 0 and w1 % 256 == 0
+    # residual stream x, x0, x_bo in fp32 plus bf16 activations: at least this much
+    C_ = cfg.n_embd
+    assert w1 >= 8192 * C_ * (3 * 4 + 2 * (1 + 3 + 1 + 4))
+    # bf16 mode never materialises the logits; fp32 mode may
+    cfg32 = nc.nc_init_config(24, 2048, "fp32", "SSSL", 1024)
+    assert nc.nc_workspace_bytes(cfg32, 8192) > w1 + 8192 * 32768 * 4
+    cfg.n_kv_head = 6            # unsupported: H_kv != H
+    assert nc.nc_workspace_bytes(cfg, 8192) == 0
+
+
+def test_forward_rejects_bad_arguments_without_launching():
+    lib = nc.lib()
+    cfg = nc.nc_init_config(1, 256, "fp32", "L", 256)
+    p = nc.nc_params()
+    assert lib.nc_params_init(C.byref(p), C.byref(cfg)) == 0
+    buf = (C.c_byte * 4096)()
+    addr = C.addressof(buf)
+    a16 = C.c_void_p((addr + 15) & ~15)
+    # null pointers
+    assert lib.nc_forward(C.byref(p), None, a16, 1, 8, a16, None, None) == nc.STATUS_CODES["NC_ERR_ARG"]
+    # shape beyond capacity (max_tokens == 0)
+    assert lib.nc_forward(C.byref(p), a16, a16, 1, 8, a16, None, None) == nc.STATUS_CODES["NC_ERR_SHAPE"]
+    p.max_tokens = 8
+    assert lib.nc_forward(C.byref(p), a16, a16, 1, 300, a16, None, None) == nc.STATUS_CODES["NC_ERR_SHAPE"]
+    # missing parameters
+    assert lib.nc_forward(C.byref(p), a16, a16, 1, 8, a16, None, None) == nc.STATUS_CODES["NC_ERR_ARG"]
+    # misaligned pointers
+    for name in ("wte", "lm_head", "smear_gate", "resid_lambdas", "x0_lambdas"):
+        setattr(p, name, a16.value)
+    for l in range(1):
+        L = p.layer[l]
+        L.w_qkv = L.w_o = L.w_fc1 = L.w_fc2 = L.ve = L.ve_gate = a16.value
+    mis = C.c_void_p(a16.value + 4)
+    assert lib.nc_forward(C.byref(p), mis, a16, 1, 8, a16, None, None) == nc.STATUS_CODES["NC_ERR_ALIGN"]
+    # missing workspace
+    assert lib.nc_forward(C.byref(p), a16, a16, 1, 8, a16, None, None) == nc.STATUS_CODES["NC_ERR_WORKSPACE"]
+    # invalid config
+    p.cfg.head_dim = 64
+    assert lib.nc_forward(C.byref(p), a16, a16, 1, 8, a16, None, None) == nc.STATUS_CODES["NC_ERR_SHAPE"]
+
+
+def test_attention_rejects_bad_arguments():
+    lib = nc.lib()
+    buf = (C.c_byte * 4096)()
+    a16 = C.c_void_p((C.addressof(buf) + 15) & ~15)
+    args = lambda **kw: dict(dict(q=a16, k=a16, v=a16, o=a16, B=1, T=4, H=1, Hkv=1, D=128, w=0, rq=0,
+                                  dt=0, ws=None, wsb=0), **kw)
+
+    def call(a):
+        return lib.nc_attention(a["q"], a["k"], a["v"], a["o"], a["B"], a["T"], a["H"], a["Hkv"],
+                                a["D"], a["w"], a["rq"], 1.15, 0.088, 1e5, 1e-6, a["dt"], a["ws"],
+                                a["wsb"], None)
+    assert call(args(q=None)) == nc.STATUS_CODES["NC_ERR_ARG"]
+    assert call(args(D=64)) == nc.STATUS_CODES["NC_ERR_SHAPE"]
+    assert call(args(Hkv=2, H=4)) == nc.STATUS_CODES["NC_ERR_SHAPE"]
+    assert call(args(T=0)) == nc.STATUS_CODES["NC_ERR_SHAPE"]
+    assert call(args(dt=5)) == nc.STATUS_CODES["NC_ERR_ARG"]
+    assert call(args(k=C.c_void_p(a16.value + 2))) == nc.STATUS_CODES["NC_ERR_ALIGN"]
+    assert call(args(rq=1)) == nc.STATUS_CODES["NC_ERR_WORKSPACE"]
+    assert nc.nc_attention_workspace_bytes(2, 8, 4, 4, 128, "bf16", 1) >= 2 * 2 * 8 * 4 * 128 * 2
+    assert nc.nc_attention_workspace_bytes(2, 8, 4, 4, 128, "bf16", 0) == 0
+
+
+def test_status_strings():
+    lib = nc.lib()
+    for code in range(8):
+        assert lib.nc_status_string(code)
+    assert lib.nc_status_string(99) == b"unknown status"
+    assert lib.nc_loss_mean(None, None, 4, None, None) == nc.STATUS_CODES["NC_ERR_ARG"]
