@@ -1,0 +1,344 @@
+#!/usr/bin/env python
+"""Throughput of the nanochat d24 forward pass + softcapped cross-entropy on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one call of the whole forward pass (embedding + norm + smear, 24
+blocks, backout, head, softcap, per-token CE) over one batch of B = 4 rows of
+T = 2048 synthetic tokens (8192 tokens), through the C ABI.  Inputs are
+resident in HBM when the timed region starts.  The weights (1.46 GB of bf16
+matrices plus 0.33 GB of gathered embedding rows per step) are far larger
+than the 126 MB L2, so no flush is needed between steps.
+
+Prints one JSON line (rank 0).  With N > 1 (launched by torch.distributed.run)
+every rank runs an independent replica on its own 4 rows: the rows of a batch
+are independent sequences and the forward pass has no exchange step, so there
+is no data-path collective (weak scaling); the ranks only meet at the timing
+barriers and the max-over-ranks reduction of the elapsed time.
+
+--impl reference times the CPU oracle (fp64 numpy) on the host cores instead:
+each step is a bounded sample of the same workload (the first 256 positions
+of one row: by causality their losses equal those of the full row).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "d24"
+METRIC = "fwd+CE tokens/sec at d24 T=2048 on 1 B200; % of BF16 tensor peak"
+CPU_SAMPLE_TOKENS = 256
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def workload_desc(cfg, B, T):
+    return (f"d24 nanochat GPT forward+CE: depth {cfg.n_layer}, C={cfg.n_embd}, {cfg.n_head}x{cfg.head_dim} "
+            f"heads, MLP {cfg.mlp_hidden} ReLU^2, V={cfg.vocab}, SSSL windows "
+            f"{cfg.window[0]}/{cfg.max_T} (last block full), value embeddings on odd blocks, "
+            f"backout from block {cfg.backout_layer}, softcap {cfg.softcap:g}, B={B}, T={T}")
+
+
+def cpu_oracle_run(cfg_o, params, tok, tgt, ntok):
+    from oracle import nanochat_fwd as O
+    t0 = time.perf_counter()
+    O.forward(cfg_o, params, tok[:1, :ntok], tgt[:1, :ntok])
+    return time.perf_counter() - t0
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    import numpy as np  # noqa: F401
+    from decoder_only_transformer_fwd_b200 import synth
+    from oracle import nanochat_fwd as O
+    w = synth.WORKLOADS[WORKLOAD]
+    seed = synth.SEED_BASE + w["index"]
+    ocfg = O.make_config(w["depth"], w["T"], w["short"])
+    params = synth.params(seed, n_layer=ocfg["n_layer"], n_embd=ocfg["n_embd"], n_head=ocfg["n_head"],
+                          n_kv_head=ocfg["n_kv_head"], head_dim=ocfg["head_dim"], vocab=ocfg["vocab"],
+                          vocab_padded=ocfg["vocab_padded"], ve_layers=ocfg["ve_layers"], bf16=True)
+    tok = synth.tokens(seed, w["B"], w["T"], ocfg["vocab"])
+    tgt = synth.targets(seed, w["B"], w["T"], ocfg["vocab"])
+    for _ in range(args.warmup):
+        cpu_oracle_run(ocfg, params, tok, tgt, CPU_SAMPLE_TOKENS)
+    times = [cpu_oracle_run(ocfg, params, tok, tgt, CPU_SAMPLE_TOKENS) for _ in range(args.steps)]
+    total = sum(times)
+    value = CPU_SAMPLE_TOKENS * args.steps / total
+    sample = (f"first {CPU_SAMPLE_TOKENS} positions of row 0 of the d24 batch per step "
+              f"(causal prefix: exact per-token losses), fp64 numpy oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "d24 nanochat GPT forward+CE (CPU oracle, bounded sample)",
+                   "tokens_per_step": CPU_SAMPLE_TOKENS, "seq_len": w["T"]},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    from decoder_only_transformer_fwd_b200 import flops, nc, synth
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = synth.WORKLOADS[WORKLOAD]
+    B, T = (args.rows or w["B"]), w["T"]
+    M = B * T
+    seed = synth.SEED_BASE + w["index"]
+    cfg = nc.nc_init_config(w["depth"], T, "bf16", "SSSL", w["short"], -1)
+    ve_layers = [l for l in range(cfg.n_layer) if cfg.has_ve[l]]
+    params = synth.params(seed, n_layer=cfg.n_layer, n_embd=cfg.n_embd, n_head=cfg.n_head,
+                          n_kv_head=cfg.n_kv_head, head_dim=cfg.head_dim, vocab=cfg.vocab,
+                          vocab_padded=cfg.vocab_padded, ve_layers=ve_layers, bf16=True)
+    # each rank processes its own batch of B rows (rank-dependent tokens)
+    tok_h = synth.tokens(seed + 1000 * rank, B, T, cfg.vocab)
+    tgt_h = synth.targets(seed + 1000 * rank, B, T, cfg.vocab)
+    model = nc.NcModel(cfg, params, M, device=dev)
+    tok = torch.from_numpy(tok_h).to(dev)
+    tgt = torch.from_numpy(tgt_h).to(dev)
+    loss = torch.empty(M, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        nc.nc_forward(model.params, tok, tgt, loss, None, stream)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    launches_per_step = nc.nc_last_launch_count()
+    rc, bits = nc.nc_get_status(stream)
+    if rc != 0:
+        raise RuntimeError(f"device status after warm-up: {nc.STATUS.get(rc)} bits={bits}")
+
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [x.strip() for x in vis.split(",") if x.strip()]
+    clocks = ClockSampler(ids[local] if local < len(ids) else local)
+    clocks.start()
+    time.sleep(0.3)
+
+    # ---- timed region A: the whole step, device time, max over ranks ----
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_total = max_over_ranks(e0.elapsed_time(e1))
+
+    # ---- timed region B: the same steps with per-launch events on the GEMM kernel ----
+    gemm_per_step = 4 * cfg.n_layer + 1
+    timer = nc.LaunchTimer(gemm_per_step * args.steps, kinds=["gemm_tcgen05"])
+    barrier()
+    torch.cuda.synchronize()
+    with timer:
+        for _ in range(args.steps):
+            step()
+    torch.cuda.synchronize()
+    per_kind = timer.per_kind()
+
+    # ---- e2e: the host-buffer entry point, copies inside the timed region ----
+    h_tok = torch.from_numpy(tok_h).pin_memory()
+    h_tgt = torch.from_numpy(tgt_h).pin_memory()
+    h_loss = torch.empty(M, dtype=torch.float32).pin_memory()
+    nc.nc_forward_host(model.params, h_tok, h_tgt, h_loss, stream)
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        nc.nc_forward_host(model.params, h_tok, h_tgt, h_loss, stream)
+    e2e_s = max_over_ranks(time.perf_counter() - t0)
+    clk = clocks.stop()
+    rc, bits = nc.nc_get_status(stream)
+    if rc != 0:
+        raise RuntimeError(f"device status after the timed steps: {nc.STATUS.get(rc)} bits={bits}")
+    assert np.all(np.isfinite(h_loss.numpy()))
+
+    peaks, peak_src = load_peaks()
+    windows = list(cfg.window[:cfg.n_layer])
+    f_tok = flops.forward_flops_per_token(cfg.n_layer, cfg.n_embd, cfg.vocab, windows, T)
+    ms_step = ms_total / args.steps
+    tokens_all = M * world
+    value = tokens_all * args.steps / (ms_total / 1e3)
+    tflops = f_tok * M / (ms_step / 1e3) / 1e12
+
+    gemm_flops_step = flops.gemm_flops_per_token(cfg.n_layer, cfg.n_embd, cfg.vocab) * M
+    n_gemm, gemm_ms = per_kind.get("gemm_tcgen05", (0, 0.0))
+    achieved = (gemm_flops_step * args.steps) / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
+    roofline = {
+        "kernel": "gemm_tcgen05 (k_gemm_tc: QKV, O, FC1, FC2, head+CE)",
+        "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
+        "peak_kind": f"bf16 dense, sustained ({peak_src})", "unit": "TFLOP/s",
+        "frac": (achieved / peaks["bf16_tflops_sustained"]) if achieved else None,
+        "traffic": None,
+        "launches": n_gemm, "avg_launch_us": 1e3 * gemm_ms / max(n_gemm, 1),
+        "share_of_step": gemm_ms / ms_total if ms_total > 0 else None,
+    }
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import nanochat_fwd as O
+        ocfg = O.make_config(w["depth"], T, w["short"])
+        ntok = args.cpu_tokens
+        dt = cpu_oracle_run(ocfg, params, tok_h, tgt_h, ntok)
+        cpu = {"value": ntok / dt, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+               "sample": f"first {ntok} positions of row 0 (causal prefix: exact per-token losses), "
+                         f"fp64 numpy oracle, {dt:.1f} s"}
+
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": workload_desc(cfg, B, T), "global_batch": B * world, "seq_len": T,
+                       "tokens_per_step": tokens_all,
+                       "parallelism": f"replicas x{world} (independent rows, no collective)",
+                       "l2": "inputs larger than L2 (1.46 GB bf16 weights + 0.33 GB gathered rows per step)",
+                       "seed": seed},
+            "tflops": tflops, "pct_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
+            "pct_bf16_peak_sustained": 100.0 * tflops / peaks["bf16_tflops_sustained"],
+            "flops_per_token": f_tok,
+            "clocks": clk,
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": {"value": tokens_all * args.steps / e2e_s, "unit": "tokens/s",
+                    "h2d_bytes_per_step": 2 * M * 4, "d2h_bytes_per_step": M * 4},
+            "gpu_launches": launches_per_step * args.steps,
+            "kernel_ms_per_step": {k: v[1] / args.steps for k, v in per_kind.items()},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tokens", type=int, default=1024)
+    ap.add_argument("--rows", type=int, default=0, help="rows per step (default: the workload's B = 4)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

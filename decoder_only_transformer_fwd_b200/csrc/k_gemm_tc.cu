@@ -400,6 +400,7 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
   a.num_tiles = a.tiles_m * a.tiles_n;
   a.status = status;
   const int grid = a.num_tiles < num_sms ? a.num_tiles : num_sms;
+  LaunchScope scope_(KK_GEMM_TC, st);
   if (BN == 256) {
     set_smem_attr<256>();
     k_gemm_tc<256><<<grid, 192, TcCfg<256>::SMEM, st>>>(ta, tb, a, ep);
@@ -407,7 +408,6 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
     set_smem_attr<128>();
     k_gemm_tc<128><<<grid, 192, TcCfg<128>::SMEM, st>>>(ta, tb, a, ep);
   }
-  count_launch();
   return true;
 }
 

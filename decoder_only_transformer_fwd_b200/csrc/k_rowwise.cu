@@ -318,6 +318,7 @@ __global__ void k_loss_mean(const float* loss, const int32_t* targets, int n, fl
 void launch_embed(const void* wte, const int32_t* tokens, const float* smear_gate, int smear,
                   int gate_channels, const float* lam0, const float* mu0, float eps, int B, int T, int C, int V,
                   int act_bf16, float* x, float* x0, int* status, cudaStream_t st) {
+  LaunchScope scope_(KK_EMBED, st);
   const int M = B * T;
   const size_t sh = (size_t)(2 * C + 32) * sizeof(float);
   if (act_bf16)
@@ -326,12 +327,12 @@ void launch_embed(const void* wte, const int32_t* tokens, const float* smear_gat
   else
     k_embed<float><<<M, 256, sh, st>>>((const float*)wte, tokens, smear_gate, smear, gate_channels,
                                        lam0, mu0, eps, T, C, V, x, x0, status);
-  count_launch();
 }
 
 void launch_rmsnorm(const float* x, void* xn, int M, int C, float eps, int act_bf16,
                     const float* ve_gate, int Hkv, int gate_channels, float gate_scale, float* gate_out,
                     cudaStream_t st) {
+  LaunchScope scope_(KK_RMSNORM, st);
   const int warps = 8;
   const int grid = (M + warps - 1) / warps;
   if (act_bf16)
@@ -340,19 +341,19 @@ void launch_rmsnorm(const float* x, void* xn, int M, int C, float eps, int act_b
   else
     k_rmsnorm<float><<<grid, warps * 32, 0, st>>>(x, (float*)xn, M, C, eps, ve_gate, Hkv,
                                                   gate_channels, gate_scale, gate_out);
-  count_launch();
 }
 
 void launch_rope_table(float* cos_t, float* sin_t, int T, int D, float base, cudaStream_t st) {
+  LaunchScope scope_(KK_ROPE_TABLE, st);
   const int n = T * (D / 2);
   k_rope_table<<<(n + 255) / 256, 256, 0, st>>>(cos_t, sin_t, T, D, (double)base);
-  count_launch();
 }
 
 void launch_rope_qknorm_ve(void* qkv, int ld, int B, int T, int H, int Hkv, int D,
                            const float* cos_t, const float* sin_t, float alpha, float eps,
                            const int32_t* tokens, const void* ve, const float* gate, int V,
                            int act_bf16, int* status, cudaStream_t st) {
+  LaunchScope scope_(KK_ROPE_QKNORM, st);
   (void)status;
   const int M = B * T;
   const int slots = H + Hkv + (ve != nullptr ? Hkv : 0);
@@ -365,12 +366,12 @@ void launch_rope_qknorm_ve(void* qkv, int ld, int B, int T, int H, int Hkv, int 
   else
     k_rope_qknorm_ve<float><<<grid, wpb * 32, 0, st>>>((float*)qkv, ld, T, H, Hkv, D, cos_t, sin_t,
                                                        alpha, eps, tokens, (const float*)ve, gate, V, M);
-  count_launch();
 }
 
 void launch_rope_qknorm_copy(const void* q, const void* k, void* qo, void* ko, int B, int T, int H,
                              int Hkv, int D, const float* cos_t, const float* sin_t, float alpha,
                              float eps, int act_bf16, cudaStream_t st) {
+  LaunchScope scope_(KK_ROPE_QKNORM, st);
   const int M = B * T;
   const long long warps = (long long)M * (H + Hkv);
   const int wpb = 8;
@@ -383,26 +384,25 @@ void launch_rope_qknorm_copy(const void* q, const void* k, void* qo, void* ko, i
     k_rope_qknorm_copy<float><<<grid, wpb * 32, 0, st>>>((const float*)q, (const float*)k, (float*)qo,
                                                          (float*)ko, T, H, Hkv, D, cos_t, sin_t, alpha,
                                                          eps, M);
-  count_launch();
 }
 
 void launch_ce_rows(const float* logits, int ldl, const int32_t* targets, int M, int V, float* loss,
                     int* status, cudaStream_t st) {
+  LaunchScope scope_(KK_CE_ROWS, st);
   k_ce_rows<<<M, 256, 0, st>>>(logits, ldl, targets, V, loss, status);
-  count_launch();
 }
 
 void launch_ce_combine(const float* ce_sum, const float* ce_tgt, int n_tiles, float offset,
                        const int32_t* targets, int M, int V, float* loss, int* status, cudaStream_t st) {
+  LaunchScope scope_(KK_CE_COMBINE, st);
   const int wpb = 8;
   k_ce_combine<<<(M + wpb - 1) / wpb, wpb * 32, 0, st>>>(ce_sum, ce_tgt, n_tiles, offset, targets, M, V,
                                                          loss, status);
-  count_launch();
 }
 
 void launch_loss_mean(const float* loss, const int32_t* targets, int n, float* out, cudaStream_t st) {
+  LaunchScope scope_(KK_LOSS_MEAN, st);
   k_loss_mean<<<1, 1024, 0, st>>>(loss, targets, n, out);
-  count_launch();
 }
 
 }  // namespace nc

@@ -178,17 +178,18 @@ __global__ void __launch_bounds__(256) k_attn_simt(const T* __restrict__ q, cons
 
 void launch_gemm_simt(const void* A, int lda, const void* Bm, int ldb, int M, int N, int K,
                       int act_bf16, const EpiParams& ep, cudaStream_t st) {
+  LaunchScope scope_(KK_GEMM_SIMT, st);
   dim3 grid((N + 63) / 64, (M + 63) / 64);
   if (act_bf16)
     k_gemm_simt<bf16><<<grid, 256, 0, st>>>((const bf16*)A, lda, (const bf16*)Bm, ldb, M, N, K, ep);
   else
     k_gemm_simt<float><<<grid, 256, 0, st>>>((const float*)A, lda, (const float*)Bm, ldb, M, N, K, ep);
-  count_launch();
 }
 
 void launch_attn_simt(const void* q, const void* k, const void* v, int ldq, int ldk, int ldv,
                       void* o, int ldo, int B, int T, int H, int Hkv, int window, float scale,
                       int act_bf16, cudaStream_t st) {
+  LaunchScope scope_(KK_ATTN_SIMT, st);
   const size_t sh = (size_t)(2 * kAD * 65 + kAK * kAD + kAK * 65) * sizeof(float);
   dim3 grid((T + kAQ - 1) / kAQ, H, B);
   if (act_bf16) {
@@ -200,7 +201,6 @@ void launch_attn_simt(const void* q, const void* k, const void* v, int ldq, int 
     k_attn_simt<float><<<grid, 256, sh, st>>>((const float*)q, (const float*)k, (const float*)v, ldq,
                                               ldk, ldv, (float*)o, ldo, T, H, Hkv, window, scale);
   }
-  count_launch();
 }
 
 }  // namespace nc

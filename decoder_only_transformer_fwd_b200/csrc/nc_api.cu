@@ -22,7 +22,36 @@ namespace nc {
 static thread_local int t_launches = 0;
 static thread_local char t_err[256] = {0};
 
-void count_launch() { ++t_launches; }
+// optional per-launch timing (caller-owned events)
+struct Timing {
+  cudaEvent_t* events = nullptr;  // 2 * cap
+  int* kinds = nullptr;           // cap
+  int cap = 0;
+  int n = 0;
+  unsigned mask = 0;
+  bool open = false;
+};
+static thread_local Timing t_timing;
+
+void launch_begin(int kind, cudaStream_t st) {
+  Timing& t = t_timing;
+  t.open = false;
+  if (t.events != nullptr && ((t.mask >> kind) & 1u) && t.n < t.cap) {
+    cudaEventRecord(t.events[2 * t.n], st);
+    t.open = true;
+  }
+}
+
+void launch_end(int kind, cudaStream_t st) {
+  ++t_launches;
+  Timing& t = t_timing;
+  if (t.open) {
+    cudaEventRecord(t.events[2 * t.n + 1], st);
+    t.kinds[t.n] = kind;
+    ++t.n;
+    t.open = false;
+  }
+}
 
 static void set_err(const char* where, cudaError_t e) {
   snprintf(t_err, sizeof(t_err), "%s: %s", where, cudaGetErrorString(e));
@@ -456,6 +485,25 @@ const char* nc_status_string(int s) {
 const char* nc_last_error(void) { return t_err; }
 
 int nc_last_launch_count(void) { return t_launches; }
+
+int nc_set_launch_timing(void** events, int* kinds, int capacity, unsigned kind_mask) {
+  if (events != nullptr && (kinds == nullptr || capacity <= 0)) return NC_ERR_ARG;
+  t_timing = Timing();
+  t_timing.events = reinterpret_cast<cudaEvent_t*>(events);
+  t_timing.kinds = kinds;
+  t_timing.cap = events ? capacity : 0;
+  t_timing.mask = kind_mask;
+  return NC_OK;
+}
+
+int nc_launch_timing_count(void) { return t_timing.n; }
+
+const char* nc_kernel_name(int kind) {
+  static const char* names[KK_COUNT] = {
+      "embed_norm_smear", "rmsnorm", "rope_table", "rope_qknorm", "gemm_tcgen05", "gemm_cuda_core",
+      "attention_tcgen05", "attention_cuda_core", "ce_combine", "ce_rows", "loss_mean"};
+  return (kind >= 0 && kind < KK_COUNT) ? names[kind] : "unknown";
+}
 
 size_t nc_sizeof(int which) {
   switch (which) {

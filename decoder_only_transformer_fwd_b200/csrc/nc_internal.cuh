@@ -118,7 +118,21 @@ bool launch_attn_tc(const bf16* q, const bf16* k, const bf16* v, int ldq, int ld
                     int ldo, int B, int T, int H, int Hkv, int window, float scale, int* status,
                     int num_sms, cudaStream_t st);
 
-// launch counter (per host thread), incremented by every launcher
-void count_launch();
+// Kernel kinds, for the launch counter and the optional per-launch timing.
+enum KernelKind : int {
+  KK_EMBED = 0, KK_RMSNORM, KK_ROPE_TABLE, KK_ROPE_QKNORM, KK_GEMM_TC, KK_GEMM_SIMT, KK_ATTN_TC,
+  KK_ATTN_SIMT, KK_CE_COMBINE, KK_CE_ROWS, KK_LOSS_MEAN, KK_COUNT
+};
+// Every launcher holds one of these around its kernel launch: it counts the
+// launch (per host thread) and, when the caller enabled timing for this kind,
+// records a CUDA event before and after the launch on `st`.
+void launch_begin(int kind, cudaStream_t st);
+void launch_end(int kind, cudaStream_t st);
+struct LaunchScope {
+  int kind;
+  cudaStream_t st;
+  LaunchScope(int k, cudaStream_t s) : kind(k), st(s) { launch_begin(k, s); }
+  ~LaunchScope() { launch_end(kind, st); }
+};
 
 }  // namespace nc

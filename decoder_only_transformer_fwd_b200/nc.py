@@ -70,7 +70,55 @@ _SIGS = {
     "nc_last_error": (C.c_char_p, []),
     "nc_last_launch_count": (C.c_int, []),
     "nc_sizeof": (C.c_size_t, [C.c_int]),
+    "nc_set_launch_timing": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_uint]),
+    "nc_launch_timing_count": (C.c_int, []),
+    "nc_kernel_name": (C.c_char_p, [C.c_int]),
 }
+
+KERNEL_KINDS = ["embed_norm_smear", "rmsnorm", "rope_table", "rope_qknorm", "gemm_tcgen05",
+                "gemm_cuda_core", "attention_tcgen05", "attention_cuda_core", "ce_combine", "ce_rows",
+                "loss_mean"]
+
+
+class LaunchTimer:
+    """Per-launch CUDA-event timing of the library's kernels (nc_set_launch_timing).
+
+    Events are created through torch (the library allocates nothing); use as
+    a context manager around the calls to time, then read `per_kind()` after a
+    synchronize: {kind name: (launches, total ms)}."""
+
+    def __init__(self, capacity: int, kinds=None):
+        import torch
+        self.capacity = capacity
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * capacity)]
+        for e in self.events:          # materialise the cudaEvent_t handles
+            e.record()
+        self._handles = (C.c_void_p * (2 * capacity))(*[e.cuda_event for e in self.events])
+        self._kinds = (C.c_int * capacity)()
+        mask = 0
+        for k in (kinds or KERNEL_KINDS):
+            mask |= 1 << KERNEL_KINDS.index(k)
+        self.mask = mask
+        self.n = 0
+
+    def __enter__(self):
+        _check(lib().nc_set_launch_timing(C.cast(self._handles, C.c_void_p), C.cast(self._kinds, C.c_void_p),
+                                          self.capacity, self.mask), "nc_set_launch_timing")
+        return self
+
+    def __exit__(self, *exc):
+        self.n = int(lib().nc_launch_timing_count())
+        lib().nc_set_launch_timing(None, None, 0, 0)
+        return False
+
+    def per_kind(self) -> dict:
+        out = {}
+        for i in range(self.n):
+            name = KERNEL_KINDS[self._kinds[i]]
+            ms = self.events[2 * i].elapsed_time(self.events[2 * i + 1])
+            c, t = out.get(name, (0, 0.0))
+            out[name] = (c + 1, t + ms)
+        return out
 
 
 def lib():

@@ -19,6 +19,9 @@ rest.
 """
 from __future__ import annotations
 
+import concurrent.futures as _cf
+import os as _os
+
 import numpy as np
 
 SEED_BASE = 20260  # seed of workload i is SEED_BASE + i
@@ -45,12 +48,14 @@ def round_bf16(a: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bfloat16 (ties to even); the result
     is float32 holding bf16-representable values."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    r = ((u + 0x7FFF + lsb) >> 16) << 16
+    u = a.view(np.uint32)
+    # adding 0x7FFF + lsb carries into the upper half exactly when rounding up;
+    # no finite value overflows 32 bits (the largest is 0xFF7FFFFF)
+    r = (u + (np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1)))) & np.uint32(0xFFFF0000)
+    out = r.view(np.float32)
     nan = np.isnan(a)
-    out = r.astype(np.uint32).view(np.float32).copy()
-    out[nan] = np.float32("nan")
+    if nan.any():
+        out[nan] = np.float32("nan")
     return out.reshape(a.shape)
 
 
@@ -81,34 +86,45 @@ def params(seed: int, *, n_layer: int, n_embd: int, n_head: int, n_kv_head: int,
     """
     C, Hq, Hkv, D, V = n_embd, n_head, n_kv_head, head_dim, vocab
     ve_layers = set(int(l) for l in ve_layers)
-    rnd = round_bf16 if bf16 else (lambda a: a)
+    want = set(range(n_layer)) if layers is None else set(layers)
+    # (key, tensor id, shape, std, round to bf16); drawn in parallel threads
+    jobs = [("wte", _ID_WTE, (V, C), 1.0, bf16),
+            ("lm_head", _ID_HEAD, (vocab_padded, C), C ** -0.5, bf16),
+            ("smear_gate", _ID_SMEAR, (gate_channels,), gate_channels ** -0.5, False)]
+    nqkv = (Hq + 2 * Hkv) * D
+    for l in sorted(want):
+        b = _LAYER_BASE + 16 * l
+        jobs += [((l, "w_qkv"), b + 0, (nqkv, C), C ** -0.5, bf16),
+                 ((l, "w_o"), b + 1, (C, Hq * D), (Hq * D) ** -0.5, bf16),
+                 ((l, "w_fc1"), b + 2, (4 * C, C), C ** -0.5, bf16),
+                 ((l, "w_fc2"), b + 3, (C, 4 * C), (4 * C) ** -0.5, bf16)]
+        if l in ve_layers:
+            jobs += [((l, "ve"), b + 4, (V, Hkv * D), 1.0, bf16),
+                     ((l, "ve_gate"), b + 5, (Hkv, gate_channels), gate_channels ** -0.5, False)]
+
+    def draw(job):
+        key, tid, shape, std, rnd = job
+        a = normal(seed, tid, shape, std)
+        return key, (round_bf16(a) if rnd else a)
+
+    with _cf.ThreadPoolExecutor(max_workers=min(16, _os.cpu_count() or 4)) as ex:
+        drawn = dict(ex.map(draw, jobs))
     p = {
-        "wte": rnd(normal(seed, _ID_WTE, (V, C), 1.0)),
-        "lm_head": rnd(normal(seed, _ID_HEAD, (vocab_padded, C), C ** -0.5)),
-        "smear_gate": normal(seed, _ID_SMEAR, (gate_channels,), gate_channels ** -0.5),
+        "wte": drawn["wte"],
+        "lm_head": drawn["lm_head"],
+        "smear_gate": drawn["smear_gate"],
         "resid_lambdas": np.ones(n_layer, np.float32),
         "x0_lambdas": np.full(n_layer, 0.1, np.float32),
         "backout_lambda": np.float32(0.5),
         "layers": [],
     }
-    want = range(n_layer) if layers is None else set(layers)
     for l in range(n_layer):
         if l not in want:
             p["layers"].append(None)
             continue
-        b = _LAYER_BASE + 16 * l
-        nqkv = (Hq + 2 * Hkv) * D
-        lp = {
-            "w_qkv": rnd(normal(seed, b + 0, (nqkv, C), C ** -0.5)),
-            "w_o": rnd(normal(seed, b + 1, (C, Hq * D), (Hq * D) ** -0.5)),
-            "w_fc1": rnd(normal(seed, b + 2, (4 * C, C), C ** -0.5)),
-            "w_fc2": rnd(normal(seed, b + 3, (C, 4 * C), (4 * C) ** -0.5)),
-            "ve": None,
-            "ve_gate": None,
-        }
-        if l in ve_layers:
-            lp["ve"] = rnd(normal(seed, b + 4, (V, Hkv * D), 1.0))
-            lp["ve_gate"] = normal(seed, b + 5, (Hkv, gate_channels), gate_channels ** -0.5)
+        lp = {k: drawn[(l, k)] for k in ("w_qkv", "w_o", "w_fc1", "w_fc2")}
+        lp["ve"] = drawn.get((l, "ve"))
+        lp["ve_gate"] = drawn.get((l, "ve_gate"))
         p["layers"].append(lp)
     return p
 

@@ -175,6 +175,24 @@ const char* nc_last_error(void);
  * on this thread. */
 int nc_last_launch_count(void);
 
+/* Optional per-launch device timing for profiling.  `events` is an array of
+ * 2 * capacity cudaEvent_t created by the caller (passed as void*), `kinds`
+ * an int array of `capacity`.  While set, every launch by this thread whose
+ * kernel kind k has bit k set in kind_mask records events[2i] before and
+ * events[2i+1] after it on the call's stream, and kinds[i] = k, for i = 0, 1,
+ * ... up to capacity.  Calling again (or with events == NULL, which disables
+ * it) restarts the count.  Kinds: 0 embed_norm_smear, 1 rmsnorm, 2 rope_table,
+ * 3 rope_qknorm, 4 gemm_tcgen05, 5 gemm_cuda_core, 6 attention_tcgen05,
+ * 7 attention_cuda_core, 8 ce_combine, 9 ce_rows, 10 loss_mean.
+ * Returns NC_ERR_ARG if events != NULL with kinds == NULL or capacity <= 0. */
+int nc_set_launch_timing(void** events, int* kinds, int capacity, unsigned kind_mask);
+
+/* Event pairs recorded since the last nc_set_launch_timing() on this thread. */
+int nc_launch_timing_count(void);
+
+/* Name of a kernel kind ("unknown" out of range). */
+const char* nc_kernel_name(int kind);
+
 /* sizeof of the ABI structs, for bindings to check their mirrors:
  * which = 0 -> nc_config, 1 -> nc_layer_params, 2 -> nc_params; 0 otherwise. */
 size_t nc_sizeof(int which);

@@ -143,3 +143,24 @@ def test_status_strings():
         assert lib.nc_status_string(code)
     assert lib.nc_status_string(99) == b"unknown status"
     assert lib.nc_loss_mean(None, None, 4, None, None) == nc.STATUS_CODES["NC_ERR_ARG"]
+
+
+def test_flop_accounting_matches_pages():
+    """The FLOPs/token table of the StairFormer README (dense d9 and d23,
+    head_dim 64, T = 2048) under its convention 2 N_mat + 4 L C T."""
+    from golden_io import load
+    from decoder_only_transformer_fwd_b200 import flops
+    g = load("flops_per_token.txt")
+    for depth, head_dim, printed in g["rows"]:
+        C_, _ = O.model_dims(depth, head_dim=head_dim)
+        f = flops.dense_table_flops_per_token(depth, C_, 32768, g["seq_len"])
+        assert abs(f / printed - 1) < g["rtol"], (depth, f, printed)
+    # algorithmic d24 count: 12.963 TFLOP per 8192-token step
+    w = O.layer_windows(24, 2048, 1024)
+    f24 = flops.forward_flops_per_token(24, 1536, 32768, w, 2048)
+    assert abs(f24 * 8192 / 1e12 - 12.963) < 5e-3
+    assert abs(flops.mean_visible_keys(2048, 1024) - 768.25) < 1e-9
+    assert abs(flops.mean_visible_keys(2048, 2048) - 1024.5) < 1e-9
+    # brute force of the closed form
+    for T, wd in [(7, 3), (10, 10), (5, 9)]:
+        assert abs(flops.mean_visible_keys(T, wd) - sum(min(i + 1, wd) for i in range(T)) / T) < 1e-12
