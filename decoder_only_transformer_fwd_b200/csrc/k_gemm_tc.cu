@@ -42,7 +42,10 @@ struct TcCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = 2 * BN;
   static constexpr int NBARS = 2 * STAGES + 5;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+  // per epilogue warp: a 32 x 32 fp32 transpose buffer (row pitch 33)
+  static constexpr int STAGE_FLOATS = 32 * 33;
+  static constexpr int EPI_BYTES = 4 * STAGE_FLOATS * 4;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256 + EPI_BYTES;
 };
 
 struct TcArgs {
@@ -160,6 +163,128 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& ep, const TcArgs& a, 
   }
 }
 
+// Residual epilogues (EPI_RESID, EPI_BLOCK_END) for a 32-row x 32-column
+// chunk: the warp's rows arrive one per lane (TMEM lane = row); they are
+// transposed through shared memory so that for each row the warp reads and
+// writes one contiguous 128-byte segment of x (and x0 / x_bo), with all the
+// chunk's loads issued before its stores.
+__device__ __forceinline__ void epi_resid_chunk(const EpiParams& ep, const TcArgs& a, float* stage,
+                                                int row0, int n, const uint32_t (&r)[32], int lane) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = __uint_as_float(r[i]);
+  __syncwarp();
+  const int col = n + lane;
+  const bool col_ok = col < a.N;
+  float acc[32], xv[32], zv[32];
+#pragma unroll
+  for (int rr = 0; rr < 32; ++rr) acc[rr] = stage[rr * 33 + lane];
+  __syncwarp();
+  const bool bend = ep.mode == EPI_BLOCK_END;
+  const bool need_x0 = bend && ep.end_kind == 1;
+  const bool need_bo = bend && ep.end_kind == 2 && !ep.capture_bo;
+#pragma unroll
+  for (int rr = 0; rr < 32; ++rr) {
+    const int m = row0 + rr;
+    const size_t i = (size_t)m * ep.ldx + col;
+    const bool ok = col_ok && m < a.M;
+    xv[rr] = ok ? ep.x[i] : 0.f;
+    zv[rr] = (ok && need_x0) ? ep.x0[i] : ((ok && need_bo) ? ep.xbo[i] : 0.f);
+  }
+  float lam = 1.f, mu = 0.f;
+  if (need_x0) {
+    lam = *ep.lam;
+    mu = *ep.mu;
+  }
+#pragma unroll
+  for (int rr = 0; rr < 32; ++rr) {
+    const int m = row0 + rr;
+    if (!col_ok || m >= a.M) continue;
+    const size_t i = (size_t)m * ep.ldx + col;
+    float v = xv[rr] + acc[rr];
+    if (bend) {
+      if (ep.capture_bo) ep.xbo[i] = v;
+      if (ep.end_kind == 1)
+        v = lam * v + mu * zv[rr];
+      else if (ep.end_kind == 2)
+        v = v - ep.beta * (ep.capture_bo ? v : zv[rr]);
+    }
+    ep.x[i] = v;
+  }
+}
+
+// Fused QKV epilogue for the 128 columns of one head held in TMEM at taddr:
+// q and k heads get RoPE (position m % T) and alpha * RMSNorm over the head;
+// v heads get gate * VE[tok] added; one bf16 rounding at the store.
+// ("The Mathematics of Karpathy's nanochat", §Rotary Position Embeddings,
+// §QK-Norm with Sharpening, §Value Embeddings.)
+__device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& a, uint32_t taddr, int m,
+                                             int col0) {
+  float x[128];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t u[32];
+    ptx::tmem_ld32(taddr + (uint32_t)(c * 32), u);
+    ptx::tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(u[i]);
+  }
+  const bool row_ok = m < a.M;
+  if (col0 < ep.qk_cols) {
+    const int t = m % ep.T;
+    const float4* cs = reinterpret_cast<const float4*>(ep.rope_cos + (size_t)t * 64);
+    const float4* sn = reinterpret_cast<const float4*>(ep.rope_sin + (size_t)t * 64);
+    float ss = 0.f;
+#pragma unroll
+    for (int j4 = 0; j4 < 16; ++j4) {
+      const float4 c4 = cs[j4], s4 = sn[j4];
+      const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = 4 * j4 + e;
+        const float u1 = x[j], u2 = x[j + 64];
+        const float y1 = u1 * cc[e] + u2 * sv[e];
+        const float y2 = -u1 * sv[e] + u2 * cc[e];
+        x[j] = y1;
+        x[j + 64] = y2;
+        ss += y1 * y1 + y2 * y2;
+      }
+    }
+    const float r = ep.qk_alpha / sqrtf(ss * (1.0f / 128.0f) + ep.eps);
+#pragma unroll
+    for (int i = 0; i < 128; ++i) x[i] *= r;
+  } else if (ep.ve != nullptr) {
+    const int hv = (col0 - ep.qk_cols) >> 7;
+    int tok = row_ok ? ep.tokens[m] : 0;
+    tok = min(max(tok, 0), ep.vocab - 1);
+    const float g = row_ok ? ep.gate[(size_t)m * ep.n_kv_head + hv] : 0.f;
+    const uint4* e4 = reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(ep.ve) +
+                                                     ((size_t)tok * ep.n_kv_head + hv) * 128);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const uint4 w = e4[q];
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ww[e]));
+        x[8 * q + 2 * e] += g * f.x;
+        x[8 * q + 2 * e + 1] += g * f.y;
+      }
+    }
+  }
+  if (!row_ok) return;
+  uint4* d4 = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(ep.out) + (size_t)m * ep.ldo + col0);
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(x[8 * q + 2 * e], x[8 * q + 2 * e + 1]);
+      w[e] = *reinterpret_cast<uint32_t*>(&b2);
+    }
+    d4[q] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 template <int BN>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -171,6 +296,7 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * Cf::STAGE_BYTES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cf::NBARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* epi_stage = reinterpret_cast<float*>(smem + S * Cf::STAGE_BYTES + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t bar0 = ptx::smem_u32(bars);
@@ -301,12 +427,22 @@ __global__ void __launch_bounds__(192, 1)
       }
       float ce_sum = 0.f, ce_tgt = 0.f;
       const uint32_t taddr = tmem + ((uint32_t)(g * 32) << 16) + (uint32_t)(acc * BN);
+      if (ep.mode == EPI_QKV) {
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t r[32];
-        ptx::tmem_ld32(taddr + (uint32_t)c, r);
-        ptx::tmem_ld_wait();
-        epi_chunk(ep, a, m, n0 + c, r, ce_sum, ce_tgt, y);
+        for (int hh = 0; hh < BN / 128; ++hh)
+          if (n0 + hh * 128 < a.N) epi_qkv_head(ep, a, taddr + (uint32_t)(hh * 128), m, n0 + hh * 128);
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t r[32];
+          ptx::tmem_ld32(taddr + (uint32_t)c, r);
+          ptx::tmem_ld_wait();
+          if (ep.mode == EPI_RESID || ep.mode == EPI_BLOCK_END)
+            epi_resid_chunk(ep, a, epi_stage + (warp - 2) * Cf::STAGE_FLOATS, mb * kBM + g * 32, n0 + c, r,
+                            lane);
+          else
+            epi_chunk(ep, a, m, n0 + c, r, ce_sum, ce_tgt, y);
+        }
       }
       if (ep.mode == EPI_CE && m < a.M) {
         ep.ce_sum[(size_t)m * ep.ce_tiles + nb] = ce_sum;

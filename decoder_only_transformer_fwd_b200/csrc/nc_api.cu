@@ -226,7 +226,7 @@ int nc_init_config(nc_config* cfg, int depth, int max_T, int dtype, const char* 
   cfg->gate_channels = 12;
   cfg->smear = 1;
   cfg->gemm_impl = 0;
-  cfg->attn_impl = 1;
+  cfg->attn_impl = 0;
   cfg->qk_alpha = 1.15f;
   cfg->softmax_scale = 1.0f / sqrtf((float)head_dim);
   cfg->rope_base = 100000.0f;
@@ -303,15 +303,39 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
     // attention sub-block
     launch_rmsnorm(x, xn, M, C, c.eps, bf, ve ? lp.ve_gate : nullptr, Hkv, c.gate_channels,
                    c.ve_gate_scale, ve ? gate : nullptr, st);
-    EpiParams e = epi(EPI_STORE);
+    const bool tc = bf && c.gemm_impl == 0;
+    EpiParams e = epi(tc ? EPI_QKV : EPI_STORE);
     e.out = qkv;
     e.ldo = nqkv;
+    if (tc) {
+      // RoPE + QK-norm and the value-embedding mix run on the fp32 accumulator
+      e.T = T;
+      e.qk_cols = (H + Hkv) * D;
+      e.rope_cos = rcos;
+      e.rope_sin = rsin;
+      e.qk_alpha = c.qk_alpha;
+      e.eps = c.eps;
+      e.tokens = tokens;
+      e.ve = ve ? lp.ve : nullptr;
+      e.gate = gate;
+      e.n_kv_head = Hkv;
+      e.vocab = V;
+    }
     if (!gemm(c, d, xn, C, lp.w_qkv, C, M, nqkv, C, e, st)) return NC_ERR_CUDA;
-    launch_rope_qknorm_ve(qkv, nqkv, B, T, H, Hkv, D, rcos, rsin, c.qk_alpha, c.eps, tokens,
-                          ve ? lp.ve : nullptr, gate, V, bf, d.status, st);
+    if (!tc)
+      launch_rope_qknorm_ve(qkv, nqkv, B, T, H, Hkv, D, rcos, rsin, c.qk_alpha, c.eps, tokens,
+                            ve ? lp.ve : nullptr, gate, V, bf, d.status, st);
     const int w = c.window[l] >= T ? T : c.window[l];
-    launch_attn_simt(qkv, qkv + (size_t)H * D * esz, qkv + (size_t)(H + Hkv) * D * esz, nqkv, nqkv, nqkv,
-                     o, H * D, B, T, H, Hkv, w, c.softmax_scale, bf, st);
+    const char* qp = qkv;
+    const char* kp = qkv + (size_t)H * D * esz;
+    const char* vp = qkv + (size_t)(H + Hkv) * D * esz;
+    if (bf && c.attn_impl == 0) {
+      if (!launch_attn_tc((const bf16*)qp, (const bf16*)kp, (const bf16*)vp, nqkv, nqkv, nqkv, (bf16*)o, H * D,
+                          B, T, H, Hkv, w, c.softmax_scale, d.status, d.num_sms, st))
+        return NC_ERR_CUDA;
+    } else {
+      launch_attn_simt(qp, kp, vp, nqkv, nqkv, nqkv, o, H * D, B, T, H, Hkv, w, c.softmax_scale, bf, st);
+    }
     e = epi(EPI_RESID);
     e.x = x;
     e.ldx = C;
@@ -445,7 +469,13 @@ int nc_attention(const void* q, const void* k, const void* v, void* out, int B, 
     qa = qo;
     ka = ko;
   }
-  launch_attn_simt(qa, ka, v, H * D, Hkv * D, Hkv * D, out, H * D, B, T, H, Hkv, w, softmax_scale, bf, st);
+  if (bf) {
+    if (!launch_attn_tc((const bf16*)qa, (const bf16*)ka, (const bf16*)v, H * D, Hkv * D, Hkv * D, (bf16*)out,
+                        H * D, B, T, H, Hkv, w, softmax_scale, d.status, d.num_sms, st))
+      return NC_ERR_CUDA;
+  } else {
+    launch_attn_simt(qa, ka, v, H * D, Hkv * D, Hkv * D, out, H * D, B, T, H, Hkv, w, softmax_scale, bf, st);
+  }
   return check_launch("nc_attention");
 }
 

@@ -53,7 +53,8 @@ enum EpiMode : int {
   EPI_RESID = 2,     // x[m, n] += acc                        (fp32 residual)
   EPI_BLOCK_END = 3, // x += acc; capture x_bo; then re-inject for the next block or apply backout
   EPI_SOFTCAP = 4,   // logits[m, n] = cap tanh(acc / cap)    (fp32; CUDA-core path)
-  EPI_CE = 5         // softcap + per-(row, tile) log-sum-exp partials (+ optional logits)
+  EPI_CE = 5,        // softcap + per-(row, tile) log-sum-exp partials (+ optional logits)
+  EPI_QKV = 6        // q, k heads: RoPE + QK-norm; v heads: + gate * VE[tok]; bf16 out (tcgen05 path)
 };
 
 struct EpiParams {
@@ -78,6 +79,16 @@ struct EpiParams {
   float* ce_sum;      // [M, n_tiles]: sum over the tile's columns of exp(zhat - cap)
   float* ce_tgt;      // [M]
   int ce_tiles;
+  // EPI_QKV (out/ldo as for EPI_STORE)
+  int T;              // positions per row (position = m % T)
+  int qk_cols;        // (H + H_kv) * D: columns below this are q and k heads
+  const float* rope_cos;  // [T, D/2]
+  const float* rope_sin;
+  float qk_alpha, eps;
+  const int32_t* tokens;  // [M]
+  const void* ve;     // [V, H_kv D] or NULL
+  const float* gate;  // [M, H_kv]
+  int n_kv_head;
 };
 
 // launchers (host functions), all asynchronous on `st`

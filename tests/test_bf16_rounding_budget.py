@@ -1,9 +1,9 @@
 """Evidence for the bf16-mode loss tolerance.
 
 The bf16 path rounds to bf16 exactly at the GEMM operands and stored
-activations: the normalised block inputs, the fused q/k/v output, q and k
-after RoPE + QK-norm, v after the value-embedding mix, the attention output,
-the ReLU^2 output and the head input; everything else (the residual stream,
+activations: the normalised block inputs, q and k after RoPE + QK-norm and v
+after the value-embedding mix (all three applied to the fp32 accumulator of
+the QKV GEMM), the attention output, the ReLU^2 output and the head input; everything else (the residual stream,
 accumulation, softmax, softcap, log-sum-exp) stays in fp32 or better.  This
 test applies those roundings to the oracle's own fp64 steps and measures the
 per-token loss error they cause: its rms sets the bound the GPU parity tests
@@ -34,7 +34,7 @@ def _forward_rounded(cfg, p, tok, y):
         lp = p["layers"][l]
         x = p["resid_lambdas"][l] * x + p["x0_lambdas"][l] * x0
         a = O.rmsnorm(x, eps)
-        qkv = _rb(_rb(a) @ np.asarray(lp["w_qkv"], F64).T)
+        qkv = _rb(a) @ np.asarray(lp["w_qkv"], F64).T
         q = qkv[:, :H * D].reshape(T, H, D)
         k = qkv[:, H * D:2 * H * D].reshape(T, H, D)
         v = qkv[:, 2 * H * D:].reshape(T, H, D)

@@ -64,3 +64,16 @@ def test_attention_sweep_sampled(T, window):
         ref = _ref(q[b], k[b], v[b], window, positions=pos)
         err = np.max(np.abs(out[b, pos] - ref))
         assert err <= 2e-2, (b, err)
+
+
+@pytest.mark.parametrize("T,window", [(256, 0), (1000, 300), (129, 1), (2048, 1024)])
+def test_tc_attention_matches_fp32_attention(T, window):
+    """bf16 tensor-core attention vs the fp32 CUDA-core kernel on the same
+    (bf16-valued) inputs: the only differences are bf16 P and output."""
+    import torch
+    B, H, D = 2, 2, 128
+    q, k, v = synth.attention_inputs(900 + T, B, T, H, D)
+    out_tc = _run(q, k, v, window, "bf16")
+    out_32 = _run(q, k, v, window, "fp32")
+    assert np.max(np.abs(out_tc - out_32)) <= 2e-2
+    assert np.sqrt(np.mean((out_tc - out_32) ** 2)) <= 3e-3
