@@ -6,8 +6,10 @@
 //               into a STAGES-deep shared-memory ring;
 //   warp 1      allocates 2*BN TMEM columns; one thread issues tcgen05.mma
 //               (M = 128, N = BN, K = 16) into one of two accumulators;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one TMEM lane per
-//               output row), the fused element-wise op, global stores.
+//   warps 2..9  epilogue, two warps per TMEM lane quarter (one TMEM lane per
+//               output row), each on half of the tile's columns: tcgen05.ld of
+//               the accumulator, the fused element-wise op, global stores.
+// The kernel is specialised on the epilogue at compile time.
 // The two accumulators let the epilogue of tile i overlap the MMAs of tile
 // i + 1.  Every wait is bounded (see ptx::mbar_wait); on a timeout the CTA
 // records NC_ERR_TIMEOUT, stops issuing work, waits for its own copies and
@@ -33,6 +35,8 @@ namespace nc {
 namespace {
 
 constexpr int kBM = 128, kBK = 64, kUK = 16;
+constexpr int kEpiWarps = 8;                 // two per TMEM lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;  // + the TMA and MMA warps
 
 template <int BN>
 struct TcCfg {
@@ -44,7 +48,7 @@ struct TcCfg {
   static constexpr int NBARS = 2 * STAGES + 5;
   // per epilogue warp: a 32 x 32 fp32 transpose buffer (row pitch 33)
   static constexpr int STAGE_FLOATS = 32 * 33;
-  static constexpr int EPI_BYTES = 4 * STAGE_FLOATS * 4;
+  static constexpr int EPI_BYTES = kEpiWarps * STAGE_FLOATS * 4;
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256 + EPI_BYTES;
 };
 
@@ -56,110 +60,36 @@ struct TcArgs {
 
 __device__ __forceinline__ float bits2f(uint32_t u) { return __uint_as_float(u); }
 
-// Softcap via tanh(u) = 1 - 2 / (exp(2u) + 1).
-__device__ __forceinline__ float softcap_fast(float z, float cap) {
-  const float t = __expf(2.0f * z / cap);
-  return cap * (1.0f - 2.0f / (t + 1.0f));
-}
-
-// Epilogue for 32 consecutive columns [n, n + 32) of row m held in r[].
+// EPI_STORE / EPI_RELU2 for 32 consecutive columns [n, n + 32) of row m:
+// bf16 conversion and one 64-byte store per thread.
 __device__ __forceinline__ void epi_chunk(const EpiParams& ep, const TcArgs& a, int m, int n,
-                                          const uint32_t (&r)[32], float& ce_sum, float& ce_tgt,
-                                          int y) {
-  const bool row_ok = m < a.M;
-  switch (ep.mode) {
-    case EPI_STORE:
-    case EPI_RELU2: {
-      if (!row_ok) return;
-      bf16* dst = reinterpret_cast<bf16*>(ep.out) + (size_t)m * ep.ldo + n;
-      if (n + 32 <= a.N) {
-        uint4* d4 = reinterpret_cast<uint4*>(dst);
+                                          const uint32_t (&r)[32], float&, float&, int) {
+  if (m >= a.M) return;
+  const bool relu2 = ep.mode == EPI_RELU2;
+  bf16* dst = reinterpret_cast<bf16*>(ep.out) + (size_t)m * ep.ldo + n;
+  if (n + 32 <= a.N) {
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t w[4];
+    for (int q = 0; q < 4; ++q) {
+      uint32_t w[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float v0 = bits2f(r[q * 8 + 2 * e]), v1 = bits2f(r[q * 8 + 2 * e + 1]);
-            if (ep.mode == EPI_RELU2) {
-              v0 = fmaxf(v0, 0.f); v0 *= v0;
-              v1 = fmaxf(v1, 0.f); v1 *= v1;
-            }
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
-            w[e] = *reinterpret_cast<uint32_t*>(&b2);
-          }
-          d4[q] = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int e = 0; e < 4; ++e) {
+        float v0 = bits2f(r[q * 8 + 2 * e]), v1 = bits2f(r[q * 8 + 2 * e + 1]);
+        if (relu2) {
+          v0 = fmaxf(v0, 0.f);
+          v0 *= v0;
+          v1 = fmaxf(v1, 0.f);
+          v1 *= v1;
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (n + i < a.N) epi_apply<bf16>(ep, m, n + i, bits2f(r[i]));
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
+        w[e] = *reinterpret_cast<uint32_t*>(&b2);
       }
-    } break;
-    case EPI_RESID:
-    case EPI_BLOCK_END: {
-      if (!row_ok) return;
-      if (n + 32 <= a.N) {
-        float4* x4 = reinterpret_cast<float4*>(ep.x + (size_t)m * ep.ldx + n);
-        const float4* x04 = reinterpret_cast<const float4*>(ep.x0 + (size_t)m * ep.ldx + n);
-        float4* b4 = reinterpret_cast<float4*>(ep.xbo + (size_t)m * ep.ldx + n);
+      d4[q] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  } else {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float4 v = x4[q];
-          v.x += bits2f(r[4 * q + 0]);
-          v.y += bits2f(r[4 * q + 1]);
-          v.z += bits2f(r[4 * q + 2]);
-          v.w += bits2f(r[4 * q + 3]);
-          if (ep.mode == EPI_BLOCK_END) {
-            if (ep.capture_bo) b4[q] = v;
-            if (ep.end_kind == 1) {
-              const float4 z = x04[q];
-              const float lam = *ep.lam, mu = *ep.mu;
-              v.x = lam * v.x + mu * z.x;
-              v.y = lam * v.y + mu * z.y;
-              v.z = lam * v.z + mu * z.z;
-              v.w = lam * v.w + mu * z.w;
-            } else if (ep.end_kind == 2) {
-              const float4 z = b4[q];
-              v.x -= ep.beta * z.x;
-              v.y -= ep.beta * z.y;
-              v.z -= ep.beta * z.z;
-              v.w -= ep.beta * z.w;
-            }
-          }
-          x4[q] = v;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (n + i < a.N) epi_apply<float>(ep, m, n + i, bits2f(r[i]));
-      }
-    } break;
-    case EPI_CE: {
-      float zh[32];
-      float s = 0.f;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        zh[i] = softcap_fast(bits2f(r[i]), ep.cap);
-        const bool ok = (n + i) < ep.vocab;
-        s += ok ? __expf(zh[i] - ep.cap) : 0.f;
-        if (n + i == y) ce_tgt = zh[i];
-      }
-      ce_sum += s;
-      if (row_ok && ep.logits != nullptr) {
-        float* dst = ep.logits + (size_t)m * ep.ldl + n;
-        if (n + 32 <= ep.vocab) {
-          float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) d4[q] = make_float4(zh[4 * q], zh[4 * q + 1], zh[4 * q + 2], zh[4 * q + 3]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (n + i < ep.vocab) dst[i] = zh[i];
-        }
-      }
-    } break;
-    default:
-      break;
+    for (int i = 0; i < 32; ++i)
+      if (n + i < a.N) epi_apply<bf16>(ep, m, n + i, bits2f(r[i]));
   }
 }
 
@@ -175,41 +105,43 @@ __device__ __forceinline__ void epi_resid_chunk(const EpiParams& ep, const TcArg
   __syncwarp();
   const int col = n + lane;
   const bool col_ok = col < a.N;
-  float acc[32], xv[32], zv[32];
-#pragma unroll
-  for (int rr = 0; rr < 32; ++rr) acc[rr] = stage[rr * 33 + lane];
-  __syncwarp();
   const bool bend = ep.mode == EPI_BLOCK_END;
   const bool need_x0 = bend && ep.end_kind == 1;
   const bool need_bo = bend && ep.end_kind == 2 && !ep.capture_bo;
-#pragma unroll
-  for (int rr = 0; rr < 32; ++rr) {
-    const int m = row0 + rr;
-    const size_t i = (size_t)m * ep.ldx + col;
-    const bool ok = col_ok && m < a.M;
-    xv[rr] = ok ? ep.x[i] : 0.f;
-    zv[rr] = (ok && need_x0) ? ep.x0[i] : ((ok && need_bo) ? ep.xbo[i] : 0.f);
-  }
   float lam = 1.f, mu = 0.f;
   if (need_x0) {
     lam = *ep.lam;
     mu = *ep.mu;
   }
 #pragma unroll
-  for (int rr = 0; rr < 32; ++rr) {
-    const int m = row0 + rr;
-    if (!col_ok || m >= a.M) continue;
-    const size_t i = (size_t)m * ep.ldx + col;
-    float v = xv[rr] + acc[rr];
-    if (bend) {
-      if (ep.capture_bo) ep.xbo[i] = v;
-      if (ep.end_kind == 1)
-        v = lam * v + mu * zv[rr];
-      else if (ep.end_kind == 2)
-        v = v - ep.beta * (ep.capture_bo ? v : zv[rr]);
+  for (int h16 = 0; h16 < 2; ++h16) {
+    float acc[16], xv[16], zv[16];
+#pragma unroll
+    for (int rr = 0; rr < 16; ++rr) {
+      const int m = row0 + h16 * 16 + rr;
+      const size_t i = (size_t)m * ep.ldx + col;
+      const bool ok = col_ok && m < a.M;
+      acc[rr] = stage[(h16 * 16 + rr) * 33 + lane];
+      xv[rr] = ok ? ep.x[i] : 0.f;
+      zv[rr] = (ok && need_x0) ? ep.x0[i] : ((ok && need_bo) ? ep.xbo[i] : 0.f);
     }
-    ep.x[i] = v;
+#pragma unroll
+    for (int rr = 0; rr < 16; ++rr) {
+      const int m = row0 + h16 * 16 + rr;
+      if (!col_ok || m >= a.M) continue;
+      const size_t i = (size_t)m * ep.ldx + col;
+      float v = xv[rr] + acc[rr];
+      if (bend) {
+        if (ep.capture_bo) ep.xbo[i] = v;
+        if (ep.end_kind == 1)
+          v = lam * v + mu * zv[rr];
+        else if (ep.end_kind == 2)
+          v = v - ep.beta * (ep.capture_bo ? v : zv[rr]);
+      }
+      ep.x[i] = v;
+    }
   }
+  __syncwarp();
 }
 
 // Fused QKV epilogue for the 128 columns of one head held in TMEM at taddr:
@@ -219,74 +151,179 @@ __device__ __forceinline__ void epi_resid_chunk(const EpiParams& ep, const TcArg
 // §QK-Norm with Sharpening, §Value Embeddings.)
 __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& a, uint32_t taddr, int m,
                                              int col0) {
-  float x[128];
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint32_t u[32];
-    ptx::tmem_ld32(taddr + (uint32_t)(c * 32), u);
-    ptx::tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(u[i]);
-  }
   const bool row_ok = m < a.M;
+  bf16* out = reinterpret_cast<bf16*>(ep.out) + (size_t)m * ep.ldo + col0;
   if (col0 < ep.qk_cols) {
-    const int t = m % ep.T;
-    const float4* cs = reinterpret_cast<const float4*>(ep.rope_cos + (size_t)t * 64);
-    const float4* sn = reinterpret_cast<const float4*>(ep.rope_sin + (size_t)t * 64);
+    // RoPE pairs (j, j + 64) live in chunks (c, c + 2); the rotation preserves
+    // each pair's sum of squares, so the RMS comes from the raw accumulator
+    // in a first pass and the rotation + scale is applied in a second.
     float ss = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t u[32];
+      ptx::tmem_ld32(taddr + (uint32_t)(c * 32), u);
+      ptx::tmem_ld_wait();
 #pragma unroll
-    for (int j4 = 0; j4 < 16; ++j4) {
-      const float4 c4 = cs[j4], s4 = sn[j4];
-      const float cc[4] = {c4.x, c4.y, c4.z, c4.w}, sv[4] = {s4.x, s4.y, s4.z, s4.w};
+      for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(u[i]), __uint_as_float(u[i]), ss);
+    }
+    const float rs = ep.qk_alpha / sqrtf(ss * (1.0f / 128.0f) + ep.eps);
+    const int t = m % ep.T;
+    const float* cs = ep.rope_cos + (size_t)t * 64;
+    const float* sn = ep.rope_sin + (size_t)t * 64;
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      uint32_t u1[32], u2[32];
+      ptx::tmem_ld32(taddr + (uint32_t)(c * 32), u1);
+      ptx::tmem_ld32(taddr + (uint32_t)(c * 32 + 64), u2);
+      ptx::tmem_ld_wait();
+      if (!row_ok) continue;
+      const float4* c4 = reinterpret_cast<const float4*>(cs + c * 32);
+      const float4* s4 = reinterpret_cast<const float4*>(sn + c * 32);
+      uint32_t w1[16], w2[16];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = 4 * j4 + e;
-        const float u1 = x[j], u2 = x[j + 64];
-        const float y1 = u1 * cc[e] + u2 * sv[e];
-        const float y2 = -u1 * sv[e] + u2 * cc[e];
-        x[j] = y1;
-        x[j + 64] = y2;
-        ss += y1 * y1 + y2 * y2;
+      for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 cc = c4[j4], sv = s4[j4];
+        const float cf[4] = {cc.x, cc.y, cc.z, cc.w}, sf[4] = {sv.x, sv.y, sv.z, sv.w};
+        float y1[4], y2[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a1 = __uint_as_float(u1[4 * j4 + e]), a2 = __uint_as_float(u2[4 * j4 + e]);
+          y1[e] = (a1 * cf[e] + a2 * sf[e]) * rs;
+          y2[e] = (-a1 * sf[e] + a2 * cf[e]) * rs;
+        }
+        __nv_bfloat162 p;
+        p = __floats2bfloat162_rn(y1[0], y1[1]); w1[2 * j4] = *reinterpret_cast<uint32_t*>(&p);
+        p = __floats2bfloat162_rn(y1[2], y1[3]); w1[2 * j4 + 1] = *reinterpret_cast<uint32_t*>(&p);
+        p = __floats2bfloat162_rn(y2[0], y2[1]); w2[2 * j4] = *reinterpret_cast<uint32_t*>(&p);
+        p = __floats2bfloat162_rn(y2[2], y2[3]); w2[2 * j4 + 1] = *reinterpret_cast<uint32_t*>(&p);
+      }
+      uint4* d1 = reinterpret_cast<uint4*>(out + c * 32);
+      uint4* d2 = reinterpret_cast<uint4*>(out + c * 32 + 64);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        d1[q] = make_uint4(w1[4 * q], w1[4 * q + 1], w1[4 * q + 2], w1[4 * q + 3]);
+        d2[q] = make_uint4(w2[4 * q], w2[4 * q + 1], w2[4 * q + 2], w2[4 * q + 3]);
       }
     }
-    const float r = ep.qk_alpha / sqrtf(ss * (1.0f / 128.0f) + ep.eps);
-#pragma unroll
-    for (int i = 0; i < 128; ++i) x[i] *= r;
-  } else if (ep.ve != nullptr) {
+  } else {
     const int hv = (col0 - ep.qk_cols) >> 7;
     int tok = row_ok ? ep.tokens[m] : 0;
     tok = min(max(tok, 0), ep.vocab - 1);
-    const float g = row_ok ? ep.gate[(size_t)m * ep.n_kv_head + hv] : 0.f;
-    const uint4* e4 = reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(ep.ve) +
-                                                     ((size_t)tok * ep.n_kv_head + hv) * 128);
+    const float g = (row_ok && ep.ve != nullptr) ? ep.gate[(size_t)m * ep.n_kv_head + hv] : 0.f;
+    const uint4* e4 = ep.ve != nullptr ? reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(ep.ve) +
+                                                                      ((size_t)tok * ep.n_kv_head + hv) * 128)
+                                       : nullptr;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t u[32];
+      ptx::tmem_ld32(taddr + (uint32_t)(c * 32), u);
+      ptx::tmem_ld_wait();
+      if (!row_ok) continue;
+      float x[32];
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      const uint4 w = e4[q];
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+      for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(u[i]);
+      if (e4 != nullptr) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ww[e]));
-        x[8 * q + 2 * e] += g * f.x;
-        x[8 * q + 2 * e + 1] += g * f.y;
+        for (int q = 0; q < 4; ++q) {
+          const uint4 w = e4[c * 4 + q];
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ww[e]));
+            x[8 * q + 2 * e] += g * f.x;
+            x[8 * q + 2 * e + 1] += g * f.y;
+          }
+        }
+      }
+      uint4* d4 = reinterpret_cast<uint4*>(out + c * 32);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(x[8 * q + 2 * e], x[8 * q + 2 * e + 1]);
+          w[e] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        d4[q] = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
   }
-  if (!row_ok) return;
-  uint4* d4 = reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(ep.out) + (size_t)m * ep.ldo + col0);
-#pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    uint32_t w[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      __nv_bfloat162 b2 = __floats2bfloat162_rn(x[8 * q + 2 * e], x[8 * q + 2 * e + 1]);
-      w[e] = *reinterpret_cast<uint32_t*>(&b2);
+}
+
+// Epilogue work of one warp on one tile: rows g*32 .. g*32+31 of the tile
+// (its TMEM lane quarter) and the columns [c_lo, c_lo + BN/2) of its half.
+template <int BN, int MODE>
+__device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs& a, uint32_t taddr, int mb,
+                                              int nb, int g, int half, int lane, float* stage) {
+  constexpr int HALF = BN / 2;
+  const int row = g * 32 + lane;
+  const int m = mb * kBM + row;
+  const int c_lo = half * HALF;
+  const int n_lo = nb * BN + c_lo;
+  if constexpr (MODE == EPI_QKV) {
+    // one head (128 columns) per warp when BN = 256; with BN = 128 the first half does it
+    if (c_lo % 128 == 0 && n_lo < a.N) epi_qkv_head(ep, a, taddr + (uint32_t)c_lo, m, n_lo);
+  } else if constexpr (MODE == EPI_CE) {
+    int y = -1;
+    if (m < a.M) {
+      y = ep.targets[m];
+      if (y != -1) y = min(max(y, 0), ep.vocab - 1);  // out-of-range ids are flagged by the combine
     }
-    d4[q] = make_uint4(w[0], w[1], w[2], w[3]);
+    // zhat = c tanh(z/c) = c - 2c / (e^{2z/c} + 1); exp(zhat - c) = 2^(-2c log2(e) / (e^{2z/c} + 1))
+    const float k1 = 2.0f * 1.4426950408889634f / ep.cap;
+    const float k2 = -2.0f * ep.cap * 1.4426950408889634f;
+    const float c2 = -2.0f * ep.cap;
+    float sum = 0.f, tgt = 0.f;
+#pragma unroll 1
+    for (int c = 0; c < HALF; c += 32) {
+      uint32_t r[32];
+      ptx::tmem_ld32(taddr + (uint32_t)(c_lo + c), r);
+      ptx::tmem_ld_wait();
+      const int n = n_lo + c;
+      float zh[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float q = ptx::rcp(ptx::ex2(__uint_as_float(r[i]) * k1) + 1.0f);
+        zh[i] = fmaf(c2, q, ep.cap);
+        const float p = ptx::ex2(k2 * q);
+        sum += (n + i < ep.vocab) ? p : 0.f;
+        tgt = (n + i == y) ? zh[i] : tgt;
+      }
+      if (ep.logits != nullptr && m < a.M) {
+        float* dst = ep.logits + (size_t)m * ep.ldl + n;
+        if (n + 32 <= ep.vocab) {
+          float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) d4[q] = make_float4(zh[4 * q], zh[4 * q + 1], zh[4 * q + 2], zh[4 * q + 3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (n + i < ep.vocab) dst[i] = zh[i];
+        }
+      }
+    }
+    if (m < a.M) {
+      ep.ce_sum[(size_t)m * ep.ce_tiles + nb * 2 + half] = sum;
+      if (y >= n_lo && y < n_lo + HALF) ep.ce_tgt[m] = tgt;
+    }
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < HALF; c += 32) {
+      uint32_t r[32];
+      ptx::tmem_ld32(taddr + (uint32_t)(c_lo + c), r);
+      ptx::tmem_ld_wait();
+      if constexpr (MODE == EPI_RESID || MODE == EPI_BLOCK_END) {
+        epi_resid_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, r, lane);
+      } else {
+        float ce_sum = 0.f, ce_tgt = 0.f;
+        epi_chunk(ep, a, m, n_lo + c, r, ce_sum, ce_tgt, -1);
+      }
+    }
   }
 }
 
-template <int BN>
-__global__ void __launch_bounds__(192, 1)
+template <int BN, int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const TcArgs a, const EpiParams ep) {
   using Cf = TcCfg<BN>;
@@ -315,7 +352,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(tfull(i), 1);
-      ptx::mbar_init(tempty(i), 4);
+      ptx::mbar_init(tempty(i), kEpiWarps);
     }
     ptx::mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -406,9 +443,12 @@ __global__ void __launch_bounds__(192, 1)
       ptx::mbar_wait(mma_done, 0, a.status);
     }
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
-    const int g = warp & 3;  // the TMEM lane quarter this warp may access
-    const int row = g * 32 + lane;
+    // ---------------- epilogue (warps 2 .. 2 + kEpiWarps - 1) ----------------
+    // two warps per TMEM lane quarter, each taking half of the tile's columns
+    const int ew = warp - 2;
+    const int g = warp & 3;
+    const int half = ew >> 2;
+    float* stage = epi_stage + ew * Cf::STAGE_FLOATS;
     int acc = 0;
     uint32_t aph = 0;
     for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
@@ -418,36 +458,8 @@ __global__ void __launch_bounds__(192, 1)
         break;
       }
       ptx::tc_fence_after();
-      const int m = mb * kBM + row;
-      const int n0 = nb * BN;
-      int y = -1;
-      if (ep.mode == EPI_CE && m < a.M) {
-        y = ep.targets[m];
-        if (y != -1) y = min(max(y, 0), ep.vocab - 1);  // out-of-range ids are flagged by the combine
-      }
-      float ce_sum = 0.f, ce_tgt = 0.f;
       const uint32_t taddr = tmem + ((uint32_t)(g * 32) << 16) + (uint32_t)(acc * BN);
-      if (ep.mode == EPI_QKV) {
-#pragma unroll 1
-        for (int hh = 0; hh < BN / 128; ++hh)
-          if (n0 + hh * 128 < a.N) epi_qkv_head(ep, a, taddr + (uint32_t)(hh * 128), m, n0 + hh * 128);
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          uint32_t r[32];
-          ptx::tmem_ld32(taddr + (uint32_t)c, r);
-          ptx::tmem_ld_wait();
-          if (ep.mode == EPI_RESID || ep.mode == EPI_BLOCK_END)
-            epi_resid_chunk(ep, a, epi_stage + (warp - 2) * Cf::STAGE_FLOATS, mb * kBM + g * 32, n0 + c, r,
-                            lane);
-          else
-            epi_chunk(ep, a, m, n0 + c, r, ce_sum, ce_tgt, y);
-        }
-      }
-      if (ep.mode == EPI_CE && m < a.M) {
-        ep.ce_sum[(size_t)m * ep.ce_tiles + nb] = ce_sum;
-        if (y >= n0 && y < n0 + BN) ep.ce_tgt[m] = ce_tgt;
-      }
+      epilogue_tile<BN, MODE>(ep, a, taddr, mb, nb, g, half, lane, stage);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(tempty(acc));
@@ -480,12 +492,28 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
-template <int BN>
-void set_smem_attr() {
+template <int BN, int MODE>
+void launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep, int grid,
+                 cudaStream_t st) {
   static std::once_flag once;
   std::call_once(once, [] {
-    cudaFuncSetAttribute(k_gemm_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<BN>::SMEM);
+    cudaFuncSetAttribute(k_gemm_tc<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<BN>::SMEM);
   });
+  k_gemm_tc<BN, MODE><<<grid, kThreads, TcCfg<BN>::SMEM, st>>>(ta, tb, a, ep);
+}
+
+template <int BN>
+bool launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep, int grid,
+               cudaStream_t st) {
+  switch (ep.mode) {
+    case EPI_STORE: launch_mode<BN, EPI_STORE>(ta, tb, a, ep, grid, st); return true;
+    case EPI_RELU2: launch_mode<BN, EPI_RELU2>(ta, tb, a, ep, grid, st); return true;
+    case EPI_RESID: launch_mode<BN, EPI_RESID>(ta, tb, a, ep, grid, st); return true;
+    case EPI_BLOCK_END: launch_mode<BN, EPI_BLOCK_END>(ta, tb, a, ep, grid, st); return true;
+    case EPI_CE: launch_mode<BN, EPI_CE>(ta, tb, a, ep, grid, st); return true;
+    case EPI_QKV: launch_mode<BN, EPI_QKV>(ta, tb, a, ep, grid, st); return true;
+    default: return false;
+  }
 }
 
 }  // namespace
@@ -537,14 +565,7 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
   a.status = status;
   const int grid = a.num_tiles < num_sms ? a.num_tiles : num_sms;
   LaunchScope scope_(KK_GEMM_TC, st);
-  if (BN == 256) {
-    set_smem_attr<256>();
-    k_gemm_tc<256><<<grid, 192, TcCfg<256>::SMEM, st>>>(ta, tb, a, ep);
-  } else {
-    set_smem_attr<128>();
-    k_gemm_tc<128><<<grid, 192, TcCfg<128>::SMEM, st>>>(ta, tb, a, ep);
-  }
-  return true;
+  return BN == 256 ? launch_bn<256>(ta, tb, a, ep, grid, st) : launch_bn<128>(ta, tb, a, ep, grid, st);
 }
 
 }  // namespace nc

@@ -146,7 +146,7 @@ Layout layout(const nc_config& c, int max_tokens) {
   L.gate = take(M * c.n_kv_head * 4);
   L.rcos = take((size_t)c.max_T * D / 2 * 4);
   L.rsin = take((size_t)c.max_T * D / 2 * 4);
-  L.ce_tiles = (c.vocab_padded + 127) / 128;
+  L.ce_tiles = 2 * ((c.vocab_padded + 127) / 128);  // per (row, 128-or-256-column tile, half)
   L.ce_sum = take(M * L.ce_tiles * 4);
   L.ce_tgt = take(M * 4);
   const bool simt_head = c.dtype == NC_FP32 || c.gemm_impl != 0;
@@ -367,7 +367,7 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
   launch_rmsnorm(x, xn, M, C, c.eps, bf, nullptr, 0, 0, 0.f, nullptr, st);
   if (bf && c.gemm_impl == 0) {
     const int bn = gemm_tc_bn(c.vocab_padded);
-    const int tiles = (c.vocab_padded + bn - 1) / bn;
+    const int tiles = 2 * ((c.vocab_padded + bn - 1) / bn);  // two epilogue halves per tile
     EpiParams e = epi(EPI_CE);
     e.cap = c.softcap;
     e.vocab = V;
