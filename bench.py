@@ -162,6 +162,47 @@ def run_reference(args):
     return 0
 
 
+def attention_sweep(args, dev, stream):
+    """The single attention layer sweep (RoPE + QK-norm, then causal sliding-window
+    attention; B = 8, H = 12, D = 128): per case the attention kernel's own
+    device time (launch events, averaged over `steps` calls) and its
+    algorithmic TFLOP/s, plus the whole nc_attention call."""
+    import torch
+
+    from decoder_only_transformer_fwd_b200 import flops, nc, synth
+    peaks, _ = load_peaks()
+    s = synth.ATTN_SWEEP
+    B, H, D = s["B"], s["H"], s["D"]
+    out = []
+    for T, window in s["cases"]:
+        g = torch.Generator(device=dev).manual_seed(synth.SEED_BASE + s["index"])
+        q, k, v = (torch.randn(B, T, H, D, device=dev, generator=g).to(torch.bfloat16) for _ in range(3))
+        o = torch.empty_like(q)
+        ws = torch.empty(nc.nc_attention_workspace_bytes(B, T, H, H, D, "bf16", 1), dtype=torch.uint8,
+                         device=dev)
+        call = lambda: nc.nc_attention(q, k, v, o, window, 1, 1.15, D ** -0.5, 100000.0, 1e-6, ws, stream)
+        for _ in range(3):
+            call()
+        timer = nc.LaunchTimer(args.steps, kinds=["attention_tcgen05"])
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        with timer:
+            for _ in range(args.steps):
+                call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        n, kms = timer.per_kind().get("attention_tcgen05", (0, 0.0))
+        f = flops.attention_layer_flops(B, T, H, D, window)
+        us = 1e3 * kms / max(n, 1)
+        tf = f / (us * 1e-6) / 1e12
+        out.append({"T": T, "window": window if window > 0 else "full", "kernel_us": us,
+                    "call_us": 1e3 * e0.elapsed_time(e1) / args.steps, "gflop": f / 1e9, "tflops": tf,
+                    "pct_bf16_peak": 100.0 * tf / peaks["bf16_tflops"]})
+        del q, k, v, o, ws
+    return out
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -256,6 +297,7 @@ def run_ours(args):
     for _ in range(args.steps):
         nc.nc_forward_host(model.params, h_tok, h_tgt, h_loss, stream)
     e2e_s = max_over_ranks(time.perf_counter() - t0)
+    attn = None if args.no_attention_sweep else attention_sweep(args, dev, stream)
     clk = clocks.stop()
     rc, bits = nc.nc_get_status(stream)
     if rc != 0:
@@ -316,6 +358,7 @@ def run_ours(args):
                     "h2d_bytes_per_step": 2 * M * 4, "d2h_bytes_per_step": M * 4},
             "gpu_launches": launches_per_step * args.steps,
             "kernel_ms_per_step": {k: v[1] / args.steps for k, v in per_kind.items()},
+            "attention_sweep": attn,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -332,6 +375,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=1024)
     ap.add_argument("--rows", type=int, default=0, help="rows per step (default: the workload's B = 4)")
+    ap.add_argument("--no-attention-sweep", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

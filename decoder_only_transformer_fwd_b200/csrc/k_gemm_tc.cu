@@ -157,6 +157,9 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
     // RoPE pairs (j, j + 64) live in chunks (c, c + 2); the rotation preserves
     // each pair's sum of squares, so the RMS comes from the raw accumulator
     // in a first pass and the rotation + scale is applied in a second.
+    const int t = m % ep.T;
+    const float4* cs4 = reinterpret_cast<const float4*>(ep.rope_cos + (size_t)t * 64);
+    const float4* sn4 = reinterpret_cast<const float4*>(ep.rope_sin + (size_t)t * 64);
     float ss = 0.f;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
@@ -167,9 +170,6 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
       for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(u[i]), __uint_as_float(u[i]), ss);
     }
     const float rs = ep.qk_alpha / sqrtf(ss * (1.0f / 128.0f) + ep.eps);
-    const int t = m % ep.T;
-    const float* cs = ep.rope_cos + (size_t)t * 64;
-    const float* sn = ep.rope_sin + (size_t)t * 64;
 #pragma unroll 1
     for (int c = 0; c < 2; ++c) {
       uint32_t u1[32], u2[32];
@@ -177,12 +177,10 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
       ptx::tmem_ld32(taddr + (uint32_t)(c * 32 + 64), u2);
       ptx::tmem_ld_wait();
       if (!row_ok) continue;
-      const float4* c4 = reinterpret_cast<const float4*>(cs + c * 32);
-      const float4* s4 = reinterpret_cast<const float4*>(sn + c * 32);
       uint32_t w1[16], w2[16];
 #pragma unroll
       for (int j4 = 0; j4 < 8; ++j4) {
-        const float4 cc = c4[j4], sv = s4[j4];
+        const float4 cc = cs4[c * 8 + j4], sv = sn4[c * 8 + j4];
         const float cf[4] = {cc.x, cc.y, cc.z, cc.w}, sf[4] = {sv.x, sv.y, sv.z, sv.w};
         float y1[4], y2[4];
 #pragma unroll
@@ -209,11 +207,18 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
     const int hv = (col0 - ep.qk_cols) >> 7;
     int tok = row_ok ? ep.tokens[m] : 0;
     tok = min(max(tok, 0), ep.vocab - 1);
-    const float g = (row_ok && ep.ve != nullptr) ? ep.gate[(size_t)m * ep.n_kv_head + hv] : 0.f;
-    const uint4* e4 = ep.ve != nullptr ? reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(ep.ve) +
-                                                                      ((size_t)tok * ep.n_kv_head + hv) * 128)
-                                       : nullptr;
-#pragma unroll 1
+    const bool mix = row_ok && ep.ve != nullptr;
+    const float g = mix ? ep.gate[(size_t)m * ep.n_kv_head + hv] : 0.f;
+    // the row's 128 value-embedding entries are gathered up front (one memory
+    // round trip per row instead of one per chunk)
+    uint4 e[16];
+    if (mix) {
+      const uint4* e4 = reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(ep.ve) +
+                                                       ((size_t)tok * ep.n_kv_head + hv) * 128);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) e[q] = e4[q];
+    }
+#pragma unroll
     for (int c = 0; c < 4; ++c) {
       uint32_t u[32];
       ptx::tmem_ld32(taddr + (uint32_t)(c * 32), u);
@@ -222,16 +227,16 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
       float x[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(u[i]);
-      if (e4 != nullptr) {
+      if (mix) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const uint4 w = e4[c * 4 + q];
+          const uint4 w = e[c * 4 + q];
           const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ww[e]));
-            x[8 * q + 2 * e] += g * f.x;
-            x[8 * q + 2 * e + 1] += g * f.y;
+          for (int k = 0; k < 4; ++k) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ww[k]));
+            x[8 * q + 2 * k] += g * f.x;
+            x[8 * q + 2 * k + 1] += g * f.y;
           }
         }
       }
@@ -240,9 +245,9 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
       for (int q = 0; q < 4; ++q) {
         uint32_t w[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(x[8 * q + 2 * e], x[8 * q + 2 * e + 1]);
-          w[e] = *reinterpret_cast<uint32_t*>(&b2);
+        for (int k = 0; k < 4; ++k) {
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(x[8 * q + 2 * k], x[8 * q + 2 * k + 1]);
+          w[k] = *reinterpret_cast<uint32_t*>(&b2);
         }
         d4[q] = make_uint4(w[0], w[1], w[2], w[3]);
       }

@@ -119,6 +119,7 @@ bool config_ok(const nc_config& c) {
   if (c.max_T <= 0 || (c.dtype != NC_BF16 && c.dtype != NC_FP32)) return false;
   if (c.gate_channels < 0 || c.gate_channels > c.n_embd) return false;
   if (c.backout_layer >= c.n_layer) return false;
+  if (!(c.softmax_scale > 0.f) || !(c.softcap > 0.f) || !(c.eps >= 0.f)) return false;
   for (int l = 0; l < c.n_layer; ++l)
     if (c.window[l] <= 0) return false;
   return true;
@@ -443,6 +444,7 @@ int nc_attention(const void* q, const void* k, const void* v, void* out, int B, 
   t_launches = 0;
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return NC_ERR_ARG;
   if (dtype != NC_BF16 && dtype != NC_FP32) return NC_ERR_ARG;
+  if (!(softmax_scale > 0.f) || !(eps >= 0.f)) return NC_ERR_ARG;
   if (B <= 0 || T <= 0 || H <= 0 || Hkv <= 0) return NC_ERR_SHAPE;
   if (D != 128 || Hkv != H) return NC_ERR_SHAPE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return NC_ERR_ALIGN;

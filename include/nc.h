@@ -153,7 +153,8 @@ size_t nc_attention_workspace_bytes(int B, int T, int H, int Hkv, int D, int dty
  *   to the workspace; with 0 they are used as given.
  *   o_i = sum_j softmax_j(softmax_scale * qhat_i . khat_j) v_j over j <= i,
  *   i - j < window; window <= 0 or >= T means plain causal.
- * Requires D == 128, H_kv == H, 16-byte aligned pointers. */
+ * Requires D == 128, H_kv == H, softmax_scale > 0, eps >= 0, 16-byte aligned
+ * pointers (NC_ERR_SHAPE / NC_ERR_ARG / NC_ERR_ALIGN otherwise). */
 int nc_attention(const void* q, const void* k, const void* v, void* out, int B, int T, int H,
                  int Hkv, int D, int window, int rope_qknorm, float alpha, float softmax_scale,
                  float rope_base, float eps, int dtype, void* workspace, size_t workspace_bytes,

@@ -124,13 +124,15 @@ def test_attention_rejects_bad_arguments():
 
     def call(a):
         return lib.nc_attention(a["q"], a["k"], a["v"], a["o"], a["B"], a["T"], a["H"], a["Hkv"],
-                                a["D"], a["w"], a["rq"], 1.15, 0.088, 1e5, 1e-6, a["dt"], a["ws"],
-                                a["wsb"], None)
+                                a["D"], a["w"], a["rq"], 1.15, a.get("scale", 0.088), 1e5, 1e-6, a["dt"],
+                                a["ws"], a["wsb"], None)
     assert call(args(q=None)) == nc.STATUS_CODES["NC_ERR_ARG"]
     assert call(args(D=64)) == nc.STATUS_CODES["NC_ERR_SHAPE"]
     assert call(args(Hkv=2, H=4)) == nc.STATUS_CODES["NC_ERR_SHAPE"]
     assert call(args(T=0)) == nc.STATUS_CODES["NC_ERR_SHAPE"]
     assert call(args(dt=5)) == nc.STATUS_CODES["NC_ERR_ARG"]
+    assert call(args(scale=0.0)) == nc.STATUS_CODES["NC_ERR_ARG"]
+    assert call(args(scale=-1.0)) == nc.STATUS_CODES["NC_ERR_ARG"]
     assert call(args(k=C.c_void_p(a16.value + 2))) == nc.STATUS_CODES["NC_ERR_ALIGN"]
     assert call(args(rq=1)) == nc.STATUS_CODES["NC_ERR_WORKSPACE"]
     assert nc.nc_attention_workspace_bytes(2, 8, 4, 4, 128, "bf16", 1) >= 2 * 2 * 8 * 4 * 128 * 2
