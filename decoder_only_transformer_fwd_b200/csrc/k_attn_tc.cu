@@ -262,40 +262,52 @@ __global__ void __launch_bounds__(192, 1)
         ptx::tc_fence_after();
         float x[128];
         const uint32_t tS = tmem + (uint32_t)(s * 128) + lane_off;
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t u[32];
-          ptx::tmem_ld32(tS + (uint32_t)(cc * 32), u);
+        {
+          // four TMEM loads in flight behind one wait
+          uint32_t u0[32], u1[32], u2[32], u3[32];
+          ptx::tmem_ld32(tS, u0);
+          ptx::tmem_ld32(tS + 32, u1);
+          ptx::tmem_ld32(tS + 64, u2);
+          ptx::tmem_ld32(tS + 96, u3);
           ptx::tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) x[cc * 32 + i] = __uint_as_float(u[i]);
+          for (int i = 0; i < 32; ++i) {
+            x[i] = __uint_as_float(u0[i]);
+            x[32 + i] = __uint_as_float(u1[i]);
+            x[64 + i] = __uint_as_float(u2[i]);
+            x[96 + i] = __uint_as_float(u3[i]);
+          }
         }
         // visible keys of this row in this tile: columns [clo, chi]
         const int clo = qi - a.window + 1 - k0;
         const int chi = qi - k0;
-        float tmax = -INFINITY;
-        if (clo <= 0 && chi >= kK - 1) {
+        if (!(clo <= 0 && chi >= kK - 1)) {
 #pragma unroll
-          for (int i = 0; i < 128; ++i) tmax = fmaxf(tmax, x[i]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 128; ++i) {
-            x[i] = (i >= clo && i <= chi) ? x[i] : -INFINITY;
-            tmax = fmaxf(tmax, x[i]);
-          }
+          for (int i = 0; i < 128; ++i) x[i] = (i >= clo && i <= chi) ? x[i] : -INFINITY;
         }
+        // row max as a tree (short dependency chains: one softmax warp per scheduler)
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = x[k];
+#pragma unroll
+        for (int i = 8; i < 128; i += 8)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], x[i + k]);
+        const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         // lazy max (raw score units): move it only when it grows by more than 2^8 after scaling
         const bool rescale = (tmax - m_run) * c > kRescaleThreshold;
         const float m_new = rescale ? tmax : m_run;
         const float mc = (m_new == -INFINITY) ? 0.f : m_new * c;
-        float rsum = 0.f;
+        float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         uint32_t pk[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           const float p0 = ex2(fmaf(x[2 * i], c, -mc)), p1 = ex2(fmaf(x[2 * i + 1], c, -mc));
-          rsum += p0 + p1;
+          sm[i & 7] += p0 + p1;
           pk[i] = pack_bf16(p0, p1);
         }
+        const float rsum = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
         // P_{gj-1} and O through PV_{gj-1} are done before P is rewritten or O rescaled
         if (gj > 0 && !ptx::mbar_wait(bar(B_PV), (gj - 1) & 1, a.status)) { ok = false; break; }
         ptx::tc_fence_after();

@@ -60,39 +60,6 @@ struct TcArgs {
 
 __device__ __forceinline__ float bits2f(uint32_t u) { return __uint_as_float(u); }
 
-// EPI_STORE / EPI_RELU2 for 32 consecutive columns [n, n + 32) of row m:
-// bf16 conversion and one 64-byte store per thread.
-__device__ __forceinline__ void epi_chunk(const EpiParams& ep, const TcArgs& a, int m, int n,
-                                          const uint32_t (&r)[32], float&, float&, int) {
-  if (m >= a.M) return;
-  const bool relu2 = ep.mode == EPI_RELU2;
-  bf16* dst = reinterpret_cast<bf16*>(ep.out) + (size_t)m * ep.ldo + n;
-  if (n + 32 <= a.N) {
-    uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint32_t w[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float v0 = bits2f(r[q * 8 + 2 * e]), v1 = bits2f(r[q * 8 + 2 * e + 1]);
-        if (relu2) {
-          v0 = fmaxf(v0, 0.f);
-          v0 *= v0;
-          v1 = fmaxf(v1, 0.f);
-          v1 *= v1;
-        }
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
-        w[e] = *reinterpret_cast<uint32_t*>(&b2);
-      }
-      d4[q] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (n + i < a.N) epi_apply<bf16>(ep, m, n + i, bits2f(r[i]));
-  }
-}
-
 // Residual epilogues (EPI_RESID, EPI_BLOCK_END) for a 32-row x 32-column
 // chunk: the warp's rows arrive one per lane (TMEM lane = row); they are
 // transposed through shared memory so that for each row the warp reads and
@@ -139,6 +106,39 @@ __device__ __forceinline__ void epi_resid_chunk(const EpiParams& ep, const TcArg
           v = v - ep.beta * (ep.capture_bo ? v : zv[rr]);
       }
       ep.x[i] = v;
+    }
+  }
+  __syncwarp();
+}
+
+// EPI_STORE / EPI_RELU2 for a 32-row x 32-column chunk, coalesced: the rows
+// arrive one per lane, go through the shared-memory transpose buffer, and each
+// store instruction then writes two whole 64-byte bf16 row segments (lanes
+// 0..15 one row, 16..31 the next), two columns per lane.
+__device__ __forceinline__ void epi_store_chunk(const EpiParams& ep, const TcArgs& a, float* stage, int row0,
+                                                int n, const uint32_t (&r)[32], int lane, bool relu2) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    float v = __uint_as_float(r[i]);
+    if (relu2) {
+      v = fmaxf(v, 0.f);
+      v *= v;
+    }
+    stage[lane * 33 + i] = v;
+  }
+  __syncwarp();
+  const int cp = lane & 15;       // column pair
+  const int col = n + 2 * cp;
+  const bool col_ok = col < a.N;  // N is even: the pair is in or out together
+  bf16* base = reinterpret_cast<bf16*>(ep.out);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const int rr = 2 * k + (lane >> 4);
+    const int m = row0 + rr;
+    const float v0 = stage[rr * 33 + 2 * cp], v1 = stage[rr * 33 + 2 * cp + 1];
+    if (col_ok && m < a.M) {
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
+      *reinterpret_cast<__nv_bfloat162*>(base + (size_t)m * ep.ldo + col) = b2;
     }
   }
   __syncwarp();
@@ -320,8 +320,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs&
       if constexpr (MODE == EPI_RESID || MODE == EPI_BLOCK_END) {
         epi_resid_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, r, lane);
       } else {
-        float ce_sum = 0.f, ce_tgt = 0.f;
-        epi_chunk(ep, a, m, n_lo + c, r, ce_sum, ce_tgt, -1);
+        epi_store_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, r, lane, MODE == EPI_RELU2);
       }
     }
   }
