@@ -64,9 +64,11 @@ __device__ __forceinline__ float bits2f(uint32_t u) { return __uint_as_float(u);
 // chunk: the warp's rows arrive one per lane (TMEM lane = row); they are
 // transposed through shared memory so that for each row the warp reads and
 // writes one contiguous 128-byte segment of x (and x0 / x_bo), with all the
-// chunk's loads issued before its stores.
-__device__ __forceinline__ void epi_resid_chunk(const EpiParams& ep, const TcArgs& a, float* stage,
-                                                int row0, int n, const uint32_t (&r)[32], int lane) {
+// chunk's loads issued before its stores.  With ep.xb_out set, the new x is
+// also stored as bf16 (the next GEMM's A operand) and the return value is the
+// sum of squares of the lane's row over the chunk's 32 columns.
+__device__ __forceinline__ float epi_resid_chunk(const EpiParams& ep, const TcArgs& a, float* stage,
+                                                 int row0, int n, const uint32_t (&r)[32], int lane) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = __uint_as_float(r[i]);
   __syncwarp();
@@ -106,9 +108,33 @@ __device__ __forceinline__ void epi_resid_chunk(const EpiParams& ep, const TcArg
           v = v - ep.beta * (ep.capture_bo ? v : zv[rr]);
       }
       ep.x[i] = v;
+      stage[(h16 * 16 + rr) * 33 + lane] = v;
     }
   }
   __syncwarp();
+  float ss = 0.f;
+  if (ep.xb_out != nullptr) {
+    // row phase: lane t owns row row0 + t (columns past N or rows past M hold
+    // stale values but are never used: ss is only stored for valid rows and
+    // N is a multiple of 32 here)
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float v = stage[lane * 33 + i];
+      ss = fmaf(v, v, ss);
+    }
+    const int cp = lane & 15;
+    const int c2 = n + 2 * cp;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int rr = 2 * k + (lane >> 4);
+      const int m = row0 + rr;
+      const float v0 = stage[rr * 33 + 2 * cp], v1 = stage[rr * 33 + 2 * cp + 1];
+      if (c2 < a.N && m < a.M)
+        *reinterpret_cast<__nv_bfloat162*>(ep.xb_out + (size_t)m * ep.ldxb + c2) = __floats2bfloat162_rn(v0, v1);
+    }
+  }
+  __syncwarp();
+  return ss;
 }
 
 // EPI_STORE / EPI_RELU2 for a 32-row x 32-column chunk, coalesced: the rows
@@ -116,10 +142,11 @@ __device__ __forceinline__ void epi_resid_chunk(const EpiParams& ep, const TcArg
 // store instruction then writes two whole 64-byte bf16 row segments (lanes
 // 0..15 one row, 16..31 the next), two columns per lane.
 __device__ __forceinline__ void epi_store_chunk(const EpiParams& ep, const TcArgs& a, float* stage, int row0,
-                                                int n, const uint32_t (&r)[32], int lane, bool relu2) {
+                                                int n, const uint32_t (&r)[32], int lane, bool relu2,
+                                                float rscale) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    float v = __uint_as_float(r[i]);
+    float v = __uint_as_float(r[i]) * rscale;
     if (relu2) {
       v = fmaxf(v, 0.f);
       v *= v;
@@ -150,7 +177,7 @@ __device__ __forceinline__ void epi_store_chunk(const EpiParams& ep, const TcArg
 // ("The Mathematics of Karpathy's nanochat", §Rotary Position Embeddings,
 // §QK-Norm with Sharpening, §Value Embeddings.)
 __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& a, uint32_t taddr, int m,
-                                             int col0) {
+                                             int col0, float rscale) {
   const bool row_ok = m < a.M;
   bf16* out = reinterpret_cast<bf16*>(ep.out) + (size_t)m * ep.ldo + col0;
   if (col0 < ep.qk_cols) {
@@ -169,7 +196,8 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
 #pragma unroll
       for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(u[i]), __uint_as_float(u[i]), ss);
     }
-    const float rs = ep.qk_alpha / sqrtf(ss * (1.0f / 128.0f) + ep.eps);
+    // the head is rscale * acc: fold the row scale into the QK-norm factor
+    const float rs = rscale * ep.qk_alpha / sqrtf(ss * rscale * rscale * (1.0f / 128.0f) + ep.eps);
 #pragma unroll 1
     for (int c = 0; c < 2; ++c) {
       uint32_t u1[32], u2[32];
@@ -208,7 +236,19 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
     int tok = row_ok ? ep.tokens[m] : 0;
     tok = min(max(tok, 0), ep.vocab - 1);
     const bool mix = row_ok && ep.ve != nullptr;
-    const float g = mix ? ep.gate[(size_t)m * ep.n_kv_head + hv] : 0.f;
+    float g = 0.f;
+    if (mix) {
+      if (ep.gate != nullptr) {
+        g = ep.gate[(size_t)m * ep.n_kv_head + hv];
+      } else {
+        // gate from the normalised block input: rscale * x[m, :gate_c]
+        const float* xr = ep.x + (size_t)m * ep.ldx;
+        const float* wg = ep.gate_w + (size_t)hv * ep.gate_c;
+        float d = 0.f;
+        for (int c = 0; c < ep.gate_c; ++c) d = fmaf(xr[c], wg[c], d);
+        g = ep.gate_scale / (1.0f + __expf(-rscale * d));
+      }
+    }
     // the row's 128 value-embedding entries are gathered up front (one memory
     // round trip per row instead of one per chunk)
     uint4 e[16];
@@ -226,7 +266,7 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
       if (!row_ok) continue;
       float x[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(u[i]);
+      for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(u[i]) * rscale;
       if (mix) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -265,9 +305,19 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs&
   const int m = mb * kBM + row;
   const int c_lo = half * HALF;
   const int n_lo = nb * BN + c_lo;
+  // fused RMSNorm of the A operand: 1 / rms of this thread's row
+  float rscale = 1.f;
+  if constexpr (MODE == EPI_QKV || MODE == EPI_RELU2 || MODE == EPI_CE) {
+    if (ep.ss_in != nullptr && m < a.M) {
+      const float* sp = ep.ss_in + (size_t)m * ep.ss_in_parts;
+      float t = 0.f;
+      for (int j = 0; j < ep.ss_in_parts; ++j) t += sp[j];
+      rscale = 1.0f / sqrtf(t * ep.inv_c + ep.eps);
+    }
+  }
   if constexpr (MODE == EPI_QKV) {
     // one head (128 columns) per warp when BN = 256; with BN = 128 the first half does it
-    if (c_lo % 128 == 0 && n_lo < a.N) epi_qkv_head(ep, a, taddr + (uint32_t)c_lo, m, n_lo);
+    if (c_lo % 128 == 0 && n_lo < a.N) epi_qkv_head(ep, a, taddr + (uint32_t)c_lo, m, n_lo, rscale);
   } else if constexpr (MODE == EPI_CE) {
     int y = -1;
     if (m < a.M) {
@@ -288,7 +338,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs&
       float zh[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float q = ptx::rcp(ptx::ex2(__uint_as_float(r[i]) * k1) + 1.0f);
+        const float q = ptx::rcp(ptx::ex2(__uint_as_float(r[i]) * (rscale * k1)) + 1.0f);
         zh[i] = fmaf(c2, q, ep.cap);
         const float p = ptx::ex2(k2 * q);
         sum += (n + i < ep.vocab) ? p : 0.f;
@@ -312,16 +362,20 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs&
       if (y >= n_lo && y < n_lo + HALF) ep.ce_tgt[m] = tgt;
     }
   } else {
+    float ss = 0.f;
 #pragma unroll 1
     for (int c = 0; c < HALF; c += 32) {
       uint32_t r[32];
       ptx::tmem_ld32(taddr + (uint32_t)(c_lo + c), r);
       ptx::tmem_ld_wait();
       if constexpr (MODE == EPI_RESID || MODE == EPI_BLOCK_END) {
-        epi_resid_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, r, lane);
+        ss += epi_resid_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, r, lane);
       } else {
-        epi_store_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, r, lane, MODE == EPI_RELU2);
+        epi_store_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, r, lane, MODE == EPI_RELU2, rscale);
       }
+    }
+    if constexpr (MODE == EPI_RESID || MODE == EPI_BLOCK_END) {
+      if (ep.ss_out != nullptr && m < a.M) ep.ss_out[(size_t)m * ep.ss_parts + n_lo / HALF] = ss;
     }
   }
 }

@@ -34,7 +34,7 @@ template <typename T>
 __global__ void k_embed(const T* __restrict__ wte, const int32_t* __restrict__ tokens,
                         const float* __restrict__ smear_gate, int smear, int gc,
                         const float* __restrict__ lam0p, const float* __restrict__ mu0p, float eps, int T_, int C, int V, float* __restrict__ x, float* __restrict__ x0,
-                        int* status) {
+                        bf16* __restrict__ xb, float* __restrict__ ss, int ss_parts, int* status) {
   extern __shared__ float sh[];  // [2C] rows + [32] reduction
   float* cur = sh;
   float* prev = sh + C;
@@ -72,11 +72,22 @@ __global__ void k_embed(const T* __restrict__ wte, const int32_t* __restrict__ t
     g = sigmoidf_(d);
   }
   const float lam0 = *lam0p, mu0 = *mu0p;
+  float s3 = 0.f;
   for (int c = threadIdx.x; c < C; c += blockDim.x) {
     float xh = cur[c] * r1;
     if (has_prev) xh += g * (prev[c] * r2);
     x0[(size_t)m * C + c] = xh;
-    x[(size_t)m * C + c] = lam0 * xh + mu0 * xh;
+    const float v = lam0 * xh + mu0 * xh;
+    x[(size_t)m * C + c] = v;
+    if (xb != nullptr) {
+      xb[(size_t)m * C + c] = __float2bfloat16_rn(v);
+      s3 += v * v;
+    }
+  }
+  if (xb != nullptr) {
+    // the first block's norm input: sum of squares in slot 0, other slots 0
+    s3 = block_sum(s3, red);
+    for (int j = threadIdx.x; j < ss_parts; j += blockDim.x) ss[(size_t)m * ss_parts + j] = j == 0 ? s3 : 0.f;
   }
 }
 
@@ -317,16 +328,17 @@ __global__ void k_loss_mean(const float* loss, const int32_t* targets, int n, fl
 
 void launch_embed(const void* wte, const int32_t* tokens, const float* smear_gate, int smear,
                   int gate_channels, const float* lam0, const float* mu0, float eps, int B, int T, int C, int V,
-                  int act_bf16, float* x, float* x0, int* status, cudaStream_t st) {
+                  int act_bf16, float* x, float* x0, bf16* xb, float* ss, int ss_parts, int* status,
+                  cudaStream_t st) {
   LaunchScope scope_(KK_EMBED, st);
   const int M = B * T;
   const size_t sh = (size_t)(2 * C + 32) * sizeof(float);
   if (act_bf16)
     k_embed<bf16><<<M, 256, sh, st>>>((const bf16*)wte, tokens, smear_gate, smear, gate_channels, lam0,
-                                      mu0, eps, T, C, V, x, x0, status);
+                                      mu0, eps, T, C, V, x, x0, xb, ss, ss_parts, status);
   else
     k_embed<float><<<M, 256, sh, st>>>((const float*)wte, tokens, smear_gate, smear, gate_channels,
-                                       lam0, mu0, eps, T, C, V, x, x0, status);
+                                       lam0, mu0, eps, T, C, V, x, x0, xb, ss, ss_parts, status);
 }
 
 void launch_rmsnorm(const float* x, void* xn, int M, int C, float eps, int act_bf16,

@@ -105,7 +105,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
 struct Layout {
-  size_t x, x0, xbo, xn, qkv, o, h, gate, rcos, rsin, ce_sum, ce_tgt, logits, tok, tgt, loss;
+  size_t x, x0, xbo, xn, qkv, o, h, gate, ss, rcos, rsin, ce_sum, ce_tgt, logits, tok, tgt, loss;
   size_t total;
   int ce_tiles;
 };
@@ -145,6 +145,7 @@ Layout layout(const nc_config& c, int max_tokens) {
   L.o = take(M * c.n_head * D * esz);
   L.h = take(M * (size_t)c.mlp_hidden * esz);
   L.gate = take(M * c.n_kv_head * 4);
+  L.ss = take(M * (C / 64) * 4);  // per-row sums of squares of the residual, per column group
   L.rcos = take((size_t)c.max_T * D / 2 * 4);
   L.rsin = take((size_t)c.max_T * D / 2 * 4);
   L.ce_tiles = 2 * ((c.vocab_padded + 127) / 128);  // per (row, 128-or-256-column tile, half)
@@ -295,30 +296,55 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
   const size_t esz = bf ? 2 : 4;
 
   launch_rope_table(rcos, rsin, T, D, c.rope_base, st);
+  // tensor-core path: RMSNorm is fused into the GEMMs (producers write bf16(x)
+  // and per-row sums of squares, consumers scale their rows by 1 / rms)
+  const bool tc = bf && c.gemm_impl == 0;
+  float* ss = at<float>(ws, Lw.ss);
+  const int ss_parts = C / (gemm_tc_bn(C) / 2);
+  bf16* xb = tc ? static_cast<bf16*>(xn) : nullptr;
   launch_embed(p->wte, tokens, p->smear_gate, c.smear && c.gate_channels > 0, c.gate_channels,
-               p->resid_lambdas, p->x0_lambdas, c.eps, B, T, C, V, bf, x, x0, d.status, st);
+               p->resid_lambdas, p->x0_lambdas, c.eps, B, T, C, V, bf, x, x0, xb, tc ? ss : nullptr,
+               ss_parts, d.status, st);
+  // consumer / producer settings of the fused norm
+  auto norm_in = [&](EpiParams& e) {
+    e.ss_in = ss;
+    e.ss_in_parts = ss_parts;
+    e.inv_c = 1.0f / (float)C;
+    e.eps = c.eps;
+  };
+  auto norm_out = [&](EpiParams& e) {
+    e.xb_out = xb;
+    e.ldxb = C;
+    e.ss_out = ss;
+    e.ss_parts = ss_parts;
+  };
 
   for (int l = 0; l < c.n_layer; ++l) {
     const nc_layer_params& lp = p->layer[l];
     const bool ve = c.has_ve[l] != 0;
     // attention sub-block
-    launch_rmsnorm(x, xn, M, C, c.eps, bf, ve ? lp.ve_gate : nullptr, Hkv, c.gate_channels,
-                   c.ve_gate_scale, ve ? gate : nullptr, st);
-    const bool tc = bf && c.gemm_impl == 0;
+    if (!tc)
+      launch_rmsnorm(x, xn, M, C, c.eps, bf, ve ? lp.ve_gate : nullptr, Hkv, c.gate_channels,
+                     c.ve_gate_scale, ve ? gate : nullptr, st);
     EpiParams e = epi(tc ? EPI_QKV : EPI_STORE);
     e.out = qkv;
     e.ldo = nqkv;
     if (tc) {
-      // RoPE + QK-norm and the value-embedding mix run on the fp32 accumulator
+      // RoPE + QK-norm, the value-embedding gate and mix run on the fp32 accumulator
+      norm_in(e);
       e.T = T;
       e.qk_cols = (H + Hkv) * D;
       e.rope_cos = rcos;
       e.rope_sin = rsin;
       e.qk_alpha = c.qk_alpha;
-      e.eps = c.eps;
       e.tokens = tokens;
       e.ve = ve ? lp.ve : nullptr;
-      e.gate = gate;
+      e.gate = nullptr;
+      e.gate_w = lp.ve_gate;
+      e.gate_c = c.gate_channels;
+      e.gate_scale = c.ve_gate_scale;
+      e.x = x;
+      e.ldx = C;
       e.n_kv_head = Hkv;
       e.vocab = V;
     }
@@ -340,12 +366,14 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
     e = epi(EPI_RESID);
     e.x = x;
     e.ldx = C;
+    if (tc) norm_out(e);
     if (!gemm(c, d, o, H * D, lp.w_o, H * D, M, C, H * D, e, st)) return NC_ERR_CUDA;
     // MLP sub-block
-    launch_rmsnorm(x, xn, M, C, c.eps, bf, nullptr, 0, 0, 0.f, nullptr, st);
+    if (!tc) launch_rmsnorm(x, xn, M, C, c.eps, bf, nullptr, 0, 0, 0.f, nullptr, st);
     e = epi(EPI_RELU2);
     e.out = h;
     e.ldo = c.mlp_hidden;
+    if (tc) norm_in(e);
     if (!gemm(c, d, xn, C, lp.w_fc1, C, M, c.mlp_hidden, C, e, st)) return NC_ERR_CUDA;
     e = epi(EPI_BLOCK_END);
     e.x = x;
@@ -361,15 +389,16 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
       e.end_kind = c.backout_layer >= 0 ? 2 : 0;
       e.beta = p->backout_lambda;
     }
+    if (tc) norm_out(e);  // the next block's (or the head's) normalised input
     if (!gemm(c, d, h, c.mlp_hidden, lp.w_fc2, c.mlp_hidden, M, C, c.mlp_hidden, e, st)) return NC_ERR_CUDA;
   }
 
   // final norm, head, softcap, cross-entropy
-  launch_rmsnorm(x, xn, M, C, c.eps, bf, nullptr, 0, 0, 0.f, nullptr, st);
-  if (bf && c.gemm_impl == 0) {
+  if (tc) {
     const int bn = gemm_tc_bn(c.vocab_padded);
     const int tiles = 2 * ((c.vocab_padded + bn - 1) / bn);  // two epilogue halves per tile
     EpiParams e = epi(EPI_CE);
+    norm_in(e);
     e.cap = c.softcap;
     e.vocab = V;
     e.logits = out_logits;
@@ -381,6 +410,7 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
     if (!gemm(c, d, xn, C, p->lm_head, C, M, c.vocab_padded, C, e, st)) return NC_ERR_CUDA;
     launch_ce_combine(e.ce_sum, e.ce_tgt, tiles, c.softcap, targets, M, V, out_loss, d.status, st);
   } else {
+    launch_rmsnorm(x, xn, M, C, c.eps, bf, nullptr, 0, 0, 0.f, nullptr, st);
     float* logits = out_logits ? out_logits : at<float>(ws, Lw.logits);
     EpiParams e = epi(EPI_SOFTCAP);
     e.cap = c.softcap;

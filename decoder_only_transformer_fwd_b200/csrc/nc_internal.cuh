@@ -87,14 +87,34 @@ struct EpiParams {
   float qk_alpha, eps;
   const int32_t* tokens;  // [M]
   const void* ve;     // [V, H_kv D] or NULL
-  const float* gate;  // [M, H_kv]
+  const float* gate;  // [M, H_kv] precomputed gates (CUDA-core path), or NULL
   int n_kv_head;
+  // RMSNorm fused into the tcgen05 GEMMs ("The Mathematics of Karpathy's
+  // nanochat", §RMS Normalization): RMSNorm(x) W^T = (bf16(x) W^T) / rms(x).
+  // Producer side (EPI_RESID / EPI_BLOCK_END): besides the fp32 x also write
+  // xb = bf16(x) and, per row, the sum of squares of the new x over each
+  // BN/2-column group: ss_out[m, n / (BN/2)].
+  bf16* xb_out;
+  int ldxb;
+  float* ss_out;
+  int ss_parts;       // groups per row (C / (BN/2))
+  // Consumer side (EPI_QKV / EPI_RELU2 / EPI_CE, A operand = xb): each row is
+  // scaled by 1 / sqrt(sum_j ss_in[m, j] / C + eps) before the epilogue op.
+  const float* ss_in;
+  int ss_in_parts;
+  float inv_c;        // 1 / C
+  // value-embedding gate inside the QKV epilogue (when gate == NULL):
+  // g = gate_scale * sigmoid(rstd * x[m, :gate_c] . gate_w[h, :gate_c])
+  const float* gate_w;
+  int gate_c;
+  float gate_scale;
 };
 
 // launchers (host functions), all asynchronous on `st`
 void launch_embed(const void* wte, const int32_t* tokens, const float* smear_gate, int smear,
                   int gate_channels, const float* lam0, const float* mu0, float eps, int B, int T, int C, int V,
-                  int act_bf16, float* x, float* x0, int* status, cudaStream_t st);
+                  int act_bf16, float* x, float* x0, bf16* xb, float* ss, int ss_parts, int* status,
+                  cudaStream_t st);
 void launch_rmsnorm(const float* x, void* xn, int M, int C, float eps, int act_bf16,
                     const float* ve_gate, int Hkv, int gate_channels, float gate_scale, float* gate_out,
                     cudaStream_t st);
