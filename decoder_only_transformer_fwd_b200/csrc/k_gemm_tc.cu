@@ -532,6 +532,190 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// CTA-pair variant (cluster of 2, tcgen05 cta_group::2): a 256 x 256 output
+// tile per pair.  Each CTA loads its own 128 rows of A and its own 128 rows
+// (half) of B per k-slice, so a CTA moves 32 KB instead of 48 KB per 128 x 256
+// x 64 step; the even CTA issues M = 256 MMAs over both CTAs' shared memory
+// and each CTA's TMEM receives its 128 rows.  Both CTAs' copies complete on
+// the even CTA's "full" barrier; MMA completion is multicast to both CTAs'
+// "empty"/"accumulator full" barriers; both CTAs' epilogues arrive on the even
+// CTA's "accumulator empty" barrier.  No TMA multicast: every CTA reads its
+// own operand slices.
+// ---------------------------------------------------------------------------
+struct PairCfg {
+  static constexpr int BN = 256;
+  static constexpr int STAGES = 6;
+  static constexpr int A_BYTES = kBM * kBK * 2;       // 16 KB: this CTA's 128 rows of A
+  static constexpr int B_BYTES = (BN / 2) * kBK * 2;  // 16 KB: this CTA's 128 rows of B
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int NBARS = 2 * STAGES + 5;
+  static constexpr int STAGE_FLOATS = 32 * 33;
+  static constexpr int EPI_BYTES = kEpiWarps * STAGE_FLOATS * 4;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256 + EPI_BYTES;
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const TcArgs a, const EpiParams ep) {
+  using Cf = PairCfg;
+  constexpr int BN = Cf::BN;
+  constexpr int S = Cf::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * Cf::STAGE_BYTES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + Cf::NBARS);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* epi_stage = reinterpret_cast<float*>(smem + S * Cf::STAGE_BYTES + 256);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const bool leader = rank == 0;
+  const uint32_t bar0 = ptx::smem_u32(bars);
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (S + s); };
+  auto tfull = [&](int i) { return bar0 + 8u * (2 * S + i); };
+  auto tempty = [&](int i) { return bar0 + 8u * (2 * S + 2 + i); };
+  const uint32_t mma_done = bar0 + 8u * (2 * S + 4);
+  auto sA = [&](int s) { return ptx::smem_u32(smem + s * Cf::STAGE_BYTES); };
+  auto sB = [&](int s) { return ptx::smem_u32(smem + s * Cf::STAGE_BYTES + Cf::A_BYTES); };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(full(s), 1);
+      ptx::mbar_init(empty(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(tfull(i), 1);
+      ptx::mbar_init(tempty(i), 2 * kEpiWarps);  // both CTAs' epilogue warps (used on the even CTA)
+    }
+    ptx::mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::fence_proxy_async_smem();
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc2(ptx::smem_u32(tmem_slot), Cf::TMEM_COLS);
+    ptx::tmem_relinquish2();
+    ptx::tc_fence_before();
+  }
+  // barriers of both CTAs are initialised before any cross-CTA signal
+  ptx::cluster_sync_all();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int nk = a.K / kBK;
+  const int tiles_mp = (a.M + 2 * kBM - 1) / (2 * kBM);
+  const int num_pt = tiles_mp * a.tiles_n;
+  const int cid = (int)ptx::cluster_id_x(), ncl = (int)ptx::nclusters_x();
+
+  if (warp == 0) {
+    if (ptx::elect_one()) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      int stage = 0;
+      uint32_t ph = 0, issued = 0, par = 0;
+      for (int pt = cid; pt < num_pt; pt += ncl) {
+        const int mbp = pt % tiles_mp, nb = pt / tiles_mp;
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (*abort_flag || !ptx::mbar_wait_cluster(empty(stage), ph ^ 1, a.status)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          if (leader) ptx::mbar_arrive_expect_tx(full(stage), 2 * Cf::STAGE_BYTES);
+          const uint32_t fb = ptx::mapa(full(stage), 0);
+          ptx::tma_load_2d_pair(sA(stage), &tmA, fb, kb * kBK, mbp * 2 * kBM + (int)rank * kBM);
+          ptx::tma_load_2d_pair(sB(stage), &tmB, fb, kb * kBK, nb * BN + (int)rank * (BN / 2));
+          issued |= 1u << stage;
+          par = (par & ~(1u << stage)) | (ph << stage);
+          if (++stage == S) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+      // this CTA's copies have landed (and been consumed) before it may exit
+      for (int s = 0; s < S; ++s)
+        if (issued & (1u << s)) ptx::mbar_wait_cluster(empty(s), (par >> s) & 1, a.status);
+    }
+  } else if (warp == 1) {
+    if (leader && ptx::elect_one()) {
+      // ---------------- MMA issuer (even CTA) ----------------
+      constexpr uint32_t idesc = ptx::idesc_bf16(2 * kBM, BN);
+      int stage = 0, acc = 0;
+      uint32_t ph = 0, aph = 0;
+      for (int pt = cid; pt < num_pt; pt += ncl) {
+        if (*abort_flag || !ptx::mbar_wait_cluster(tempty(acc), aph ^ 1, a.status)) {
+          *abort_flag = 1;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(acc * BN);
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (*abort_flag || !ptx::mbar_wait_cluster(full(stage), ph, a.status)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint64_t da = ptx::desc_kmajor_sw128(sA(stage));
+          const uint64_t db = ptx::desc_kmajor_sw128(sB(stage));
+#pragma unroll
+          for (int k = 0; k < kBK / kUK; ++k)
+            ptx::mma_bf16_ss2(d, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          ptx::mma_commit2_mc(empty(stage), 0x3);
+          if (++stage == S) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        ptx::mma_commit2_mc(tfull(acc), 0x3);
+        acc ^= 1;
+        if (acc == 0) aph ^= 1;
+      }
+      // all MMAs have completed before either CTA releases its TMEM
+      ptx::mma_commit2(mma_done);
+      ptx::mbar_wait_cluster(mma_done, 0, a.status);
+    }
+  } else {
+    // ---------------- epilogue (both CTAs, warps 2 .. 2 + kEpiWarps - 1) ----------------
+    const int ew = warp - 2;
+    const int g = warp & 3;
+    const int half = ew >> 2;
+    float* stage = epi_stage + ew * Cf::STAGE_FLOATS;
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int pt = cid; pt < num_pt; pt += ncl) {
+      const int mbp = pt % tiles_mp, nb = pt / tiles_mp;
+      if (*abort_flag || !ptx::mbar_wait_cluster(tfull(acc), aph, a.status)) {
+        *abort_flag = 1;
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t taddr = tmem + ((uint32_t)(g * 32) << 16) + (uint32_t)(acc * BN);
+      epilogue_tile<BN, MODE>(ep, a, taddr, mbp * 2 + (int)rank, nb, g, half, lane, stage);
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa(tempty(acc), 0));
+      acc ^= 1;
+      if (acc == 0) aph ^= 1;
+    }
+  }
+  __syncthreads();
+  ptx::cluster_sync_all();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc2(tmem, Cf::TMEM_COLS);
+  }
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
@@ -558,6 +742,41 @@ void launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, 
     cudaFuncSetAttribute(k_gemm_tc<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<BN>::SMEM);
   });
   k_gemm_tc<BN, MODE><<<grid, kThreads, TcCfg<BN>::SMEM, st>>>(ta, tb, a, ep);
+}
+
+template <int MODE>
+void launch_pair_mode(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep,
+                      int nclusters, cudaStream_t st) {
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaFuncSetAttribute(k_gemm_tc2<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM);
+  });
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * nclusters, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = PairCfg::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, k_gemm_tc2<MODE>, ta, tb, a, ep);
+}
+
+bool launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep, int nclusters,
+                 cudaStream_t st) {
+  switch (ep.mode) {
+    case EPI_STORE: launch_pair_mode<EPI_STORE>(ta, tb, a, ep, nclusters, st); return true;
+    case EPI_RELU2: launch_pair_mode<EPI_RELU2>(ta, tb, a, ep, nclusters, st); return true;
+    case EPI_RESID: launch_pair_mode<EPI_RESID>(ta, tb, a, ep, nclusters, st); return true;
+    case EPI_BLOCK_END: launch_pair_mode<EPI_BLOCK_END>(ta, tb, a, ep, nclusters, st); return true;
+    case EPI_CE: launch_pair_mode<EPI_CE>(ta, tb, a, ep, nclusters, st); return true;
+    case EPI_QKV: launch_pair_mode<EPI_QKV>(ta, tb, a, ep, nclusters, st); return true;
+    default: return false;
+  }
 }
 
 template <int BN>
@@ -608,8 +827,26 @@ bool make_tmap_4d(CUtensorMap* map, const void* ptr, const uint64_t (&dims)[4],
 int gemm_tc_bn(int N) { return (N % 256 == 0) ? 256 : 128; }
 
 bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int N, int K,
-                    const EpiParams& ep, int* status, int num_sms, cudaStream_t st) {
+                    const EpiParams& ep, int* status, int num_sms, cudaStream_t st, bool pair) {
   const int BN = gemm_tc_bn(N);
+  if (pair && BN == 256 && num_sms >= 2) {
+    // CTA pairs: each CTA loads 128 rows of A and 128 rows of B per k-slice
+    CUtensorMap ta, tb;
+    if (!make_tmap_2d(&ta, A, M, K, lda, kBM, kBK)) return false;
+    if (!make_tmap_2d(&tb, Bm, N, K, ldb, BN / 2, kBK)) return false;
+    TcArgs a;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.tiles_m = (M + kBM - 1) / kBM;
+    a.tiles_n = N / BN;
+    a.num_tiles = a.tiles_m * a.tiles_n;
+    a.status = status;
+    const int num_pt = ((M + 2 * kBM - 1) / (2 * kBM)) * a.tiles_n;
+    const int ncl = num_pt < num_sms / 2 ? num_pt : num_sms / 2;
+    LaunchScope scope_(KK_GEMM_TC, st);
+    return launch_pair(ta, tb, a, ep, ncl, st);
+  }
   CUtensorMap ta, tb;
   if (!make_tmap_2d(&ta, A, M, K, lda, kBM, kBK)) return false;
   if (!make_tmap_2d(&tb, Bm, N, K, ldb, BN, kBK)) return false;

@@ -169,7 +169,8 @@ T* at(void* base, size_t off) {
 bool gemm(const nc_config& c, const DevInfo& d, const void* A, int lda, const void* B, int ldb, int M,
           int N, int K, const EpiParams& ep, cudaStream_t st) {
   if (c.dtype == NC_BF16 && c.gemm_impl == 0)
-    return launch_gemm_tc((const bf16*)A, lda, (const bf16*)B, ldb, M, N, K, ep, d.status, d.num_sms, st);
+    return launch_gemm_tc((const bf16*)A, lda, (const bf16*)B, ldb, M, N, K, ep, d.status, d.num_sms, st,
+                          c.gemm_pair != 0);
   launch_gemm_simt(A, lda, B, ldb, M, N, K, c.dtype == NC_BF16, ep, st);
   return true;
 }
@@ -228,6 +229,7 @@ int nc_init_config(nc_config* cfg, int depth, int max_T, int dtype, const char* 
   cfg->gate_channels = 12;
   cfg->smear = 1;
   cfg->gemm_impl = 0;
+  cfg->gemm_pair = 1;
   cfg->attn_impl = 0;
   cfg->qk_alpha = 1.15f;
   cfg->softmax_scale = 1.0f / sqrtf((float)head_dim);

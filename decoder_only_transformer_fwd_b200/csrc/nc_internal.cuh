@@ -142,8 +142,9 @@ void launch_attn_simt(const void* q, const void* k, const void* v, int ldq, int 
 
 // tcgen05 GEMM (bf16 only).  Returns false if the tensor maps cannot be built.
 int gemm_tc_bn(int N);  // output tile width the tcgen05 GEMM uses for N columns
+// pair = true selects the CTA-pair (cta_group::2) kernel when N % 256 == 0.
 bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int N, int K,
-                    const EpiParams& ep, int* status, int num_sms, cudaStream_t st);
+                    const EpiParams& ep, int* status, int num_sms, cudaStream_t st, bool pair);
 // tcgen05 attention (bf16 only)
 bool launch_attn_tc(const bf16* q, const bf16* k, const bf16* v, int ldq, int ldk, int ldv, bf16* o,
                     int ldo, int B, int T, int H, int Hkv, int window, float scale, int* status,

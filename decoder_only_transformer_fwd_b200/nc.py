@@ -28,7 +28,7 @@ class nc_config(C.Structure):
                 ("dtype", C.c_int), ("window", C.c_int * NC_MAX_LAYERS),
                 ("has_ve", C.c_int * NC_MAX_LAYERS), ("backout_layer", C.c_int),
                 ("gate_channels", C.c_int), ("smear", C.c_int), ("gemm_impl", C.c_int),
-                ("attn_impl", C.c_int), ("qk_alpha", C.c_float), ("softmax_scale", C.c_float),
+                ("attn_impl", C.c_int), ("gemm_pair", C.c_int), ("qk_alpha", C.c_float), ("softmax_scale", C.c_float),
                 ("rope_base", C.c_float), ("eps", C.c_float), ("softcap", C.c_float),
                 ("ve_gate_scale", C.c_float)]
 

@@ -60,13 +60,15 @@ def test_d1_fp32_full():
     _compare(loss, ref_loss, logits, ref_logits, "fp32")
 
 
-@pytest.mark.parametrize("gemm_impl,attn_impl", [(0, 0), (1, 1)])
-def test_d4_bf16_full(gemm_impl, attn_impl):
+@pytest.mark.parametrize("gemm_impl,attn_impl,gemm_pair", [(0, 0, 1), (0, 0, 0), (1, 1, 0)])
+def test_d4_bf16_full(gemm_impl, attn_impl, gemm_pair):
+    """gemm_pair selects the CTA-pair (cta_group::2) or the single-CTA tcgen05 GEMM."""
     w = synth.WORKLOADS["d4"]
     seed = synth.SEED_BASE + w["index"]
     cfg, ocfg, p, tok, tgt = make_case(w["depth"], w["B"], w["T"], w["short"], w["dtype"], seed)
     cfg.gemm_impl = gemm_impl
     cfg.attn_impl = attn_impl
+    cfg.gemm_pair = gemm_pair
     loss, logits, rc, _ = run_gpu(cfg, p, tok, tgt, want_logits=True)
     assert rc == 0
     rows = [0, 3]
