@@ -192,6 +192,15 @@ int check_launch(const char* what) {
 }
 
 }  // namespace
+
+// The device status word of the current device (for launchers in other files).
+bool status_word(int** out) {
+  DevInfo d;
+  if (!dev_info(&d)) return false;
+  *out = d.status;
+  return true;
+}
+
 }  // namespace nc
 
 using namespace nc;

@@ -73,6 +73,10 @@ _SIGS = {
     "nc_set_launch_timing": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_uint]),
     "nc_launch_timing_count": (C.c_int, []),
     "nc_kernel_name": (C.c_char_p, [C.c_int]),
+    "nc_attention_noalloc": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int,
+                                       C.c_int, C.c_int, C.c_int, C.c_int, C.c_float, C.c_float, C.c_float,
+                                       C.c_float, C.c_int, C.c_void_p]),
+    "nc_attention_noalloc_max_bytes": (C.c_size_t, []),
 }
 
 KERNEL_KINDS = ["embed_norm_smear", "rmsnorm", "rope_table", "rope_qknorm", "gemm_tcgen05",

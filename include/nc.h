@@ -161,6 +161,33 @@ int nc_attention(const void* q, const void* k, const void* v, void* out, int B, 
                  float rope_base, float eps, int dtype, void* workspace, size_t workspace_bytes,
                  void* stream);
 
+/* nc_attention without a workspace, for callers that have no way to obtain
+ * device memory for scratch: code embedded in a host program whose memory is
+ * managed by a runtime that does not expose an allocator, or a latency-bound
+ * loop that must not call cudaMalloc (it can synchronise the device).  There is
+ * no counterpart on the pages: this is a deployment convenience.
+ *   Computes exactly what nc_attention(q, k, v, out, B, T, H, Hkv, D, window,
+ *   rope_qknorm = 1, alpha, softmax_scale, rope_base, eps, dtype, ...) does,
+ *   with the same argument meanings and requirements.
+ *   Scratch: one array of nc_attention_noalloc_max_bytes() bytes (32 MiB) in
+ *   device memory, defined in the library, held by every GPU that loads the
+ *   library until the process exits.  Calls whose RoPE tables plus normalised
+ *   q and k do not fit (about 2 * T * 256 + 2 * B * T * H * 128 * sizeof(dtype)
+ *   bytes) return NC_ERR_WORKSPACE and launch nothing.  The call allocates and
+ *   frees nothing itself.
+ *   The first call on a device looks up the array's device address with that
+ *   device current (host code cannot use the array's name as a device pointer);
+ *   make that first call before any stream capture.
+ *   All calls on a device share the array: every byte a call reads from it is
+ *   written earlier by the same call, but calls that overlap on the GPU (other
+ *   streams, or other threads) race on it and must be serialised by the caller. */
+int nc_attention_noalloc(const void* q, const void* k, const void* v, void* out, int B, int T, int H,
+                         int Hkv, int D, int window, float alpha, float softmax_scale, float rope_base,
+                         float eps, int dtype, void* stream);
+
+/* Size in bytes of nc_attention_noalloc's fixed scratch array. */
+size_t nc_attention_noalloc_max_bytes(void);
+
 /* Synchronise `stream`, read the device status word (an OR of
  * 1 << NC_ERR_DATA and 1 << NC_ERR_TIMEOUT bits set by kernels since the last
  * read), clear it, and return NC_OK, NC_ERR_DATA or NC_ERR_TIMEOUT (timeout
