@@ -105,7 +105,9 @@ def dist_setup():
 
 
 def workload_desc(cfg, B, T):
-    return (f"d24 nanochat GPT forward+CE: depth {cfg.n_layer}, C={cfg.n_embd}, {cfg.n_head}x{cfg.head_dim} "
+    head = "d24 nanochat GPT forward+CE" if cfg.n_layer == 24 else \
+        f"profiling case: d24 dimensions cut to {cfg.n_layer} blocks, forward+CE"
+    return (f"{head}: depth {cfg.n_layer}, C={cfg.n_embd}, {cfg.n_head}x{cfg.head_dim} "
             f"heads, MLP {cfg.mlp_hidden} ReLU^2, V={cfg.vocab}, SSSL windows "
             f"{cfg.window[0]}/{cfg.max_T} (last block full), value embeddings on odd blocks, "
             f"backout from block {cfg.backout_layer}, softcap {cfg.softcap:g}, B={B}, T={T}")
@@ -222,6 +224,13 @@ def run_ours(args):
     M = B * T
     seed = synth.SEED_BASE + w["index"]
     cfg = nc.nc_init_config(w["depth"], T, "bf16", "SSSL", w["short"], -1)
+    if args.layers:
+        # a shorter stack of the same blocks, for profiler captures of single launches
+        L = args.layers
+        cfg.n_layer = L
+        cfg.window[L - 1] = T
+        cfg.backout_layer = L // 2
+        args.no_cpu_baseline = True
     ve_layers = [l for l in range(cfg.n_layer) if cfg.has_ve[l]]
     params = synth.params(seed, n_layer=cfg.n_layer, n_embd=cfg.n_embd, n_head=cfg.n_head,
                           n_kv_head=cfg.n_kv_head, head_dim=cfg.head_dim, vocab=cfg.vocab,
@@ -376,9 +385,13 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=1024)
     ap.add_argument("--rows", type=int, default=0, help="rows per step (default: the workload's B = 4)")
     ap.add_argument("--no-attention-sweep", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling only: keep the first N blocks of the d24 stack (1..24)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if not 0 <= args.layers <= 24:
+        ap.error("--layers must be in 0..24 (0: all 24 blocks)")
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

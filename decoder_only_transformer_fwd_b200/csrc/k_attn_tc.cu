@@ -5,27 +5,35 @@
 // with Sliding Window: query i sees key j iff j <= i and i - j < w;
 // o_i = sum_j softmax_j(scale q_i . k_j) v_j.
 //
-// Persistent: one CTA per SM walks work items (one 128-query tile of one
-// head each), heaviest first (the last query tiles see the most keys).
-//   warp 0      TMA: the item's Q tile, then its K and V tiles (128 keys) into
-//               a two-stage ring that runs on across items; only key tiles
-//               that hold a visible key are visited, so masked work is
-//               skipped tile by tile;
-//   warp 1      TMEM allocation (512 columns: S0 | S1 | O0 | O1) and one
-//               thread issuing tcgen05.mma: S_j = Q K_j^T (M = N = 128, K = 16
-//               steps over D), then O += P_j V_j with V read as an MN-major
-//               operand straight from the TMA tile;
-//   warps 2..5  online softmax, one query row per thread (its TMEM lane):
-//               row max on the raw scores, p = 2^(s c - m c) with the scale c
-//               folded into one FMA, P_j to shared memory as bf16 in the
-//               128-byte-swizzled K-major layout the MMA reads; the running
-//               max moves (and O is rescaled through TMEM) only when it grows
-//               by more than 2^8, so p <= 256; finally O / l to global memory.
-// S_{j+1} is computed while the softmax works on S_j, and the two O buffers
-// let the output of item i drain while the MMAs of item i + 1 run.  All
-// barrier phases are counted over the CTA's whole sequence of tiles.  Every
-// wait is bounded; on a timeout the CTA records NC_ERR_TIMEOUT and returns
-// after its copies and MMAs have landed.
+// Persistent: one CTA per SM walks work items, heaviest first.  An item is a
+// pair of adjacent 128-query tiles (A, B) of one head, which share one stream
+// of 128-key K/V tiles:
+//   warps 0..3  softmax of tile A, one query row per thread (its TMEM lane);
+//   warps 4..7  softmax of tile B;
+//   warp 8      TMA: the item's two Q tiles, then K_t and V_t for every key
+//               tile t that holds a key visible to A or B, into a 5-slot ring
+//               (32 KB slots) that runs on across items;
+//   warp 9      TMEM allocation (512 columns: S_A | S_B | O_A | O_B) and one
+//               thread issuing tcgen05.mma: S_g = Q_g K_t^T (M = N = 128,
+//               K = 16 steps over D) and O_g += P_g V_t, with P_g read from
+//               tensor memory and V read as an MN-major operand straight from
+//               the TMA tile;
+//   warps 10,11 idle (they complete the TMA/MMA warpgroup, which hands its
+//               registers to the softmax warpgroups).
+// P_g overwrites the first 64 columns of S_g as packed bf16 (two keys per
+// 32-bit column), so no shared memory holds P and the ring gets five slots.
+// For each key tile the MMA warp issues, per group, PV_g(t) once P_g(t) is
+// written and then S_g(t+1) = Q_g K_{t+1}^T into the same columns; the tensor
+// core runs them in issue order, so S_g(t+1) never overwrites P_g(t) before
+// it has been read, and "S_g(t+1) ready" also means "O_g holds PV_g(t)".  One
+// group's exponentials overlap the other group's MMAs.  A group skips key
+// tiles that hold no key visible to it, so masked work is skipped tile by
+// tile.  Softmax: row max on the raw scores, p = 2^(s c - m c) with the scale
+// c folded into one FMA; the running max moves (and O is rescaled through
+// TMEM) only when it grows by more than 2^8, so p <= 256.  All barrier phases
+// are counted over the CTA's whole sequence.  Every wait is bounded; on a
+// timeout the CTA records NC_ERR_TIMEOUT and returns after its copies and
+// MMAs have landed.
 #include <mutex>
 
 #include "nc_internal.cuh"
@@ -39,45 +47,66 @@ bool make_tmap_2d(CUtensorMap* map, const void* ptr, int rows, int cols, int ld,
 namespace {
 
 constexpr int kQ = 128, kK = 128, kD = 128;
-constexpr int TILE_BYTES = kQ * kD * 2;   // 32 KB: a 128 x 128 bf16 tile (two 64-column boxes)
-constexpr int BOX_BYTES = TILE_BYTES / 2; // 16 KB: 128 rows x 64 columns
-constexpr int STAGES = 2;
-// shared memory: Q | K[2] | V[2] | P | barriers
+constexpr int TILE_BYTES = kQ * kD * 2;    // 32 KB: a 128 x 128 bf16 tile (two 64-column boxes)
+constexpr int BOX_BYTES = TILE_BYTES / 2;  // 16 KB: 128 rows x 64 columns
+constexpr int SLOTS = 5;
+// shared memory: Q_A | Q_B | slot[5] | barriers
 constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + TILE_BYTES;
-constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
-constexpr int OFF_P = OFF_V + STAGES * TILE_BYTES;
-constexpr int OFF_BAR = OFF_P + TILE_BYTES;
+constexpr int OFF_SLOT = OFF_Q + 2 * TILE_BYTES;
+constexpr int OFF_BAR = OFF_SLOT + SLOTS * TILE_BYTES;
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
-constexpr uint32_t TMEM_COLS = 512;  // S0 | S1 | O0 | O1
+constexpr uint32_t TMEM_COLS = 512;  // S_A | S_B | O_A | O_B
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// warps 0..3: softmax of tile A, 4..7: softmax of tile B, 8: TMA, 9: MMA, 10..11: idle
+constexpr int kThreads = 384;
+constexpr int kWarpTma = 8, kWarpMma = 9;
+// registers: launched at 168 per thread (65536 / 384, rounded down to 8);
+// the TMA/MMA warpgroup drops to 104 and the two softmax warpgroups rise to
+// 200: 2 * 128 * 200 + 128 * 104 = 64512 = 384 * 168
+constexpr int kRegsLow = 104, kRegsHigh = 200;
+static_assert(2 * 128 * kRegsHigh + 128 * kRegsLow <= kThreads * 168, "register split");
 
 struct AttnArgs {
   int B, T, H, Hkv, window;
   int ldo;
-  int n_qblocks, n_items;
+  int n_qblocks, n_pairs, n_items;
   float scale_log2;  // softmax_scale * log2(e)
   bf16* o;
   int* status;
 };
 
 struct Item {
-  int b, h, q0, kt_lo, n_tiles;
+  int b, h, q0;  // q0: first query of tile A; tile B starts at q0 + 128
+  int has_b;
+  int lo0, hi0;  // key tiles visible to tile A
+  int lo1, hi1;  // key tiles visible to tile B (when has_b)
+  int lo, hi;    // their union, which is contiguous
 };
 
-// item i: query tile n_qblocks - 1 - i / (B H) (heaviest first), head-batch i % (B H)
+__device__ __forceinline__ int first_key_tile(const AttnArgs& a, int q0) { return max(0, q0 - a.window + 1) / kK; }
+__device__ __forceinline__ int last_key_tile(const AttnArgs& a, int q0) { return min(q0 + kQ - 1, a.T - 1) / kK; }
+
+// item i: query-tile pair n_pairs - 1 - i / (B H) (heaviest first), head-batch i % (B H)
 __device__ __forceinline__ Item decode_item(const AttnArgs& a, int i) {
   Item it;
   const int bh = a.B * a.H;
-  const int qb = a.n_qblocks - 1 - i / bh;
+  const int p = a.n_pairs - 1 - i / bh;
   const int r = i % bh;
   it.b = r / a.H;
   it.h = r % a.H;
-  it.q0 = qb * kQ;
-  it.kt_lo = max(0, it.q0 - a.window + 1) / kK;
-  const int kt_hi = min(it.q0 + kQ - 1, a.T - 1) / kK;
-  it.n_tiles = kt_hi - it.kt_lo + 1;
+  it.q0 = 2 * p * kQ;
+  it.has_b = (2 * p + 1) < a.n_qblocks;
+  it.lo0 = first_key_tile(a, it.q0);
+  it.hi0 = last_key_tile(a, it.q0);
+  it.lo1 = first_key_tile(a, it.q0 + kQ);
+  it.hi1 = last_key_tile(a, it.q0 + kQ);
+  it.lo = it.lo0;
+  it.hi = it.has_b ? it.hi1 : it.hi0;
   return it;
+}
+
+__device__ __forceinline__ bool active(const Item& it, int g, int t) {
+  return g == 0 ? (t >= it.lo0 && t <= it.hi0) : (it.has_b && t >= it.lo1 && t <= it.hi1);
 }
 
 using ptx::ex2;
@@ -87,16 +116,17 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   enum {
-    B_QF = 0, B_QE = 1, B_KF = 2, B_VF = 4, B_KE = 6, B_VE = 8, B_SF = 10, B_PF = 12, B_PV = 13,
-    B_OE = 14, B_DONE = 16, NB = 17
+    B_QF = 0, B_QE = 1, B_SLF = 2, B_SLE = B_SLF + SLOTS, B_S = B_SLE + SLOTS, B_P = B_S + 2, B_O = B_P + 2,
+    B_OE = B_O + 2, B_DONE = B_OE + 2, NB = B_DONE + 1
   };
+  static_assert(NB * 8 + 8 <= 256, "barrier area");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NB);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const uint32_t bar0 = ptx::smem_u32(bars);
@@ -106,16 +136,16 @@ __global__ void __launch_bounds__(192, 1)
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar(B_QF), 1);
     ptx::mbar_init(bar(B_QE), 1);
-    for (int s = 0; s < STAGES; ++s) {
-      ptx::mbar_init(bar(B_KF + s), 1);
-      ptx::mbar_init(bar(B_VF + s), 1);
-      ptx::mbar_init(bar(B_KE + s), 1);
-      ptx::mbar_init(bar(B_VE + s), 1);
-      ptx::mbar_init(bar(B_SF + s), 1);
-      ptx::mbar_init(bar(B_OE + s), 4);
+    for (int s = 0; s < SLOTS; ++s) {
+      ptx::mbar_init(bar(B_SLF + s), 1);
+      ptx::mbar_init(bar(B_SLE + s), 1);
     }
-    ptx::mbar_init(bar(B_PF), 4);
-    ptx::mbar_init(bar(B_PV), 1);
+    for (int g = 0; g < 2; ++g) {
+      ptx::mbar_init(bar(B_S + g), 1);
+      ptx::mbar_init(bar(B_P + g), 4);
+      ptx::mbar_init(bar(B_O + g), 1);
+      ptx::mbar_init(bar(B_OE + g), 4);
+    }
     ptx::mbar_init(bar(B_DONE), 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
@@ -124,7 +154,7 @@ __global__ void __launch_bounds__(192, 1)
     ptx::prefetch_tmap(&tmK);
     ptx::prefetch_tmap(&tmV);
   }
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TMEM_COLS);
     ptx::tmem_relinquish();
     ptx::tc_fence_before();
@@ -132,136 +162,170 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t sQ = ptx::smem_u32(smem + OFF_Q);
-  const uint32_t sP = ptx::smem_u32(smem + OFF_P);
-  auto sK = [&](int s) { return ptx::smem_u32(smem + OFF_K + s * TILE_BYTES); };
-  auto sV = [&](int s) { return ptx::smem_u32(smem + OFF_V + s * TILE_BYTES); };
+  auto sQ = [&](int g) { return ptx::smem_u32(smem + OFF_Q + g * TILE_BYTES); };
+  auto sSlot = [&](int s) { return ptx::smem_u32(smem + OFF_SLOT + s * TILE_BYTES); };
 
-  if (warp == 0) {
+  if (warp >= 8) {
+    ptx::setmaxnreg_dec<kRegsLow>();
+    if (warp == kWarpTma) {
     if (ptx::elect_one()) {
       // ---------------- TMA producer ----------------
-      uint32_t kissued = 0, vissued = 0, kpar = 0, vpar = 0, qpar = 0;
-      bool qissued = false;
-      int g = 0, it = 0;
-      bool ok = true;
+      uint32_t issued = 0, par = 0, qpar = 0;
+      bool qissued = false, ok = true;
+      int sc = 0, it = 0;
       for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x, ++it) {
         const Item w = decode_item(a, item);
         const int row_base = w.b * a.T;
         const int qcol = w.h * kD, kcol = (w.h / (a.H / a.Hkv)) * kD;
-        // the previous item's QK MMAs have finished reading the Q buffer
+        // K_t then V_t into the next ring slots
+        auto load_kv = [&](int t) -> bool {
+          const int krow = row_base + t * kK;
+          for (int kv = 0; kv < 2; ++kv, ++sc) {
+            const int s = sc % SLOTS;
+            const uint32_t ph = (uint32_t)(sc / SLOTS) & 1u;
+            if (*abort_flag || !ptx::mbar_wait(bar(B_SLE + s), ph ^ 1, a.status)) return false;
+            const void* tm = kv == 0 ? (const void*)&tmK : (const void*)&tmV;
+            ptx::mbar_arrive_expect_tx(bar(B_SLF + s), TILE_BYTES);
+            ptx::tma_load_2d(sSlot(s), tm, bar(B_SLF + s), kcol, krow);
+            ptx::tma_load_2d(sSlot(s) + BOX_BYTES, tm, bar(B_SLF + s), kcol + 64, krow);
+            issued |= 1u << s;
+            par = (par & ~(1u << s)) | (ph << s);
+          }
+          return true;
+        };
+        // the item's first K/V tiles do not need the Q buffers: start them first
+        if (!load_kv(w.lo)) { ok = false; break; }
+        // the previous item's QK MMAs have finished reading the Q buffers
         if (*abort_flag || !ptx::mbar_wait(bar(B_QE), (it & 1) ^ 1, a.status)) { ok = false; break; }
-        ptx::mbar_arrive_expect_tx(bar(B_QF), TILE_BYTES);
-        ptx::tma_load_2d(sQ, &tmQ, bar(B_QF), qcol, row_base + w.q0);
-        ptx::tma_load_2d(sQ + BOX_BYTES, &tmQ, bar(B_QF), qcol + 64, row_base + w.q0);
+        ptx::mbar_arrive_expect_tx(bar(B_QF), (w.has_b ? 2 : 1) * TILE_BYTES);
+        for (int g = 0; g < (w.has_b ? 2 : 1); ++g) {
+          ptx::tma_load_2d(sQ(g), &tmQ, bar(B_QF), qcol, row_base + w.q0 + g * kQ);
+          ptx::tma_load_2d(sQ(g) + BOX_BYTES, &tmQ, bar(B_QF), qcol + 64, row_base + w.q0 + g * kQ);
+        }
         qissued = true;
         qpar = it & 1;
-        for (int j = 0; j < w.n_tiles; ++j, ++g) {
-          const int s = g & 1;
-          const uint32_t ph = (g >> 1) & 1;
-          const int krow = row_base + (w.kt_lo + j) * kK;
-          if (*abort_flag || !ptx::mbar_wait(bar(B_KE + s), ph ^ 1, a.status)) { ok = false; break; }
-          ptx::mbar_arrive_expect_tx(bar(B_KF + s), TILE_BYTES);
-          ptx::tma_load_2d(sK(s), &tmK, bar(B_KF + s), kcol, krow);
-          ptx::tma_load_2d(sK(s) + BOX_BYTES, &tmK, bar(B_KF + s), kcol + 64, krow);
-          kissued |= 1u << s;
-          kpar = (kpar & ~(1u << s)) | (ph << s);
-          if (*abort_flag || !ptx::mbar_wait(bar(B_VE + s), ph ^ 1, a.status)) { ok = false; break; }
-          ptx::mbar_arrive_expect_tx(bar(B_VF + s), TILE_BYTES);
-          ptx::tma_load_2d(sV(s), &tmV, bar(B_VF + s), kcol, krow);
-          ptx::tma_load_2d(sV(s) + BOX_BYTES, &tmV, bar(B_VF + s), kcol + 64, krow);
-          vissued |= 1u << s;
-          vpar = (vpar & ~(1u << s)) | (ph << s);
-        }
+        for (int t = w.lo + 1; ok && t <= w.hi; ++t)
+          if (!load_kv(t)) ok = false;
       }
       if (!ok) *abort_flag = 1;
       // every copy this thread issued has landed before the CTA may exit
       if (qissued) ptx::mbar_wait(bar(B_QF), qpar, a.status);
-      for (int s = 0; s < STAGES; ++s) {
-        if (kissued & (1u << s)) ptx::mbar_wait(bar(B_KF + s), (kpar >> s) & 1, a.status);
-        if (vissued & (1u << s)) ptx::mbar_wait(bar(B_VF + s), (vpar >> s) & 1, a.status);
-      }
+      for (int s = 0; s < SLOTS; ++s)
+        if (issued & (1u << s)) ptx::mbar_wait(bar(B_SLF + s), (par >> s) & 1, a.status);
     }
-  } else if (warp == 1) {
+  } else if (warp == kWarpMma) {
     if (ptx::elect_one()) {
       // ---------------- MMA issuer ----------------
       constexpr uint32_t idesc_qk = ptx::idesc_bf16(kQ, kK, 0, 0);
       constexpr uint32_t idesc_pv = ptx::idesc_bf16(kQ, kD, 0, 1);  // V is MN-major
-      auto issue_qk = [&](int gj) -> bool {
-        const int s = gj & 1;
-        if (*abort_flag || !ptx::mbar_wait(bar(B_KF + s), (gj >> 1) & 1, a.status)) return false;
-        ptx::tc_fence_after();
-        const uint32_t tS = tmem + (uint32_t)(s * 128);
+      auto slot_wait = [&](int sc) -> bool {
+        return !*abort_flag && ptx::mbar_wait(bar(B_SLF + sc % SLOTS), (uint32_t)(sc / SLOTS) & 1u, a.status);
+      };
+      auto qk = [&](int g, int sc) {
+        const uint32_t tS = tmem + (uint32_t)(g * 128);
+        const uint32_t k = sSlot(sc % SLOTS);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (uint32_t)((kk >> 2) * BOX_BYTES + (kk & 3) * 32);
-          ptx::mma_bf16_ss(tS, ptx::desc_kmajor_sw128(sQ + off), ptx::desc_kmajor_sw128(sK(s) + off),
-                           idesc_qk, kk > 0 ? 1u : 0u);
+          ptx::mma_bf16_ss(tS, ptx::desc_kmajor_sw128(sQ(g) + off), ptx::desc_kmajor_sw128(k + off), idesc_qk,
+                           kk > 0 ? 1u : 0u);
         }
-        ptx::mma_commit(bar(B_KE + s));
-        ptx::mma_commit(bar(B_SF + s));
-        return true;
+      };
+      auto pv = [&](int g, int sc, bool first) {
+        const uint32_t tP = tmem + (uint32_t)(g * 128);  // P_g: packed bf16 over the first 64 columns of S_g
+        const uint32_t tO = tmem + 256 + (uint32_t)(g * 128);
+        const uint32_t v = sSlot(sc % SLOTS);
+#pragma unroll
+        for (int kk = 0; kk < kK / 16; ++kk)
+          ptx::mma_bf16_ts(tO, tP + (uint32_t)(kk * 8), ptx::desc_mnmajor_sw128(v + (uint32_t)(kk * 2048), BOX_BYTES),
+                           idesc_pv, (!first || kk > 0) ? 1u : 0u);
       };
       bool ok = true;
-      int g = 0, it = 0;
+      int sc = 0, it = 0;
+      int pc0 = 0, pc1 = 0, ic0 = 0, ic1 = 0;  // P phases consumed, items finished, per group
       for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x, ++it) {
         const Item w = decode_item(a, item);
-        const int ob = it & 1;
-        const uint32_t tO = tmem + 256 + (uint32_t)(ob * 128);
         if (*abort_flag || !ptx::mbar_wait(bar(B_QF), it & 1, a.status)) { ok = false; break; }
         ptx::tc_fence_after();
-        if (!issue_qk(g)) { ok = false; break; }
-        if (w.n_tiles == 1) ptx::mma_commit(bar(B_QE));
-        for (int j = 0; j < w.n_tiles; ++j) {
-          const int gj = g + j;
-          const int s = gj & 1;
-          // S_{j+1} goes to the other buffer; the softmax released it with P_{j-1}
-          if (j + 1 < w.n_tiles) {
-            if (!issue_qk(gj + 1)) { ok = false; break; }
-            if (j + 2 == w.n_tiles) ptx::mma_commit(bar(B_QE));  // last QK of the item issued
+        // K_lo feeds the first S of every group that sees key tile lo
+        if (!slot_wait(sc)) { ok = false; break; }
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int g = 0; g < 2; ++g)
+          if (active(w, g, w.lo)) {
+            qk(g, sc);
+            ptx::mma_commit(bar(B_S + g));
           }
-          if (*abort_flag || !ptx::mbar_wait(bar(B_PF), gj & 1, a.status) ||
-              !ptx::mbar_wait(bar(B_VF + s), (gj >> 1) & 1, a.status)) { ok = false; break; }
-          // the output of the item two back has been read out of this O buffer
-          if (j == 0 && !ptx::mbar_wait(bar(B_OE + ob), ((it >> 1) & 1) ^ 1, a.status)) { ok = false; break; }
+        if (w.lo == w.hi) ptx::mma_commit(bar(B_QE));
+        ptx::mma_commit(bar(B_SLE + sc % SLOTS));
+        for (int t = w.lo; ok && t <= w.hi; ++t) {
+          const int scV = sc + 2 * (t - w.lo) + 1, scK1 = scV + 1;
+          const bool more = t < w.hi;
+          if (!slot_wait(scV) || (more && !slot_wait(scK1))) { ok = false; break; }
           ptx::tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < kK / 16; ++kk) {
-            const uint32_t aoff = (uint32_t)((kk >> 2) * BOX_BYTES + (kk & 3) * 32);
-            ptx::mma_bf16_ss(tO, ptx::desc_kmajor_sw128(sP + aoff),
-                             ptx::desc_mnmajor_sw128(sV(s) + (uint32_t)(kk * 2048), BOX_BYTES), idesc_pv,
-                             (j > 0 || kk > 0) ? 1u : 0u);
+          for (int g = 0; g < 2; ++g) {
+            const bool act = active(w, g, t);
+            const bool next = more && active(w, g, t + 1);
+            if (act) {
+              // group g has written P_g(t)
+              int& pc = g == 0 ? pc0 : pc1;
+              if (*abort_flag || !ptx::mbar_wait(bar(B_P + g), pc & 1, a.status)) { ok = false; break; }
+              ++pc;
+              const bool first = t == (g == 0 ? w.lo0 : w.lo1);
+              // the output of this group's previous item has been read out of O_g
+              const int ic = g == 0 ? ic0 : ic1;
+              if (first && !ptx::mbar_wait(bar(B_OE + g), (ic & 1) ^ 1, a.status)) { ok = false; break; }
+              ptx::tc_fence_after();
+              pv(g, scV, first);
+            }
+            if (next) {
+              qk(g, scK1);
+              ptx::mma_commit(bar(B_S + g));
+            } else if (act) {
+              ptx::mma_commit(bar(B_O + g));  // g's last tile of this item: O_g is final
+            }
           }
-          ptx::mma_commit(bar(B_VE + s));
-          ptx::mma_commit(bar(B_PV));
+          if (!ok) break;
+          if (t + 1 == w.hi) ptx::mma_commit(bar(B_QE));  // the item's last QKs are issued
+          ptx::mma_commit(bar(B_SLE + scV % SLOTS));
+          if (more) ptx::mma_commit(bar(B_SLE + scK1 % SLOTS));
         }
-        g += w.n_tiles;
+        ++ic0;
+        if (w.has_b) ++ic1;
+        sc += 2 * (w.hi - w.lo + 1);
       }
       if (!ok) *abort_flag = 1;
       ptx::mma_commit(bar(B_DONE));
       ptx::mbar_wait(bar(B_DONE), 0, a.status);
     }
+    }
   } else {
-    // ---------------- softmax + epilogue (warps 2..5) ----------------
+    ptx::setmaxnreg_inc<kRegsHigh>();
+    // ---------------- softmax + epilogue: group 0 = warps 0..3, group 1 = warps 4..7 ----------------
+    const int g = warp >> 2;
     const int gq = warp & 3;
     const int r = gq * 32 + lane;  // row of the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(gq * 32) << 16;
+    const uint32_t tS = tmem + (uint32_t)(g * 128) + lane_off;
+    const uint32_t tO = tmem + 256 + (uint32_t)(g * 128) + lane_off;
     const float c = a.scale_log2;
     bool ok = true;
-    int g = 0, it = 0;
-    for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x, ++it) {
+    int cnt = 0, icnt = 0;
+    for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
       const Item w = decode_item(a, item);
-      const int qi = w.q0 + r;  // query position
-      const int ob = it & 1;
-      const uint32_t tO = tmem + 256 + (uint32_t)(ob * 128) + lane_off;
+      if (g == 1 && !w.has_b) continue;
+      const int qg = w.q0 + g * kQ;  // first query of this group's tile
+      const int qi = qg + r;         // query position
+      const int t_lo = first_key_tile(a, qg);
+      const int t_hi = last_key_tile(a, qg);
       float m_run = -INFINITY, l_run = 0.f;
-      for (int j = 0; j < w.n_tiles; ++j) {
-        const int gj = g + j;
-        const int s = gj & 1;
-        const int k0 = (w.kt_lo + j) * kK;
-        if (*abort_flag || !ptx::mbar_wait(bar(B_SF + s), (gj >> 1) & 1, a.status)) { ok = false; break; }
+      for (int t = t_lo; t <= t_hi; ++t) {
+        const int k0 = t * kK;
+        // S_g(t) is ready, and O_g holds every PV of this group issued before it
+        if (*abort_flag || !ptx::mbar_wait(bar(B_S + g), cnt & 1, a.status)) { ok = false; break; }
         ptx::tc_fence_after();
         float x[128];
-        const uint32_t tS = tmem + (uint32_t)(s * 128) + lane_off;
         {
           // four TMEM loads in flight behind one wait
           uint32_t u0[32], u1[32], u2[32], u3[32];
@@ -285,7 +349,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int i = 0; i < 128; ++i) x[i] = (i >= clo && i <= chi) ? x[i] : -INFINITY;
         }
-        // row max as a tree (short dependency chains: one softmax warp per scheduler)
+        // row max as a tree of eight short chains
         float mx[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) mx[k] = x[k];
@@ -299,26 +363,28 @@ __global__ void __launch_bounds__(192, 1)
         const bool rescale = (tmax - m_run) * c > kRescaleThreshold;
         const float m_new = rescale ? tmax : m_run;
         const float mc = (m_new == -INFINITY) ? 0.f : m_new * c;
+        // p = 2^(s c - m c), packed to bf16 pairs over S's first 64 columns
         float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        uint32_t pk[64];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float p0 = ex2(fmaf(x[2 * i], c, -mc)), p1 = ex2(fmaf(x[2 * i + 1], c, -mc));
-          sm[i & 7] += p0 + p1;
-          pk[i] = pack_bf16(p0, p1);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float p0 = ex2(fmaf(x[64 * h + 2 * i], c, -mc)), p1 = ex2(fmaf(x[64 * h + 2 * i + 1], c, -mc));
+            sm[i & 7] += p0 + p1;
+            pk[i] = pack_bf16(p0, p1);
+          }
+          ptx::tmem_st32(tS + (uint32_t)(32 * h), pk);
         }
-        const float rsum = ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
-        // P_{gj-1} and O through PV_{gj-1} are done before P is rewritten or O rescaled
-        if (gj > 0 && !ptx::mbar_wait(bar(B_PV), (gj - 1) & 1, a.status)) { ok = false; break; }
-        ptx::tc_fence_after();
         const float alpha = rescale ? ex2(m_run * c - mc) : 1.f;  // 0 when m_run == -inf
         if (rescale) {
           l_run *= alpha;
           m_run = m_new;
         }
-        // O is rescaled by the whole warp (tcgen05.ld/st are warp-collective);
-        // rows that keep their max use alpha = 1
-        if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+        // O (which holds every earlier PV of this group) is rescaled by the
+        // whole warp, as tcgen05.ld/st are warp-collective; rows that keep
+        // their max use alpha = 1
+        if (t != t_lo && __any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
           for (int cc = 0; cc < 4; ++cc) {
             uint32_t u[32];
@@ -328,26 +394,18 @@ __global__ void __launch_bounds__(192, 1)
             for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
             ptx::tmem_st32(tO + (uint32_t)(cc * 32), u);
           }
-          ptx::tmem_st_wait();
         }
-        l_run += rsum;
-        // P tile: row r, keys 8q..8q+7 -> box q/8, 16-byte chunk (q%8) ^ (r%8)
-        uint8_t* prow = smem + OFF_P + r * 128;
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const int box = q >> 3, qq = q & 7;
-          uint4* dst = reinterpret_cast<uint4*>(prow + box * BOX_BYTES + ((qq ^ (r & 7)) << 4));
-          *dst = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        }
-        ptx::fence_proxy_async_smem();
+        l_run += ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
+        ptx::tmem_st_wait();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar(B_PF));
+        if (lane == 0) ptx::mbar_arrive(bar(B_P + g));
+        ++cnt;
       }
       if (!ok) break;
-      // output: O / l once the item's last PV has landed
-      const int glast = g + w.n_tiles - 1;
-      if (!ptx::mbar_wait(bar(B_PV), glast & 1, a.status)) { ok = false; break; }
+      // output: O / l once the group's last PV of the item has landed
+      if (!ptx::mbar_wait(bar(B_O + g), icnt & 1, a.status)) { ok = false; break; }
+      ++icnt;
       ptx::tc_fence_after();
       const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;
       const bool store = qi < a.T;
@@ -369,13 +427,12 @@ __global__ void __launch_bounds__(192, 1)
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(B_OE + ob));
-      g += w.n_tiles;
+      if (lane == 0) ptx::mbar_arrive(bar(B_OE + g));
     }
     if (!ok) *abort_flag = 1;
   }
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kWarpMma) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -399,7 +456,8 @@ bool launch_attn_tc(const bf16* q, const bf16* k, const bf16* v, int ldq, int ld
   a.window = (window <= 0 || window > T) ? T : window;
   a.ldo = ldo;
   a.n_qblocks = (T + kQ - 1) / kQ;
-  a.n_items = a.n_qblocks * B * H;
+  a.n_pairs = (a.n_qblocks + 1) / 2;
+  a.n_items = a.n_pairs * B * H;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.o = o;
   a.status = status;
@@ -409,7 +467,7 @@ bool launch_attn_tc(const bf16* q, const bf16* k, const bf16* v, int ldq, int ld
   });
   LaunchScope scope_(KK_ATTN_TC, st);
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
-  k_attn_tc<<<grid, 192, SMEM_BYTES, st>>>(tq, tk, tv, a);
+  k_attn_tc<<<grid, kThreads, SMEM_BYTES, st>>>(tq, tk, tv, a);
   return true;
 }
 

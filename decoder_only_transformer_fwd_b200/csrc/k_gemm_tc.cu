@@ -55,92 +55,104 @@ struct TcCfg {
 struct TcArgs {
   int M, N, K;
   int tiles_m, tiles_n, num_tiles;
+  int n_fastest;  // pair kernel: tile order with the column tile varying fastest
   int* status;
 };
 
+// Pair tile pt -> (row-pair block, column tile).  Column-fastest order keeps
+// the A rows that the CTAs of one wave share few enough to stay in L2 (for
+// GEMMs whose B is the smaller operand); row-fastest order does the same for
+// B (the head, whose weight is the larger operand).
+__device__ __forceinline__ void pair_tile(const TcArgs& a, int pt, int tiles_mp, int& mbp, int& nb) {
+  if (a.n_fastest) {
+    mbp = pt / a.tiles_n;
+    nb = pt % a.tiles_n;
+  } else {
+    mbp = pt % tiles_mp;
+    nb = pt / tiles_mp;
+  }
+}
+
 __device__ __forceinline__ float bits2f(uint32_t u) { return __uint_as_float(u); }
 
-// Residual epilogues (EPI_RESID, EPI_BLOCK_END) for a 32-row x 32-column
-// chunk: the warp's rows arrive one per lane (TMEM lane = row); they are
-// transposed through shared memory so that for each row the warp reads and
-// writes one contiguous 128-byte segment of x (and x0 / x_bo), with all the
-// chunk's loads issued before its stores.  With ep.xb_out set, the new x is
-// also stored as bf16 (the next GEMM's A operand) and the return value is the
-// sum of squares of the lane's row over the chunk's 32 columns.
-__device__ __forceinline__ float epi_resid_chunk(const EpiParams& ep, const TcArgs& a, float* stage,
-                                                 int row0, int n, const uint32_t (&r)[32], int lane) {
+// The 32 x 32 chunk epilogues below receive the accumulator one row per lane
+// (TMEM lane = row) and stage it in the warp's shared-memory buffer (row
+// pitch 33: conflict-free both ways).  They then work on it transposed: lane
+// (q = lane / 8, c4 = lane % 8) takes columns 4 c4 .. 4 c4 + 3 of rows 4 i + q,
+// i = 0..7, so every global access is a 16-byte (or 8-byte) vector and the 8
+// lanes of a quarter-warp cover one contiguous row segment.
+
+// Residual epilogues (EPI_RESID, EPI_BLOCK_END): x += acc, then for
+// EPI_BLOCK_END the next block's lambda x + mu x0 or the backout capture /
+// subtraction.  All of the chunk's loads are issued before its first store.
+// With ep.xb_out set the new x is also stored as bf16 (the next GEMM's A
+// operand) and ssr[i] accumulates the sum of squares of row 4 i + q over the
+// chunk's columns (the same value in the 8 lanes of the quarter-warp).
+__device__ __forceinline__ void epi_resid_chunk(const EpiParams& ep, const TcArgs& a, float* stage, int row0,
+                                                int n, const uint32_t (&r)[32], int lane, float (&ssr)[8]) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = __uint_as_float(r[i]);
   __syncwarp();
-  const int col = n + lane;
-  const bool col_ok = col < a.N;
+  const int q = lane >> 3, c4 = lane & 7;
+  const int col = n + 4 * c4;
+  const bool col_ok = col + 3 < a.N;  // N is a multiple of 32 on this path
   const bool bend = ep.mode == EPI_BLOCK_END;
   const bool need_x0 = bend && ep.end_kind == 1;
   const bool need_bo = bend && ep.end_kind == 2 && !ep.capture_bo;
+  const float* zsrc = need_x0 ? ep.x0 : ep.xbo;
   float lam = 1.f, mu = 0.f;
   if (need_x0) {
     lam = *ep.lam;
     mu = *ep.mu;
   }
+  float4 xv[8], zv[8];
 #pragma unroll
-  for (int h16 = 0; h16 < 2; ++h16) {
-    float acc[16], xv[16], zv[16];
+  for (int i = 0; i < 8; ++i) {
+    const int m = row0 + 4 * i + q;
+    const bool ok = col_ok && m < a.M;
+    const size_t off = (size_t)m * ep.ldx + col;
+    xv[i] = ok ? *reinterpret_cast<const float4*>(ep.x + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+    zv[i] = (ok && (need_x0 || need_bo)) ? *reinterpret_cast<const float4*>(zsrc + off)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 #pragma unroll
-    for (int rr = 0; rr < 16; ++rr) {
-      const int m = row0 + h16 * 16 + rr;
-      const size_t i = (size_t)m * ep.ldx + col;
-      const bool ok = col_ok && m < a.M;
-      acc[rr] = stage[(h16 * 16 + rr) * 33 + lane];
-      xv[rr] = ok ? ep.x[i] : 0.f;
-      zv[rr] = (ok && need_x0) ? ep.x0[i] : ((ok && need_bo) ? ep.xbo[i] : 0.f);
-    }
+  for (int i = 0; i < 8; ++i) {
+    const int rr = 4 * i + q;
+    const int m = row0 + rr;
+    const bool ok = col_ok && m < a.M;
+    const float* sr = stage + rr * 33 + 4 * c4;
+    float v[4] = {xv[i].x + sr[0], xv[i].y + sr[1], xv[i].z + sr[2], xv[i].w + sr[3]};
+    const float z[4] = {zv[i].x, zv[i].y, zv[i].z, zv[i].w};
+    const size_t off = (size_t)m * ep.ldx + col;
+    if (bend) {
+      if (ep.capture_bo && ok) *reinterpret_cast<float4*>(ep.xbo + off) = make_float4(v[0], v[1], v[2], v[3]);
 #pragma unroll
-    for (int rr = 0; rr < 16; ++rr) {
-      const int m = row0 + h16 * 16 + rr;
-      if (!col_ok || m >= a.M) continue;
-      const size_t i = (size_t)m * ep.ldx + col;
-      float v = xv[rr] + acc[rr];
-      if (bend) {
-        if (ep.capture_bo) ep.xbo[i] = v;
+      for (int e = 0; e < 4; ++e) {
         if (ep.end_kind == 1)
-          v = lam * v + mu * zv[rr];
+          v[e] = lam * v[e] + mu * z[e];
         else if (ep.end_kind == 2)
-          v = v - ep.beta * (ep.capture_bo ? v : zv[rr]);
+          v[e] = v[e] - ep.beta * (ep.capture_bo ? v[e] : z[e]);
       }
-      ep.x[i] = v;
-      stage[(h16 * 16 + rr) * 33 + lane] = v;
     }
+    if (ok) {
+      *reinterpret_cast<float4*>(ep.x + off) = make_float4(v[0], v[1], v[2], v[3]);
+      if (ep.xb_out != nullptr) {
+        const __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]), b1 = __floats2bfloat162_rn(v[2], v[3]);
+        *reinterpret_cast<uint2*>(ep.xb_out + (size_t)m * ep.ldxb + col) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
+      }
+    }
+    float sq = ok ? fmaf(v[0], v[0], fmaf(v[1], v[1], fmaf(v[2], v[2], v[3] * v[3]))) : 0.f;
+    sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+    sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+    sq += __shfl_xor_sync(0xffffffffu, sq, 4);
+    ssr[i] += sq;
   }
   __syncwarp();
-  float ss = 0.f;
-  if (ep.xb_out != nullptr) {
-    // row phase: lane t owns row row0 + t (columns past N or rows past M hold
-    // stale values but are never used: ss is only stored for valid rows and
-    // N is a multiple of 32 here)
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const float v = stage[lane * 33 + i];
-      ss = fmaf(v, v, ss);
-    }
-    const int cp = lane & 15;
-    const int c2 = n + 2 * cp;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const int rr = 2 * k + (lane >> 4);
-      const int m = row0 + rr;
-      const float v0 = stage[rr * 33 + 2 * cp], v1 = stage[rr * 33 + 2 * cp + 1];
-      if (c2 < a.N && m < a.M)
-        *reinterpret_cast<__nv_bfloat162*>(ep.xb_out + (size_t)m * ep.ldxb + c2) = __floats2bfloat162_rn(v0, v1);
-    }
-  }
-  __syncwarp();
-  return ss;
 }
 
-// EPI_STORE / EPI_RELU2 for a 32-row x 32-column chunk, coalesced: the rows
-// arrive one per lane, go through the shared-memory transpose buffer, and each
-// store instruction then writes two whole 64-byte bf16 row segments (lanes
-// 0..15 one row, 16..31 the next), two columns per lane.
+// EPI_STORE / EPI_RELU2: rscale (this lane's row scale) and ReLU^2 are applied
+// while staging; the transposed pass stores 8-byte bf16 quads.
 __device__ __forceinline__ void epi_store_chunk(const EpiParams& ep, const TcArgs& a, float* stage, int row0,
                                                 int n, const uint32_t (&r)[32], int lane, bool relu2,
                                                 float rscale) {
@@ -154,39 +166,46 @@ __device__ __forceinline__ void epi_store_chunk(const EpiParams& ep, const TcArg
     stage[lane * 33 + i] = v;
   }
   __syncwarp();
-  const int cp = lane & 15;       // column pair
-  const int col = n + 2 * cp;
-  const bool col_ok = col < a.N;  // N is even: the pair is in or out together
+  const int q = lane >> 3, c4 = lane & 7;
+  const int col = n + 4 * c4;
   bf16* base = reinterpret_cast<bf16*>(ep.out);
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const int rr = 2 * k + (lane >> 4);
+  for (int i = 0; i < 8; ++i) {
+    const int rr = 4 * i + q;
     const int m = row0 + rr;
-    const float v0 = stage[rr * 33 + 2 * cp], v1 = stage[rr * 33 + 2 * cp + 1];
-    if (col_ok && m < a.M) {
-      __nv_bfloat162 b2 = __floats2bfloat162_rn(v0, v1);
-      *reinterpret_cast<__nv_bfloat162*>(base + (size_t)m * ep.ldo + col) = b2;
+    const float* sr = stage + rr * 33 + 4 * c4;
+    if (m < a.M) {
+      bf16* dst = base + (size_t)m * ep.ldo + col;
+      if (col + 3 < a.N) {
+        const __nv_bfloat162 b0 = __floats2bfloat162_rn(sr[0], sr[1]), b1 = __floats2bfloat162_rn(sr[2], sr[3]);
+        *reinterpret_cast<uint2*>(dst) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (col + e < a.N) dst[e] = __float2bfloat16_rn(sr[e]);
+      }
     }
   }
   __syncwarp();
 }
 
-// Fused QKV epilogue for the 128 columns of one head held in TMEM at taddr:
-// q and k heads get RoPE (position m % T) and alpha * RMSNorm over the head;
-// v heads get gate * VE[tok] added; one bf16 rounding at the store.
-// ("The Mathematics of Karpathy's nanochat", §Rotary Position Embeddings,
-// §QK-Norm with Sharpening, §Value Embeddings.)
-__device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& a, uint32_t taddr, int m,
-                                             int col0, float rscale) {
-  const bool row_ok = m < a.M;
-  bf16* out = reinterpret_cast<bf16*>(ep.out) + (size_t)m * ep.ldo + col0;
+// Fused QKV epilogue for the 128 columns of one head held in TMEM at taddr,
+// rows m0 .. m0 + 31 (one per lane): q and k heads get RoPE (position m % T)
+// and alpha * RMSNorm over the head; v heads get gate * VE[tok] added; one
+// bf16 rounding at the store.  ("The Mathematics of Karpathy's nanochat",
+// §Rotary Position Embeddings, §QK-Norm with Sharpening, §Value Embeddings.)
+// The accumulator arrives one row per lane; it goes through the warp's
+// shared-memory transpose buffer so that the RoPE table reads, the
+// value-embedding reads and the output stores are row segments shared by
+// groups of lanes instead of one row per lane.  Per-row values (the norm
+// scale, position, token and gate) move between lanes by shuffles.
+__device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& a, float* stage, uint32_t taddr,
+                                             int m0, int lane, int col0, float rscale, float gate, int tok) {
+  bf16* out = reinterpret_cast<bf16*>(ep.out) + col0;
   if (col0 < ep.qk_cols) {
-    // RoPE pairs (j, j + 64) live in chunks (c, c + 2); the rotation preserves
-    // each pair's sum of squares, so the RMS comes from the raw accumulator
-    // in a first pass and the rotation + scale is applied in a second.
-    const int t = m % ep.T;
-    const float4* cs4 = reinterpret_cast<const float4*>(ep.rope_cos + (size_t)t * 64);
-    const float4* sn4 = reinterpret_cast<const float4*>(ep.rope_sin + (size_t)t * 64);
+    // RoPE pairs (j, j + 64); the rotation preserves each pair's sum of
+    // squares, so the RMS comes from the raw accumulator in a first pass
     float ss = 0.f;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
@@ -197,99 +216,170 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
       for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(u[i]), __uint_as_float(u[i]), ss);
     }
     // the head is rscale * acc: fold the row scale into the QK-norm factor
-    const float rs = rscale * ep.qk_alpha / sqrtf(ss * rscale * rscale * (1.0f / 128.0f) + ep.eps);
+    const float rs_lane = rscale * ep.qk_alpha / sqrtf(ss * rscale * rscale * (1.0f / 128.0f) + ep.eps);
+    const int t_lane = (m0 + lane) % ep.T;
+    const int fp = lane & 7, rsub = lane >> 3;  // lane -> (frequency pair, row within a group of 4)
 #pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
-      uint32_t u1[32], u2[32];
-      ptx::tmem_ld32(taddr + (uint32_t)(c * 32), u1);
-      ptx::tmem_ld32(taddr + (uint32_t)(c * 32 + 64), u2);
+    for (int k = 0; k < 4; ++k) {
+      // frequencies 16k .. 16k + 15: columns 16k.. of the first half and 64 + 16k.. of the second
+      uint32_t r1[16], r2[16];
+      ptx::tmem_ld16(taddr + (uint32_t)(16 * k), r1);
+      ptx::tmem_ld16(taddr + (uint32_t)(64 + 16 * k), r2);
       ptx::tmem_ld_wait();
-      if (!row_ok) continue;
-      uint32_t w1[16], w2[16];
 #pragma unroll
-      for (int j4 = 0; j4 < 8; ++j4) {
-        const float4 cc = cs4[c * 8 + j4], sv = sn4[c * 8 + j4];
-        const float cf[4] = {cc.x, cc.y, cc.z, cc.w}, sf[4] = {sv.x, sv.y, sv.z, sv.w};
-        float y1[4], y2[4];
+      for (int i = 0; i < 16; ++i) {
+        stage[lane * 33 + i] = __uint_as_float(r1[i]);
+        stage[lane * 33 + 16 + i] = __uint_as_float(r2[i]);
+      }
+      __syncwarp();
+      const int f0 = 16 * k + 2 * fp;
+      // all table reads of the chunk are issued before its first store (the
+      // stores could alias the table as far as the compiler knows)
+      float2 cs[8], sn[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a1 = __uint_as_float(u1[4 * j4 + e]), a2 = __uint_as_float(u2[4 * j4 + e]);
-          y1[e] = (a1 * cf[e] + a2 * sf[e]) * rs;
-          y2[e] = (-a1 * sf[e] + a2 * cf[e]) * rs;
+      for (int i = 0; i < 8; ++i) {
+        const int t = __shfl_sync(0xffffffffu, t_lane, 4 * i + rsub);
+        cs[i] = __ldg(reinterpret_cast<const float2*>(ep.rope_cos + (size_t)t * 64 + f0));
+        sn[i] = __ldg(reinterpret_cast<const float2*>(ep.rope_sin + (size_t)t * 64 + f0));
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int rr = 4 * i + rsub;
+        const float rs = __shfl_sync(0xffffffffu, rs_lane, rr);
+        const float a1x = stage[rr * 33 + 2 * fp], a1y = stage[rr * 33 + 2 * fp + 1];
+        const float a2x = stage[rr * 33 + 16 + 2 * fp], a2y = stage[rr * 33 + 16 + 2 * fp + 1];
+        if (m0 + rr < a.M) {
+          const float2 c2 = cs[i], s2 = sn[i];
+          bf16* o = out + (size_t)(m0 + rr) * ep.ldo + f0;
+          *reinterpret_cast<__nv_bfloat162*>(o) = __floats2bfloat162_rn((a1x * c2.x + a2x * s2.x) * rs,
+                                                                        (a1y * c2.y + a2y * s2.y) * rs);
+          *reinterpret_cast<__nv_bfloat162*>(o + 64) = __floats2bfloat162_rn((-a1x * s2.x + a2x * c2.x) * rs,
+                                                                             (-a1y * s2.y + a2y * c2.y) * rs);
         }
-        __nv_bfloat162 p;
-        p = __floats2bfloat162_rn(y1[0], y1[1]); w1[2 * j4] = *reinterpret_cast<uint32_t*>(&p);
-        p = __floats2bfloat162_rn(y1[2], y1[3]); w1[2 * j4 + 1] = *reinterpret_cast<uint32_t*>(&p);
-        p = __floats2bfloat162_rn(y2[0], y2[1]); w2[2 * j4] = *reinterpret_cast<uint32_t*>(&p);
-        p = __floats2bfloat162_rn(y2[2], y2[3]); w2[2 * j4 + 1] = *reinterpret_cast<uint32_t*>(&p);
       }
-      uint4* d1 = reinterpret_cast<uint4*>(out + c * 32);
-      uint4* d2 = reinterpret_cast<uint4*>(out + c * 32 + 64);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        d1[q] = make_uint4(w1[4 * q], w1[4 * q + 1], w1[4 * q + 2], w1[4 * q + 3]);
-        d2[q] = make_uint4(w2[4 * q], w2[4 * q + 1], w2[4 * q + 2], w2[4 * q + 3]);
-      }
+      __syncwarp();
     }
   } else {
     const int hv = (col0 - ep.qk_cols) >> 7;
-    int tok = row_ok ? ep.tokens[m] : 0;
-    tok = min(max(tok, 0), ep.vocab - 1);
-    const bool mix = row_ok && ep.ve != nullptr;
-    float g = 0.f;
-    if (mix) {
+    const bool mix = ep.ve != nullptr;
+    const bf16* ve_head = mix ? reinterpret_cast<const bf16*>(ep.ve) + (size_t)hv * 128 : nullptr;
+    const int cp = lane & 15, rsub = lane >> 4;  // lane -> (column pair, row within a pair of rows)
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t u[32];
+      ptx::tmem_ld32(taddr + (uint32_t)(c * 32), u);
+      ptx::tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = __uint_as_float(u[i]) * rscale;
+      __syncwarp();
+      const int n = c * 32 + 2 * cp;
+      // the chunk's value-embedding reads are all issued before its first store
+      uint32_t e2[16];
+#pragma unroll
+      for (int kk = 0; kk < 16; ++kk) {
+        const int tk = __shfl_sync(0xffffffffu, tok, 2 * kk + rsub);
+        e2[kk] = mix ? __ldg(reinterpret_cast<const unsigned int*>(ve_head + (size_t)tk * ep.n_kv_head * 128 + n)) : 0u;
+      }
+#pragma unroll
+      for (int kk = 0; kk < 16; ++kk) {
+        const int rr = 2 * kk + rsub;
+        float v0 = stage[rr * 33 + 2 * cp], v1 = stage[rr * 33 + 2 * cp + 1];
+        const float g = __shfl_sync(0xffffffffu, gate, rr);
+        if (m0 + rr < a.M) {
+          const float2 e = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e2[kk]));
+          v0 = fmaf(g, e.x, v0);
+          v1 = fmaf(g, e.y, v1);
+          *reinterpret_cast<__nv_bfloat162*>(out + (size_t)(m0 + rr) * ep.ldo + n) = __floats2bfloat162_rn(v0, v1);
+        }
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// Per-row values of a tile that do not depend on its accumulator.  They are
+// loaded before the epilogue waits for the accumulator, so their memory
+// latency overlaps the tile's MMAs; the rows the epilogue will read later are
+// pulled into L2 at the same time.
+struct RowPre {
+  float rscale;  // 1 / rms of the A row (fused RMSNorm); 1 when unused
+  float gate;    // QKV value heads: the value-embedding gate
+  int y;         // CE: the row's target id, or -1
+  int tok;       // QKV value heads: the row's token id, clamped
+};
+
+template <int BN, int MODE>
+__device__ __forceinline__ RowPre epilogue_pre(const EpiParams& ep, const TcArgs& a, int mb, int nb, int g,
+                                               int half, int lane) {
+  constexpr int HALF = BN / 2;
+  const int m = mb * kBM + g * 32 + lane;
+  const int n_lo = nb * BN + half * HALF;
+  RowPre p{1.f, 0.f, -1, 0};
+  if (m >= a.M) return p;
+  if constexpr (MODE == EPI_QKV || MODE == EPI_RELU2 || MODE == EPI_CE) {
+    if (ep.ss_in != nullptr) {
+      const float* sp = ep.ss_in + (size_t)m * ep.ss_in_parts;
+      float t = 0.f;
+#pragma unroll 4
+      for (int j = 0; j < ep.ss_in_parts; ++j) t += sp[j];
+      p.rscale = 1.0f / sqrtf(t * ep.inv_c + ep.eps);
+    }
+  }
+  if constexpr (MODE == EPI_QKV) {
+    if (n_lo % 128 == 0 && n_lo >= ep.qk_cols && n_lo < a.N && ep.ve != nullptr) {
+      const int hv = (n_lo - ep.qk_cols) >> 7;
+      int tok = ep.tokens[m];
+      tok = min(max(tok, 0), ep.vocab - 1);
+      p.tok = tok;
+      const char* row = reinterpret_cast<const char*>(reinterpret_cast<const bf16*>(ep.ve) +
+                                                      ((size_t)tok * ep.n_kv_head + hv) * 128);
+      ptx::prefetch_l2(row);
+      ptx::prefetch_l2(row + 128);
       if (ep.gate != nullptr) {
-        g = ep.gate[(size_t)m * ep.n_kv_head + hv];
+        p.gate = ep.gate[(size_t)m * ep.n_kv_head + hv];
       } else {
         // gate from the normalised block input: rscale * x[m, :gate_c]
         const float* xr = ep.x + (size_t)m * ep.ldx;
         const float* wg = ep.gate_w + (size_t)hv * ep.gate_c;
         float d = 0.f;
+#pragma unroll 4
         for (int c = 0; c < ep.gate_c; ++c) d = fmaf(xr[c], wg[c], d);
-        g = ep.gate_scale / (1.0f + __expf(-rscale * d));
+        p.gate = ep.gate_scale / (1.0f + __expf(-p.rscale * d));
       }
     }
-    // the row's 128 value-embedding entries are gathered up front (one memory
-    // round trip per row instead of one per chunk)
-    uint4 e[16];
-    if (mix) {
-      const uint4* e4 = reinterpret_cast<const uint4*>(reinterpret_cast<const bf16*>(ep.ve) +
-                                                       ((size_t)tok * ep.n_kv_head + hv) * 128);
+  } else if constexpr (MODE == EPI_CE) {
+    int y = ep.targets[m];
+    if (y != -1) y = min(max(y, 0), ep.vocab - 1);  // out-of-range ids are flagged by the combine
+    p.y = y;
+  }
+  return p;
+}
+
+// Pull into L2 the rows of x (and x0 / x_bo) that the residual epilogue of
+// tile (mb, nb) will read: called one tile ahead, so the reads hit L2.
+template <int BN, int MODE>
+__device__ __forceinline__ void epilogue_prefetch(const EpiParams& ep, const TcArgs& a, int mb, int nb, int g,
+                                                  int half, int lane) {
+  constexpr int HALF = BN / 2;
+  const int m = mb * kBM + g * 32 + lane;
+  const int n_lo = nb * BN + half * HALF;
+  if (m >= a.M) return;
+  if constexpr (MODE == EPI_RESID || MODE == EPI_BLOCK_END) {
+    // this thread's row of the warp's column half of x (and x0 / x_bo)
+    const int nc = min(HALF, a.N - n_lo);
+    if (nc > 0) {
+      const char* xr = reinterpret_cast<const char*>(ep.x + (size_t)m * ep.ldx + n_lo);
 #pragma unroll
-      for (int q = 0; q < 16; ++q) e[q] = e4[q];
-    }
+      for (int o = 0; o < HALF * 4; o += 128)
+        if (o < nc * 4) ptx::prefetch_l2(xr + o);
+      if (MODE == EPI_BLOCK_END) {
+        const float* z = ep.end_kind == 1 ? ep.x0 : ((ep.end_kind == 2 && !ep.capture_bo) ? ep.xbo : nullptr);
+        if (z != nullptr) {
+          const char* zr = reinterpret_cast<const char*>(z + (size_t)m * ep.ldx + n_lo);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t u[32];
-      ptx::tmem_ld32(taddr + (uint32_t)(c * 32), u);
-      ptx::tmem_ld_wait();
-      if (!row_ok) continue;
-      float x[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(u[i]) * rscale;
-      if (mix) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 w = e[c * 4 + q];
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ww[k]));
-            x[8 * q + 2 * k] += g * f.x;
-            x[8 * q + 2 * k + 1] += g * f.y;
-          }
+          for (int o = 0; o < HALF * 4; o += 128)
+            if (o < nc * 4) ptx::prefetch_l2(zr + o);
         }
-      }
-      uint4* d4 = reinterpret_cast<uint4*>(out + c * 32);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t w[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(x[8 * q + 2 * k], x[8 * q + 2 * k + 1]);
-          w[k] = *reinterpret_cast<uint32_t*>(&b2);
-        }
-        d4[q] = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
   }
@@ -299,31 +389,20 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
 // (its TMEM lane quarter) and the columns [c_lo, c_lo + BN/2) of its half.
 template <int BN, int MODE>
 __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs& a, uint32_t taddr, int mb,
-                                              int nb, int g, int half, int lane, float* stage) {
+                                              int nb, int g, int half, int lane, float* stage,
+                                              const RowPre& pre) {
   constexpr int HALF = BN / 2;
   const int row = g * 32 + lane;
   const int m = mb * kBM + row;
   const int c_lo = half * HALF;
   const int n_lo = nb * BN + c_lo;
-  // fused RMSNorm of the A operand: 1 / rms of this thread's row
-  float rscale = 1.f;
-  if constexpr (MODE == EPI_QKV || MODE == EPI_RELU2 || MODE == EPI_CE) {
-    if (ep.ss_in != nullptr && m < a.M) {
-      const float* sp = ep.ss_in + (size_t)m * ep.ss_in_parts;
-      float t = 0.f;
-      for (int j = 0; j < ep.ss_in_parts; ++j) t += sp[j];
-      rscale = 1.0f / sqrtf(t * ep.inv_c + ep.eps);
-    }
-  }
+  const float rscale = pre.rscale;  // fused RMSNorm of the A operand: 1 / rms of this thread's row
   if constexpr (MODE == EPI_QKV) {
     // one head (128 columns) per warp when BN = 256; with BN = 128 the first half does it
-    if (c_lo % 128 == 0 && n_lo < a.N) epi_qkv_head(ep, a, taddr + (uint32_t)c_lo, m, n_lo, rscale);
+    if (c_lo % 128 == 0 && n_lo < a.N)
+      epi_qkv_head(ep, a, stage, taddr + (uint32_t)c_lo, mb * kBM + g * 32, lane, n_lo, rscale, pre.gate, pre.tok);
   } else if constexpr (MODE == EPI_CE) {
-    int y = -1;
-    if (m < a.M) {
-      y = ep.targets[m];
-      if (y != -1) y = min(max(y, 0), ep.vocab - 1);  // out-of-range ids are flagged by the combine
-    }
+    const int y = pre.y;
     // zhat = c tanh(z/c) = c - 2c / (e^{2z/c} + 1); exp(zhat - c) = 2^(-2c log2(e) / (e^{2z/c} + 1))
     const float k1 = 2.0f * 1.4426950408889634f / ep.cap;
     const float k2 = -2.0f * ep.cap * 1.4426950408889634f;
@@ -362,20 +441,27 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs&
       if (y >= n_lo && y < n_lo + HALF) ep.ce_tgt[m] = tgt;
     }
   } else {
-    float ss = 0.f;
+    float ssr[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
     for (int c = 0; c < HALF; c += 32) {
       uint32_t r[32];
       ptx::tmem_ld32(taddr + (uint32_t)(c_lo + c), r);
       ptx::tmem_ld_wait();
       if constexpr (MODE == EPI_RESID || MODE == EPI_BLOCK_END) {
-        ss += epi_resid_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, r, lane);
+        epi_resid_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, r, lane, ssr);
       } else {
         epi_store_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, r, lane, MODE == EPI_RELU2, rscale);
       }
     }
     if constexpr (MODE == EPI_RESID || MODE == EPI_BLOCK_END) {
-      if (ep.ss_out != nullptr && m < a.M) ep.ss_out[(size_t)m * ep.ss_parts + n_lo / HALF] = ss;
+      // lane (q, 0) holds the sums of rows 4 i + q
+      if (ep.ss_out != nullptr && (lane & 7) == 0) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int mr = mb * kBM + g * 32 + 4 * i + (lane >> 3);
+          if (mr < a.M) ep.ss_out[(size_t)mr * ep.ss_parts + n_lo / HALF] = ssr[i];
+        }
+      }
     }
   }
 }
@@ -509,15 +595,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* stage = epi_stage + ew * Cf::STAGE_FLOATS;
     int acc = 0;
     uint32_t aph = 0;
+    if (blockIdx.x < a.num_tiles)
+      epilogue_prefetch<BN, MODE>(ep, a, blockIdx.x % a.tiles_m, blockIdx.x / a.tiles_m, g, half, lane);
     for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
       const int mb = tile % a.tiles_m, nb = tile / a.tiles_m;
+      const RowPre pre = epilogue_pre<BN, MODE>(ep, a, mb, nb, g, half, lane);
+      const int nxt = tile + gridDim.x;
+      if (nxt < a.num_tiles) epilogue_prefetch<BN, MODE>(ep, a, nxt % a.tiles_m, nxt / a.tiles_m, g, half, lane);
       if (*abort_flag || !ptx::mbar_wait(tfull(acc), aph, a.status)) {
         *abort_flag = 1;
         break;
       }
       ptx::tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(g * 32) << 16) + (uint32_t)(acc * BN);
-      epilogue_tile<BN, MODE>(ep, a, taddr, mb, nb, g, half, lane, stage);
+      epilogue_tile<BN, MODE>(ep, a, taddr, mb, nb, g, half, lane, stage, pre);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(tempty(acc));
@@ -618,7 +709,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t ph = 0, issued = 0, par = 0;
       for (int pt = cid; pt < num_pt; pt += ncl) {
-        const int mbp = pt % tiles_mp, nb = pt / tiles_mp;
+        int mbp, nb;
+        pair_tile(a, pt, tiles_mp, mbp, nb);
         bool ok = true;
         for (int kb = 0; kb < nk; ++kb) {
           if (*abort_flag || !ptx::mbar_wait_cluster(empty(stage), ph ^ 1, a.status)) {
@@ -692,15 +784,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* stage = epi_stage + ew * Cf::STAGE_FLOATS;
     int acc = 0;
     uint32_t aph = 0;
+    if (cid < num_pt) {
+      int mbp, nb;
+      pair_tile(a, cid, tiles_mp, mbp, nb);
+      epilogue_prefetch<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, half, lane);
+    }
     for (int pt = cid; pt < num_pt; pt += ncl) {
-      const int mbp = pt % tiles_mp, nb = pt / tiles_mp;
+      int mbp, nb;
+      pair_tile(a, pt, tiles_mp, mbp, nb);
+      const RowPre pre = epilogue_pre<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, half, lane);
+      const int nxt = pt + ncl;
+      if (nxt < num_pt) {
+        int mbn, nbn;
+        pair_tile(a, nxt, tiles_mp, mbn, nbn);
+        epilogue_prefetch<BN, MODE>(ep, a, mbn * 2 + (int)rank, nbn, g, half, lane);
+      }
       if (*abort_flag || !ptx::mbar_wait_cluster(tfull(acc), aph, a.status)) {
         *abort_flag = 1;
         break;
       }
       ptx::tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(g * 32) << 16) + (uint32_t)(acc * BN);
-      epilogue_tile<BN, MODE>(ep, a, taddr, mbp * 2 + (int)rank, nb, g, half, lane, stage);
+      epilogue_tile<BN, MODE>(ep, a, taddr, mbp * 2 + (int)rank, nb, g, half, lane, stage, pre);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa(tempty(acc), 0));
@@ -841,6 +946,7 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
     a.tiles_m = (M + kBM - 1) / kBM;
     a.tiles_n = N / BN;
     a.num_tiles = a.tiles_m * a.tiles_n;
+    a.n_fastest = ep.mode != EPI_CE;
     a.status = status;
     const int num_pt = ((M + 2 * kBM - 1) / (2 * kBM)) * a.tiles_n;
     const int ncl = num_pt < num_sms / 2 ? num_pt : num_sms / 2;
@@ -857,6 +963,7 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
   a.tiles_m = (M + kBM - 1) / kBM;
   a.tiles_n = (N + BN - 1) / BN;
   a.num_tiles = a.tiles_m * a.tiles_n;
+  a.n_fastest = 0;  // unused by the single-CTA kernel
   a.status = status;
   const int grid = a.num_tiles < num_sms ? a.num_tiles : num_sms;
   LaunchScope scope_(KK_GEMM_TC, st);
