@@ -284,16 +284,19 @@ def run_ours(args):
     barrier()
     ms_total = max_over_ranks(e0.elapsed_time(e1))
 
-    # ---- timed region B: the same steps with per-launch events on the GEMM kernel ----
-    gemm_per_step = 4 * cfg.n_layer + 1
-    timer = nc.LaunchTimer(gemm_per_step * args.steps, kinds=["gemm_tcgen05"])
+    # ---- timed region B: the same steps with per-launch events on every kernel ----
+    timer = nc.LaunchTimer(launches_per_step * args.steps)
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
+    b0.record(stream)
     with timer:
         for _ in range(args.steps):
             step()
+    b1.record(stream)
     torch.cuda.synchronize()
     per_kind = timer.per_kind()
+    ms_step_b = b0.elapsed_time(b1) / args.steps
 
     # ---- e2e: the host-buffer entry point, copies inside the timed region ----
     h_tok = torch.from_numpy(tok_h).pin_memory()
@@ -367,6 +370,9 @@ def run_ours(args):
                     "h2d_bytes_per_step": 2 * M * 4, "d2h_bytes_per_step": M * 4},
             "gpu_launches": launches_per_step * args.steps,
             "kernel_ms_per_step": {k: v[1] / args.steps for k, v in per_kind.items()},
+            # region B's step time minus the summed kernel times: launch gaps,
+            # pipeline fill/drain between kernels and the timing events themselves
+            "gap_ms_per_step": ms_step_b - sum(v[1] for v in per_kind.values()) / args.steps,
             "attention_sweep": attn,
         }
         print(json.dumps(line), flush=True)

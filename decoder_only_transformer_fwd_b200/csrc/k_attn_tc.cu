@@ -119,6 +119,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 __global__ void __launch_bounds__(kThreads, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+  pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
@@ -162,6 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // q, k, v come from the previous kernel; o may still be read by it
   auto sQ = [&](int g) { return ptx::smem_u32(smem + OFF_Q + g * TILE_BYTES); };
   auto sSlot = [&](int s) { return ptx::smem_u32(smem + OFF_SLOT + s * TILE_BYTES); };
 
@@ -467,8 +469,7 @@ bool launch_attn_tc(const bf16* q, const bf16* k, const bf16* v, int ldq, int ld
   });
   LaunchScope scope_(KK_ATTN_TC, st);
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
-  k_attn_tc<<<grid, kThreads, SMEM_BYTES, st>>>(tq, tk, tv, a);
-  return true;
+  return launch_pdl(k_attn_tc, dim3(grid), dim3(kThreads), SMEM_BYTES, st, 1, tq, tk, tv, a) == cudaSuccess;
 }
 
 }  // namespace nc

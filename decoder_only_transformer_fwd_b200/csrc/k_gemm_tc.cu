@@ -472,6 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const TcArgs a, const EpiParams ep) {
   using Cf = TcCfg<BN>;
   constexpr int S = Cf::STAGES;
+  pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * Cf::STAGE_BYTES);
@@ -514,6 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int nk = a.K / kBK;
+  pdl_wait();  // the operands and the epilogue's inputs come from earlier kernels
 
   if (warp == 0) {
     if (ptx::elect_one()) {
@@ -654,6 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using Cf = PairCfg;
   constexpr int BN = Cf::BN;
   constexpr int S = Cf::STAGES;
+  pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * Cf::STAGE_BYTES);
@@ -699,6 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int nk = a.K / kBK;
+  pdl_wait();  // the operands and the epilogue's inputs come from earlier kernels
   const int tiles_mp = (a.M + 2 * kBM - 1) / (2 * kBM);
   const int num_pt = tiles_mp * a.tiles_n;
   const int cid = (int)ptx::cluster_id_x(), ncl = (int)ptx::nclusters_x();
@@ -846,7 +850,7 @@ void launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, 
   std::call_once(once, [] {
     cudaFuncSetAttribute(k_gemm_tc<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<BN>::SMEM);
   });
-  k_gemm_tc<BN, MODE><<<grid, kThreads, TcCfg<BN>::SMEM, st>>>(ta, tb, a, ep);
+  launch_pdl(k_gemm_tc<BN, MODE>, dim3(grid), dim3(kThreads), TcCfg<BN>::SMEM, st, 1, ta, tb, a, ep);
 }
 
 template <int MODE>
@@ -856,19 +860,7 @@ void launch_pair_mode(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs
   std::call_once(once, [] {
     cudaFuncSetAttribute(k_gemm_tc2<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM);
   });
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * nclusters, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = PairCfg::SMEM;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, k_gemm_tc2<MODE>, ta, tb, a, ep);
+  launch_pdl(k_gemm_tc2<MODE>, dim3(2 * nclusters), dim3(kThreads), PairCfg::SMEM, st, 2, ta, tb, a, ep);
 }
 
 bool launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep, int nclusters,

@@ -35,6 +35,8 @@ __global__ void k_embed(const T* __restrict__ wte, const int32_t* __restrict__ t
                         const float* __restrict__ smear_gate, int smear, int gc,
                         const float* __restrict__ lam0p, const float* __restrict__ mu0p, float eps, int T_, int C, int V, float* __restrict__ x, float* __restrict__ x0,
                         bf16* __restrict__ xb, float* __restrict__ ss, int ss_parts, int* status) {
+  pdl_launch_dependents();
+  pdl_wait();
   extern __shared__ float sh[];  // [2C] rows + [32] reduction
   float* cur = sh;
   float* prev = sh + C;
@@ -167,6 +169,8 @@ __global__ void k_rmsnorm<bf16>(const float* __restrict__ x, bf16* __restrict__ 
 // cos/sin of phi_{t,j} = t * base^(-2j/D), evaluated in double and rounded
 // once to fp32 (an fp32 product t * omega would lose ~5e-4 rad at t ~ 8k).
 __global__ void k_rope_table(float* cos_t, float* sin_t, int T_, int D, double base) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int half = D / 2;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= T_ * half) return;
@@ -232,6 +236,8 @@ template <typename T>
 __global__ void k_rope_qknorm_copy(const T* q, const T* k, T* qo, T* ko, int T_, int H, int Hkv,
                                    int D, const float* cos_t, const float* sin_t, float alpha,
                                    float eps, int M) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int slots = H + Hkv;
   const long long wid = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -279,6 +285,8 @@ __global__ void k_ce_rows(const float* logits, int ldl, const int32_t* targets, 
 // row's log-sum-exp and subtract the target's zhat.  One warp per row.
 __global__ void k_ce_combine(const float* ce_sum, const float* ce_tgt, int n_tiles, float offset,
                              const int32_t* targets, int M, int V, float* loss, int* status) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (m >= M) return;
@@ -299,6 +307,8 @@ __global__ void k_ce_combine(const float* ce_sum, const float* ce_tgt, int n_til
 
 // Mean of loss over valid targets, fixed reduction order (deterministic).
 __global__ void k_loss_mean(const float* loss, const int32_t* targets, int n, float* out) {
+  pdl_launch_dependents();
+  pdl_wait();
   __shared__ float rs[32];
   __shared__ float rc[32];
   float s = 0.f, c = 0.f;
@@ -334,11 +344,11 @@ void launch_embed(const void* wte, const int32_t* tokens, const float* smear_gat
   const int M = B * T;
   const size_t sh = (size_t)(2 * C + 32) * sizeof(float);
   if (act_bf16)
-    k_embed<bf16><<<M, 256, sh, st>>>((const bf16*)wte, tokens, smear_gate, smear, gate_channels, lam0,
-                                      mu0, eps, T, C, V, x, x0, xb, ss, ss_parts, status);
+    launch_pdl(k_embed<bf16>, dim3(M), dim3(256), sh, st, 1, (const bf16*)wte, tokens, smear_gate, smear,
+               gate_channels, lam0, mu0, eps, T, C, V, x, x0, xb, ss, ss_parts, status);
   else
-    k_embed<float><<<M, 256, sh, st>>>((const float*)wte, tokens, smear_gate, smear, gate_channels,
-                                       lam0, mu0, eps, T, C, V, x, x0, xb, ss, ss_parts, status);
+    launch_pdl(k_embed<float>, dim3(M), dim3(256), sh, st, 1, (const float*)wte, tokens, smear_gate, smear,
+               gate_channels, lam0, mu0, eps, T, C, V, x, x0, xb, ss, ss_parts, status);
 }
 
 void launch_rmsnorm(const float* x, void* xn, int M, int C, float eps, int act_bf16,
@@ -358,7 +368,7 @@ void launch_rmsnorm(const float* x, void* xn, int M, int C, float eps, int act_b
 void launch_rope_table(float* cos_t, float* sin_t, int T, int D, float base, cudaStream_t st) {
   LaunchScope scope_(KK_ROPE_TABLE, st);
   const int n = T * (D / 2);
-  k_rope_table<<<(n + 255) / 256, 256, 0, st>>>(cos_t, sin_t, T, D, (double)base);
+  launch_pdl(k_rope_table, dim3((n + 255) / 256), dim3(256), 0, st, 1, cos_t, sin_t, T, D, (double)base);
 }
 
 void launch_rope_qknorm_ve(void* qkv, int ld, int B, int T, int H, int Hkv, int D,
@@ -389,13 +399,11 @@ void launch_rope_qknorm_copy(const void* q, const void* k, void* qo, void* ko, i
   const int wpb = 8;
   const unsigned grid = (unsigned)((warps + wpb - 1) / wpb);
   if (act_bf16)
-    k_rope_qknorm_copy<bf16><<<grid, wpb * 32, 0, st>>>((const bf16*)q, (const bf16*)k, (bf16*)qo,
-                                                        (bf16*)ko, T, H, Hkv, D, cos_t, sin_t, alpha,
-                                                        eps, M);
+    launch_pdl(k_rope_qknorm_copy<bf16>, dim3(grid), dim3(wpb * 32), 0, st, 1, (const bf16*)q, (const bf16*)k,
+               (bf16*)qo, (bf16*)ko, T, H, Hkv, D, cos_t, sin_t, alpha, eps, M);
   else
-    k_rope_qknorm_copy<float><<<grid, wpb * 32, 0, st>>>((const float*)q, (const float*)k, (float*)qo,
-                                                         (float*)ko, T, H, Hkv, D, cos_t, sin_t, alpha,
-                                                         eps, M);
+    launch_pdl(k_rope_qknorm_copy<float>, dim3(grid), dim3(wpb * 32), 0, st, 1, (const float*)q,
+               (const float*)k, (float*)qo, (float*)ko, T, H, Hkv, D, cos_t, sin_t, alpha, eps, M);
 }
 
 void launch_ce_rows(const float* logits, int ldl, const int32_t* targets, int M, int V, float* loss,
@@ -408,13 +416,13 @@ void launch_ce_combine(const float* ce_sum, const float* ce_tgt, int n_tiles, fl
                        const int32_t* targets, int M, int V, float* loss, int* status, cudaStream_t st) {
   LaunchScope scope_(KK_CE_COMBINE, st);
   const int wpb = 8;
-  k_ce_combine<<<(M + wpb - 1) / wpb, wpb * 32, 0, st>>>(ce_sum, ce_tgt, n_tiles, offset, targets, M, V,
-                                                         loss, status);
+  launch_pdl(k_ce_combine, dim3((M + wpb - 1) / wpb), dim3(wpb * 32), 0, st, 1, ce_sum, ce_tgt, n_tiles, offset,
+             targets, M, V, loss, status);
 }
 
 void launch_loss_mean(const float* loss, const int32_t* targets, int n, float* out, cudaStream_t st) {
   LaunchScope scope_(KK_LOSS_MEAN, st);
-  k_loss_mean<<<1, 1024, 0, st>>>(loss, targets, n, out);
+  launch_pdl(k_loss_mean, dim3(1), dim3(1024), 0, st, 1, loss, targets, n, out);
 }
 
 }  // namespace nc

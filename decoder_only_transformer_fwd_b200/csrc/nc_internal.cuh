@@ -167,4 +167,40 @@ struct LaunchScope {
   ~LaunchScope() { launch_end(kind, st); }
 };
 
+// Programmatic dependent launch.  Kernels launched through launch_pdl may be
+// scheduled while the previous kernel on the stream is still finishing, so
+// each of them runs pdl_launch_dependents() first (letting the next kernel be
+// scheduled in turn) and pdl_wait() before its first access to global memory:
+// pdl_wait() returns once the previous kernel has completed and its writes
+// are visible (at once when there is no such kernel).  Only set-up work that
+// touches no global memory (barrier init, TMEM allocation, descriptor
+// prefetch) runs before it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              int cluster_x, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 }  // namespace nc
