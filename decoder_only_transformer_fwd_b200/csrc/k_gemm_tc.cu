@@ -151,6 +151,48 @@ __device__ __forceinline__ void epi_resid_chunk(const EpiParams& ep, const TcArg
   __syncwarp();
 }
 
+// EPI_RESID, software-pipelined by the caller: resid_load requests x for a
+// chunk (transposed lane layout) and resid_apply finishes a staged chunk
+// with those values, so the loads of chunk c + 1 overlap the stores of c.
+__device__ __forceinline__ void resid_load(const EpiParams& ep, const TcArgs& a, int row0, int n, int lane,
+                                           float4 (&xv)[8]) {
+  const int q = lane >> 3, c4 = lane & 7;
+  const int col = n + 4 * c4;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int m = row0 + 4 * i + q;
+    xv[i] = (col + 3 < a.N && m < a.M) ? *reinterpret_cast<const float4*>(ep.x + (size_t)m * ep.ldx + col)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+__device__ __forceinline__ void resid_apply(const EpiParams& ep, const TcArgs& a, const float* stage, int row0,
+                                            int n, int lane, const float4 (&xv)[8], float (&ssr)[8]) {
+  const int q = lane >> 3, c4 = lane & 7;
+  const int col = n + 4 * c4;
+  const bool col_ok = col + 3 < a.N;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int rr = 4 * i + q;
+    const int m = row0 + rr;
+    const bool ok = col_ok && m < a.M;
+    const float* sr = stage + rr * 33 + 4 * c4;
+    const float v0 = xv[i].x + sr[0], v1 = xv[i].y + sr[1], v2 = xv[i].z + sr[2], v3 = xv[i].w + sr[3];
+    if (ok) {
+      *reinterpret_cast<float4*>(ep.x + (size_t)m * ep.ldx + col) = make_float4(v0, v1, v2, v3);
+      if (ep.xb_out != nullptr) {
+        const __nv_bfloat162 b0 = __floats2bfloat162_rn(v0, v1), b1 = __floats2bfloat162_rn(v2, v3);
+        *reinterpret_cast<uint2*>(ep.xb_out + (size_t)m * ep.ldxb + col) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
+      }
+    }
+    float sq = ok ? fmaf(v0, v0, fmaf(v1, v1, fmaf(v2, v2, v3 * v3))) : 0.f;
+    sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+    sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+    sq += __shfl_xor_sync(0xffffffffu, sq, 4);
+    ssr[i] += sq;
+  }
+}
+
 // EPI_STORE / EPI_RELU2: rscale (this lane's row scale) and ReLU^2 are applied
 // while staging; the transposed pass stores 8-byte bf16 quads.
 __device__ __forceinline__ void epi_store_chunk(const EpiParams& ep, const TcArgs& a, float* stage, int row0,
@@ -204,27 +246,32 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
                                              int m0, int lane, int col0, float rscale, float gate, int tok) {
   bf16* out = reinterpret_cast<bf16*>(ep.out) + col0;
   if (col0 < ep.qk_cols) {
-    // RoPE pairs (j, j + 64); the rotation preserves each pair's sum of
-    // squares, so the RMS comes from the raw accumulator in a first pass
-    float ss = 0.f;
+    const int t_lane = (m0 + lane) % ep.T;
+    const int fp = lane & 7, rsub = lane >> 3;  // lane -> (frequency pair, row within a group of 4)
+    // RoPE pairs (j, j + 64) preserve each pair's sum of squares, so the RMS
+    // comes from the raw accumulator in a first pass
+    float ssa = 0.f, ssb = 0.f;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       uint32_t u[32];
       ptx::tmem_ld32(taddr + (uint32_t)(c * 32), u);
       ptx::tmem_ld_wait();
 #pragma unroll
-      for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(u[i]), __uint_as_float(u[i]), ss);
+      for (int i = 0; i < 32; i += 2) {
+        ssa = fmaf(__uint_as_float(u[i]), __uint_as_float(u[i]), ssa);
+        ssb = fmaf(__uint_as_float(u[i + 1]), __uint_as_float(u[i + 1]), ssb);
+      }
     }
     // the head is rscale * acc: fold the row scale into the QK-norm factor
-    const float rs_lane = rscale * ep.qk_alpha / sqrtf(ss * rscale * rscale * (1.0f / 128.0f) + ep.eps);
-    const int t_lane = (m0 + lane) % ep.T;
-    const int fp = lane & 7, rsub = lane >> 3;  // lane -> (frequency pair, row within a group of 4)
+    const float rs_lane = rscale * ep.qk_alpha / sqrtf((ssa + ssb) * rscale * rscale * (1.0f / 128.0f) + ep.eps);
+    // second pass over four groups of 16 frequencies; group k + 1's TMEM
+    // columns are requested before group k is rotated and stored
+    uint32_t r1[16], r2[16];
+    ptx::tmem_ld16(taddr, r1);
+    ptx::tmem_ld16(taddr + 64u, r2);
 #pragma unroll 1
     for (int k = 0; k < 4; ++k) {
       // frequencies 16k .. 16k + 15: columns 16k.. of the first half and 64 + 16k.. of the second
-      uint32_t r1[16], r2[16];
-      ptx::tmem_ld16(taddr + (uint32_t)(16 * k), r1);
-      ptx::tmem_ld16(taddr + (uint32_t)(64 + 16 * k), r2);
       ptx::tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
@@ -232,29 +279,35 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
         stage[lane * 33 + 16 + i] = __uint_as_float(r2[i]);
       }
       __syncwarp();
-      const int f0 = 16 * k + 2 * fp;
-      // all table reads of the chunk are issued before its first store (the
-      // stores could alias the table as far as the compiler knows)
-      float2 cs[8], sn[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int t = __shfl_sync(0xffffffffu, t_lane, 4 * i + rsub);
-        cs[i] = __ldg(reinterpret_cast<const float2*>(ep.rope_cos + (size_t)t * 64 + f0));
-        sn[i] = __ldg(reinterpret_cast<const float2*>(ep.rope_sin + (size_t)t * 64 + f0));
+      if (k < 3) {
+        ptx::tmem_ld16(taddr + (uint32_t)(16 * (k + 1)), r1);
+        ptx::tmem_ld16(taddr + (uint32_t)(64 + 16 * (k + 1)), r2);
       }
+      const int f0 = 16 * k + 2 * fp;
+      // this lane's two frequencies in cycles per position, split so that the
+      // phase t f mod 1 is exact to ~1e-7 (the angle then goes to the
+      // hardware sine / cosine within [-pi, pi])
+      const float fh0 = __ldg(ep.rope_fsplit + f0), fh1 = __ldg(ep.rope_fsplit + f0 + 1);
+      const float fl0 = __ldg(ep.rope_fsplit + 64 + f0), fl1 = __ldg(ep.rope_fsplit + 64 + f0 + 1);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int rr = 4 * i + rsub;
         const float rs = __shfl_sync(0xffffffffu, rs_lane, rr);
+        const float tf = (float)__shfl_sync(0xffffffffu, t_lane, rr);
+        float p0 = tf * fh0, p1 = tf * fh1;  // exact
+        p0 = fmaf(tf, fl0, p0 - floorf(p0));
+        p1 = fmaf(tf, fl1, p1 - floorf(p1));
+        p0 = (p0 - rintf(p0)) * 6.2831853071795865f;
+        p1 = (p1 - rintf(p1)) * 6.2831853071795865f;
+        const float c0 = __cosf(p0), s0 = __sinf(p0), c1 = __cosf(p1), s1 = __sinf(p1);
         const float a1x = stage[rr * 33 + 2 * fp], a1y = stage[rr * 33 + 2 * fp + 1];
         const float a2x = stage[rr * 33 + 16 + 2 * fp], a2y = stage[rr * 33 + 16 + 2 * fp + 1];
         if (m0 + rr < a.M) {
-          const float2 c2 = cs[i], s2 = sn[i];
           bf16* o = out + (size_t)(m0 + rr) * ep.ldo + f0;
-          *reinterpret_cast<__nv_bfloat162*>(o) = __floats2bfloat162_rn((a1x * c2.x + a2x * s2.x) * rs,
-                                                                        (a1y * c2.y + a2y * s2.y) * rs);
-          *reinterpret_cast<__nv_bfloat162*>(o + 64) = __floats2bfloat162_rn((-a1x * s2.x + a2x * c2.x) * rs,
-                                                                             (-a1y * s2.y + a2y * c2.y) * rs);
+          *reinterpret_cast<__nv_bfloat162*>(o) = __floats2bfloat162_rn((a1x * c0 + a2x * s0) * rs,
+                                                                        (a1y * c1 + a2y * s1) * rs);
+          *reinterpret_cast<__nv_bfloat162*>(o + 64) = __floats2bfloat162_rn((-a1x * s0 + a2x * c0) * rs,
+                                                                             (-a1y * s1 + a2y * c1) * rs);
         }
       }
       __syncwarp();
@@ -263,36 +316,57 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
     const int hv = (col0 - ep.qk_cols) >> 7;
     const bool mix = ep.ve != nullptr;
     const bf16* ve_head = mix ? reinterpret_cast<const bf16*>(ep.ve) + (size_t)hv * 128 : nullptr;
-    const int cp = lane & 15, rsub = lane >> 4;  // lane -> (column pair, row within a pair of rows)
+    const int q = lane >> 3, c4 = lane & 7;  // lane -> (row within a group of 4, column quad)
+    // value-embedding row offsets of this lane's rows 4 i + q
+    const uint32_t vrow_lane = (uint32_t)tok * (uint32_t)ep.n_kv_head * 128u;
+    uint32_t vr[8];
+    float gr[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      vr[i] = __shfl_sync(0xffffffffu, vrow_lane, 4 * i + q);
+      gr[i] = __shfl_sync(0xffffffffu, gate, 4 * i + q);
+    }
+    // chunk c + 1's TMEM columns and value-embedding entries are requested
+    // before chunk c is mixed and stored
+    uint32_t u[32];
+    uint2 e[8];
+    ptx::tmem_ld32(taddr, u);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      e[i] = mix ? __ldg(reinterpret_cast<const uint2*>(ve_head + vr[i] + 4 * c4)) : make_uint2(0u, 0u);
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
-      uint32_t u[32];
-      ptx::tmem_ld32(taddr + (uint32_t)(c * 32), u);
       ptx::tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = __uint_as_float(u[i]) * rscale;
       __syncwarp();
-      const int n = c * 32 + 2 * cp;
-      // the chunk's value-embedding reads are all issued before its first store
-      uint32_t e2[16];
+      uint2 en[8];
+      if (c < 3) {
+        ptx::tmem_ld32(taddr + (uint32_t)(32 * (c + 1)), u);
 #pragma unroll
-      for (int kk = 0; kk < 16; ++kk) {
-        const int tk = __shfl_sync(0xffffffffu, tok, 2 * kk + rsub);
-        e2[kk] = mix ? __ldg(reinterpret_cast<const unsigned int*>(ve_head + (size_t)tk * ep.n_kv_head * 128 + n)) : 0u;
+        for (int i = 0; i < 8; ++i)
+          en[i] = mix ? __ldg(reinterpret_cast<const uint2*>(ve_head + vr[i] + 32 * (c + 1) + 4 * c4))
+                      : make_uint2(0u, 0u);
       }
+      const int n = c * 32 + 4 * c4;
 #pragma unroll
-      for (int kk = 0; kk < 16; ++kk) {
-        const int rr = 2 * kk + rsub;
-        float v0 = stage[rr * 33 + 2 * cp], v1 = stage[rr * 33 + 2 * cp + 1];
-        const float g = __shfl_sync(0xffffffffu, gate, rr);
+      for (int i = 0; i < 8; ++i) {
+        const int rr = 4 * i + q;
+        const float* sr = stage + rr * 33 + 4 * c4;
         if (m0 + rr < a.M) {
-          const float2 e = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e2[kk]));
-          v0 = fmaf(g, e.x, v0);
-          v1 = fmaf(g, e.y, v1);
-          *reinterpret_cast<__nv_bfloat162*>(out + (size_t)(m0 + rr) * ep.ldo + n) = __floats2bfloat162_rn(v0, v1);
+          const float2 e01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e[i].x));
+          const float2 e23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&e[i].y));
+          const __nv_bfloat162 b0 = __floats2bfloat162_rn(fmaf(gr[i], e01.x, sr[0]), fmaf(gr[i], e01.y, sr[1]));
+          const __nv_bfloat162 b1 = __floats2bfloat162_rn(fmaf(gr[i], e23.x, sr[2]), fmaf(gr[i], e23.y, sr[3]));
+          *reinterpret_cast<uint2*>(out + (size_t)(m0 + rr) * ep.ldo + n) =
+              make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
         }
       }
       __syncwarp();
+      if (c < 3) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) e[i] = en[i];
+      }
     }
   }
 }
@@ -385,6 +459,23 @@ __device__ __forceinline__ void epilogue_prefetch(const EpiParams& ep, const TcA
   }
 }
 
+// Before the first tile: touch (prefetch into L2) one line of each output
+// row this thread will write first, so that the address translations and L2
+// lines of the output region are in place when the first accumulator is ready.
+template <int BN, int MODE>
+__device__ __forceinline__ void epilogue_touch_outputs(const EpiParams& ep, const TcArgs& a, int mb, int nb, int g,
+                                                       int half, int lane) {
+  constexpr int HALF = BN / 2;
+  const int m = mb * kBM + g * 32 + lane;
+  const int n_lo = nb * BN + half * HALF;
+  if (m >= a.M || n_lo >= a.N) return;
+  if constexpr (MODE == EPI_STORE || MODE == EPI_RELU2 || MODE == EPI_QKV) {
+    ptx::prefetch_l2(reinterpret_cast<const bf16*>(ep.out) + (size_t)m * ep.ldo + n_lo);
+  } else if constexpr (MODE == EPI_RESID || MODE == EPI_BLOCK_END) {
+    if (ep.xb_out != nullptr) ptx::prefetch_l2(ep.xb_out + (size_t)m * ep.ldxb + n_lo);
+  }
+}
+
 // Epilogue work of one warp on one tile: rows g*32 .. g*32+31 of the tile
 // (its TMEM lane quarter) and the columns [c_lo, c_lo + BN/2) of its half.
 template <int BN, int MODE>
@@ -440,20 +531,58 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs&
       ep.ce_sum[(size_t)m * ep.ce_tiles + nb * 2 + half] = sum;
       if (y >= n_lo && y < n_lo + HALF) ep.ce_tgt[m] = tgt;
     }
-  } else {
+  } else if constexpr (MODE == EPI_RESID) {
     float ssr[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const int row0 = mb * kBM + g * 32;
+    uint32_t r[32];
+    float4 xv[8];
+    ptx::tmem_ld32(taddr + (uint32_t)c_lo, r);
+    resid_load(ep, a, row0, n_lo, lane, xv);
 #pragma unroll 1
     for (int c = 0; c < HALF; c += 32) {
-      uint32_t r[32];
-      ptx::tmem_ld32(taddr + (uint32_t)(c_lo + c), r);
       ptx::tmem_ld_wait();
-      if constexpr (MODE == EPI_RESID || MODE == EPI_BLOCK_END) {
-        epi_resid_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, r, lane, ssr);
-      } else {
-        epi_store_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, r, lane, MODE == EPI_RELU2, rscale);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = __uint_as_float(r[i]);
+      __syncwarp();
+      float4 xn[8];
+      if (c + 32 < HALF) {
+        ptx::tmem_ld32(taddr + (uint32_t)(c_lo + c + 32), r);
+        resid_load(ep, a, row0, n_lo + c + 32, lane, xn);
+      }
+      resid_apply(ep, a, stage, row0, n_lo + c, lane, xv, ssr);
+      __syncwarp();
+      if (c + 32 < HALF) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xv[i] = xn[i];
       }
     }
-    if constexpr (MODE == EPI_RESID || MODE == EPI_BLOCK_END) {
+    // lane (q, 0) holds the sums of rows 4 i + q
+    if (ep.ss_out != nullptr && (lane & 7) == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int mr = row0 + 4 * i + (lane >> 3);
+        if (mr < a.M) ep.ss_out[(size_t)mr * ep.ss_parts + n_lo / HALF] = ssr[i];
+      }
+    }
+  } else {
+    float ssr[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    // chunk c + 1's TMEM columns are requested before chunk c is processed
+    uint32_t r[32];
+    ptx::tmem_ld32(taddr + (uint32_t)c_lo, r);
+#pragma unroll 1
+    for (int c = 0; c < HALF; c += 32) {
+      ptx::tmem_ld_wait();
+      uint32_t rc[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) rc[i] = r[i];
+      if (c + 32 < HALF) ptx::tmem_ld32(taddr + (uint32_t)(c_lo + c + 32), r);
+      if constexpr (MODE == EPI_BLOCK_END) {
+        epi_resid_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, rc, lane, ssr);
+      } else {
+        epi_store_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, rc, lane, MODE == EPI_RELU2, rscale);
+      }
+    }
+    if constexpr (MODE == EPI_BLOCK_END) {
       // lane (q, 0) holds the sums of rows 4 i + q
       if (ep.ss_out != nullptr && (lane & 7) == 0) {
 #pragma unroll
@@ -597,8 +726,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* stage = epi_stage + ew * Cf::STAGE_FLOATS;
     int acc = 0;
     uint32_t aph = 0;
-    if (blockIdx.x < a.num_tiles)
+    if (blockIdx.x < a.num_tiles) {
       epilogue_prefetch<BN, MODE>(ep, a, blockIdx.x % a.tiles_m, blockIdx.x / a.tiles_m, g, half, lane);
+      epilogue_touch_outputs<BN, MODE>(ep, a, blockIdx.x % a.tiles_m, blockIdx.x / a.tiles_m, g, half, lane);
+    }
     for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
       const int mb = tile % a.tiles_m, nb = tile / a.tiles_m;
       const RowPre pre = epilogue_pre<BN, MODE>(ep, a, mb, nb, g, half, lane);
@@ -636,6 +767,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 // CTA's "accumulator empty" barrier.  No TMA multicast: every CTA reads its
 // own operand slices.
 // ---------------------------------------------------------------------------
+// Pair kernel roles: warps 0..7 epilogue (two warpgroups), warp 8 TMA,
+// warp 9 MMA + TMEM allocation, warps 10..11 idle.  Registers: launched at
+// 168 per thread (65536 / 384); the TMA/MMA warpgroup drops to 88 and the
+// epilogue warpgroups rise to 208: 2 * 128 * 208 + 128 * 88 = 64512 = 384 * 168.
+constexpr int kPairThreads = 384;
+constexpr int kPairWarpTma = 8, kPairWarpMma = 9;
+constexpr int kPairRegsLow = 88, kPairRegsHigh = 208;
+static_assert(2 * 128 * kPairRegsHigh + 128 * kPairRegsLow <= kPairThreads * 168, "register split");
+
 struct PairCfg {
   static constexpr int BN = 256;
   static constexpr int STAGES = 6;
@@ -650,7 +790,7 @@ struct PairCfg {
 };
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
     k_gemm_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const TcArgs a, const EpiParams ep) {
   using Cf = PairCfg;
@@ -692,7 +832,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::prefetch_tmap(&tmA);
     ptx::prefetch_tmap(&tmB);
   }
-  if (warp == 1) {
+  if (warp == kPairWarpMma) {
     ptx::tmem_alloc2(ptx::smem_u32(tmem_slot), Cf::TMEM_COLS);
     ptx::tmem_relinquish2();
     ptx::tc_fence_before();
@@ -707,7 +847,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_pt = tiles_mp * a.tiles_n;
   const int cid = (int)ptx::cluster_id_x(), ncl = (int)ptx::nclusters_x();
 
-  if (warp == 0) {
+  if (warp >= 8) {
+    ptx::setmaxnreg_dec<kPairRegsLow>();
+    if (warp == kPairWarpTma) {
     if (ptx::elect_one()) {
       // ---------------- TMA producer (both CTAs) ----------------
       int stage = 0;
@@ -739,7 +881,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < S; ++s)
         if (issued & (1u << s)) ptx::mbar_wait_cluster(empty(s), (par >> s) & 1, a.status);
     }
-  } else if (warp == 1) {
+  } else if (warp == kPairWarpMma) {
     if (leader && ptx::elect_one()) {
       // ---------------- MMA issuer (even CTA) ----------------
       constexpr uint32_t idesc = ptx::idesc_bf16(2 * kBM, BN);
@@ -780,10 +922,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mma_commit2(mma_done);
       ptx::mbar_wait_cluster(mma_done, 0, a.status);
     }
+    }
   } else {
-    // ---------------- epilogue (both CTAs, warps 2 .. 2 + kEpiWarps - 1) ----------------
-    const int ew = warp - 2;
-    const int g = warp & 3;
+    ptx::setmaxnreg_inc<kPairRegsHigh>();
+    // ---------------- epilogue (both CTAs, warps 0 .. kEpiWarps - 1) ----------------
+    const int ew = warp;
+    const int g = warp & 3;  // TMEM lane quarter
     const int half = ew >> 2;
     float* stage = epi_stage + ew * Cf::STAGE_FLOATS;
     int acc = 0;
@@ -792,6 +936,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int mbp, nb;
       pair_tile(a, cid, tiles_mp, mbp, nb);
       epilogue_prefetch<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, half, lane);
+      epilogue_touch_outputs<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, half, lane);
     }
     for (int pt = cid; pt < num_pt; pt += ncl) {
       int mbp, nb;
@@ -819,7 +964,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   ptx::cluster_sync_all();
-  if (warp == 1) {
+  if (warp == kPairWarpMma) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc2(tmem, Cf::TMEM_COLS);
   }
@@ -860,7 +1005,7 @@ void launch_pair_mode(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs
   std::call_once(once, [] {
     cudaFuncSetAttribute(k_gemm_tc2<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM);
   });
-  launch_pdl(k_gemm_tc2<MODE>, dim3(2 * nclusters), dim3(kThreads), PairCfg::SMEM, st, 2, ta, tb, a, ep);
+  launch_pdl(k_gemm_tc2<MODE>, dim3(2 * nclusters), dim3(kPairThreads), PairCfg::SMEM, st, 2, ta, tb, a, ep);
 }
 
 bool launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep, int nclusters,

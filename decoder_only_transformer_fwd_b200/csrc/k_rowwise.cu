@@ -168,11 +168,25 @@ __global__ void k_rmsnorm<bf16>(const float* __restrict__ x, bf16* __restrict__ 
 
 // cos/sin of phi_{t,j} = t * base^(-2j/D), evaluated in double and rounded
 // once to fp32 (an fp32 product t * omega would lose ~5e-4 rad at t ~ 8k).
-__global__ void k_rope_table(float* cos_t, float* sin_t, int T_, int D, double base) {
+// Also, when fsplit is given, the rotation frequencies in cycles per
+// position, f_j = omega_j / (2 pi), split as fh_j + fl_j: fh_j keeps
+// 24 - tbits significant bits, so that t * fh_j is exact in fp32 for every
+// t < 2^tbits, and fl_j is the rest (fsplit = fh[0..D/2) | fl[0..D/2)).  The
+// phase t f_j mod 1 then follows in fp32 to about 1e-7 cycles.
+__global__ void k_rope_table(float* cos_t, float* sin_t, int T_, int D, double base, float* fsplit, int tbits) {
   pdl_launch_dependents();
   pdl_wait();
   const int half = D / 2;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (fsplit != nullptr && i < half) {
+    const double f = pow(base, -2.0 * (double)i / (double)D) / (2.0 * 3.14159265358979323846);
+    int e = 0;
+    frexp(f, &e);  // f = m 2^e, m in [0.5, 1)
+    const int keep = 24 - tbits;
+    const double fh = ldexp(rint(ldexp(f, keep - e)), e - keep);
+    fsplit[i] = (float)fh;
+    fsplit[half + i] = (float)(f - fh);
+  }
   if (i >= T_ * half) return;
   const int t = i / half, j = i % half;
   const double omega = pow(base, -2.0 * (double)j / (double)D);
@@ -365,10 +379,12 @@ void launch_rmsnorm(const float* x, void* xn, int M, int C, float eps, int act_b
                                                   gate_channels, gate_scale, gate_out);
 }
 
-void launch_rope_table(float* cos_t, float* sin_t, int T, int D, float base, cudaStream_t st) {
+void launch_rope_table(float* cos_t, float* sin_t, int T, int D, float base, cudaStream_t st, float* fsplit,
+                       int tbits) {
   LaunchScope scope_(KK_ROPE_TABLE, st);
   const int n = T * (D / 2);
-  launch_pdl(k_rope_table, dim3((n + 255) / 256), dim3(256), 0, st, 1, cos_t, sin_t, T, D, (double)base);
+  launch_pdl(k_rope_table, dim3((n + 255) / 256), dim3(256), 0, st, 1, cos_t, sin_t, T, D, (double)base, fsplit,
+             tbits);
 }
 
 void launch_rope_qknorm_ve(void* qkv, int ld, int B, int T, int H, int Hkv, int D,

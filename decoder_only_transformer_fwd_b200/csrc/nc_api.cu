@@ -105,7 +105,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
 struct Layout {
-  size_t x, x0, xbo, xn, qkv, o, h, gate, ss, rcos, rsin, ce_sum, ce_tgt, logits, tok, tgt, loss;
+  size_t x, x0, xbo, xn, qkv, o, h, gate, ss, rcos, rsin, rfreq, ce_sum, ce_tgt, logits, tok, tgt, loss;
   size_t total;
   int ce_tiles;
 };
@@ -148,6 +148,7 @@ Layout layout(const nc_config& c, int max_tokens) {
   L.ss = take(M * (C / 64) * 4);  // per-row sums of squares of the residual, per column group
   L.rcos = take((size_t)c.max_T * D / 2 * 4);
   L.rsin = take((size_t)c.max_T * D / 2 * 4);
+  L.rfreq = take(D * 4);
   L.ce_tiles = 2 * ((c.vocab_padded + 127) / 128);  // per (row, 128-or-256-column tile, half)
   L.ce_sum = take(M * L.ce_tiles * 4);
   L.ce_tgt = take(M * 4);
@@ -304,9 +305,12 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
   float* gate = at<float>(ws, Lw.gate);
   float* rcos = at<float>(ws, Lw.rcos);
   float* rsin = at<float>(ws, Lw.rsin);
+  float* rfreq = at<float>(ws, Lw.rfreq);
   const size_t esz = bf ? 2 : 4;
 
-  launch_rope_table(rcos, rsin, T, D, c.rope_base, st);
+  int tbits = 1;
+  while ((1 << tbits) < T) ++tbits;
+  launch_rope_table(rcos, rsin, T, D, c.rope_base, st, rfreq, tbits);
   // tensor-core path: RMSNorm is fused into the GEMMs (producers write bf16(x)
   // and per-row sums of squares, consumers scale their rows by 1 / rms)
   const bool tc = bf && c.gemm_impl == 0;
@@ -347,6 +351,7 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
       e.qk_cols = (H + Hkv) * D;
       e.rope_cos = rcos;
       e.rope_sin = rsin;
+      e.rope_fsplit = rfreq;
       e.qk_alpha = c.qk_alpha;
       e.tokens = tokens;
       e.ve = ve ? lp.ve : nullptr;

@@ -84,6 +84,7 @@ struct EpiParams {
   int qk_cols;        // (H + H_kv) * D: columns below this are q and k heads
   const float* rope_cos;  // [T, D/2]
   const float* rope_sin;
+  const float* rope_fsplit;  // [2, D/2]: per-frequency cycles per position, split hi | lo (see k_rope_table)
   float qk_alpha, eps;
   const int32_t* tokens;  // [M]
   const void* ve;     // [V, H_kv D] or NULL
@@ -118,7 +119,8 @@ void launch_embed(const void* wte, const int32_t* tokens, const float* smear_gat
 void launch_rmsnorm(const float* x, void* xn, int M, int C, float eps, int act_bf16,
                     const float* ve_gate, int Hkv, int gate_channels, float gate_scale, float* gate_out,
                     cudaStream_t st);
-void launch_rope_table(float* cos_t, float* sin_t, int T, int D, float base, cudaStream_t st);
+void launch_rope_table(float* cos_t, float* sin_t, int T, int D, float base, cudaStream_t st,
+                       float* fsplit = nullptr, int tbits = 0);
 void launch_rope_qknorm_ve(void* qkv, int ld, int B, int T, int H, int Hkv, int D,
                            const float* cos_t, const float* sin_t, float alpha, float eps,
                            const int32_t* tokens, const void* ve, const float* gate, int V,
