@@ -111,21 +111,29 @@ __device__ __forceinline__ bool active(const Item& it, int g, int t) {
 
 using ptx::ex2;
 
-// 2^x on the FMA/ALU pipes, for the share of the exponentials that would
-// otherwise queue on the special-function unit (whose rate per SM matches the
-// tensor core's on this path).  Range reduction x = n + f with n = round(x):
-// adding 1.5 * 2^23 leaves n in the low mantissa bits, so no conversion
-// instruction is needed; 2^f on [-1/2, 1/2] by a cubic whose coefficients were
-// fitted for minimum relative error (7.5e-5, far below the bf16 rounding of
-// P); n is then added to the exponent field.  x < -125 (masked or negligible
-// scores) gives 0, as the hardware exponential does for -inf.
-__device__ __forceinline__ float exp2_poly(float x) {
-  const float xc = fmaxf(x, -125.0f);
-  const float y = xc + 12582912.0f;
-  const float f = xc - (y - 12582912.0f);
-  const float p = fmaf(fmaf(fmaf(0.05517132f, f, 0.24261054f), f, 0.69326097f), f, 0.99992812f);
-  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(y) << 23));
-  return x < -125.0f ? 0.0f : r;
+// Packed fp32 pairs (the f32x2 forms of add / fma on this architecture).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -368,35 +376,33 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 128; ++i) x[i] = (i >= clo && i <= chi) ? x[i] : -INFINITY;
         }
-        // row max as a tree of eight short chains
+        // row max: eight chains of three-input max
         float mx[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = x[k];
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(x[2 * k], x[2 * k + 1]);
 #pragma unroll
-        for (int i = 8; i < 128; i += 8)
+        for (int i = 16; i < 128; i += 16)
 #pragma unroll
-          for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], x[i + k]);
-        const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+          for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], x[i + 2 * k], x[i + 2 * k + 1]);
+        const float tmax = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
         // lazy max (raw score units): move it only when it grows by more than 2^8 after scaling
         const bool rescale = (tmax - m_run) * c > kRescaleThreshold;
         const float m_new = rescale ? tmax : m_run;
         const float mc = (m_new == -INFINITY) ? 0.f : m_new * c;
-        // p = 2^(s c - m c), packed to bf16 pairs over S's first 64 columns
-        float sm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // p = 2^(s c - m c) on pairs, packed to bf16 over S's first 64 columns
+        float2 sm[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        const float2 c2 = make_float2(c, c), mc2 = make_float2(-mc, -mc);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pk[32];
+        for (int qd = 0; qd < 4; ++qd) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            // one pair in four goes to the FMA pipes
-            const float e0 = fmaf(x[64 * h + 2 * i], c, -mc), e1 = fmaf(x[64 * h + 2 * i + 1], c, -mc);
-            const float p0 = (i & 3) == 3 ? exp2_poly(e0) : ex2(e0);
-            const float p1 = (i & 3) == 3 ? exp2_poly(e1) : ex2(e1);
-            sm[i & 7] += p0 + p1;
-            pk[i] = pack_bf16(p0, p1);
+          for (int i = 0; i < 16; ++i) {
+            const float2 e = ffma2(make_float2(x[32 * qd + 2 * i], x[32 * qd + 2 * i + 1]), c2, mc2);
+            const float2 p = make_float2(ex2(e.x), ex2(e.y));
+            sm[i & 3] = fadd2(sm[i & 3], p);
+            pk[i] = pack_bf16(p.x, p.y);
           }
-          ptx::tmem_st32(tS + (uint32_t)(32 * h), pk);
+          ptx::tmem_st16(tS + (uint32_t)(16 * qd), pk);
         }
         const float alpha = rescale ? ex2(m_run * c - mc) : 1.f;  // 0 when m_run == -inf
         if (rescale) {
@@ -417,7 +423,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tmem_st32(tO + (uint32_t)(cc * 32), u);
           }
         }
-        l_run += ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
+        const float2 s01 = fadd2(sm[0], sm[1]), s23 = fadd2(sm[2], sm[3]);
+        const float2 s4 = fadd2(s01, s23);
+        l_run += s4.x + s4.y;
         ptx::tmem_st_wait();
         ptx::tc_fence_before();
         __syncwarp();

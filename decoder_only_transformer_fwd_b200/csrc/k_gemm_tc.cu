@@ -57,6 +57,13 @@ struct TcArgs {
   int tiles_m, tiles_n, num_tiles;
   int n_fastest;  // pair kernel: tile order with the column tile varying fastest
   int* status;
+  // pair kernel, stream-K schedule (see PairSched); sk_ws holds one fp32
+  // partial accumulator per CTA (128 x 256, column-major), sk_flags one word
+  // per CTA, set to sk_gen once that CTA's partial is written
+  int streamk;
+  float* sk_ws;
+  unsigned* sk_flags;
+  unsigned sk_gen;
 };
 
 // Pair tile pt -> (row-pair block, column tile).  Column-fastest order keeps
@@ -71,6 +78,94 @@ __device__ __forceinline__ void pair_tile(const TcArgs& a, int pt, int tiles_mp,
     mbp = pt % tiles_mp;
     nb = pt / tiles_mp;
   }
+}
+
+// Work of one CTA pair (cluster cid of ncl): njobs jobs, job j being pair
+// tile pt with k-blocks [kb_lo, kb_hi).  Plain schedule: tiles cid, cid + ncl,
+// ... with all k-blocks.  Stream-K schedule (data-parallel waves plus a split
+// tail): the W = num_pt / ncl full waves stay as they are (so the tiles in
+// flight at any time share their A rows in L2), and the k-blocks of the
+// num_pt % ncl tiles of the last, partial wave are cut into ncl equal ranges,
+// one per pair.  A range lies within one tile or spans the end of one tile
+// and the start of the next.  The pair whose range holds a tile's last
+// k-block finishes that tile (its "owner" job) after adding the partial sums
+// of the pairs before it that hold the tile's earlier k-blocks
+// ("contributor" jobs).  Order per pair: contributor job first, full waves,
+// owner job last, so the partials are written long before they are needed.
+struct PairSched {
+  int streamk, nk, cid, ncl, waves, tail_pt0;
+  long long u0, u1;        // this pair's range of tail (tile, k-block) units
+  int contrib, owner;      // has a contributor job / an owner job
+  int njobs;
+};
+
+__device__ __forceinline__ PairSched make_sched(const TcArgs& a, int num_pt, int nk, int cid, int ncl) {
+  PairSched s;
+  s.streamk = a.streamk;
+  s.nk = nk;
+  s.cid = cid;
+  s.ncl = ncl;
+  s.waves = num_pt / ncl;
+  s.tail_pt0 = s.waves * ncl;
+  s.u0 = s.u1 = 0;
+  s.contrib = s.owner = 0;
+  if (!a.streamk) {
+    s.njobs = cid < num_pt ? (num_pt - cid + ncl - 1) / ncl : 0;
+    return s;
+  }
+  const long long U = (long long)(num_pt - s.tail_pt0) * nk;
+  s.u0 = U * cid / ncl;
+  s.u1 = U * (cid + 1) / ncl;
+  if (s.u1 > s.u0) {
+    s.contrib = (s.u1 % nk) != 0;                                   // range ends inside a tile
+    s.owner = (s.u1 - s.u0) > (s.contrib ? s.u1 % nk : 0);          // it also holds some tile's end
+  }
+  s.njobs = s.contrib + s.waves + s.owner;
+  return s;
+}
+
+// kind: 0 full tile, 1 contributor (writes a partial), 2 owner (adds partials)
+__device__ __forceinline__ void job_at(const PairSched& s, int j, int& pt, int& kb_lo, int& kb_hi, int& kind) {
+  kind = 0;
+  if (!s.streamk) {
+    pt = s.cid + j * s.ncl;
+    kb_lo = 0;
+    kb_hi = s.nk;
+    return;
+  }
+  if (s.contrib && j == 0) {  // the start of the tile holding this range's end
+    const long long tt = (s.u1 - 1) / s.nk;
+    pt = s.tail_pt0 + (int)tt;
+    kb_lo = (int)(s.u0 > tt * s.nk ? s.u0 - tt * s.nk : 0);
+    kb_hi = (int)(s.u1 - tt * s.nk);
+    kind = 1;
+    return;
+  }
+  const int w = j - s.contrib;
+  if (w < s.waves) {
+    pt = s.cid + w * s.ncl;
+    kb_lo = 0;
+    kb_hi = s.nk;
+    return;
+  }
+  // the end of the tile holding this range's start
+  const long long tt = s.u0 / s.nk;
+  pt = s.tail_pt0 + (int)tt;
+  kb_lo = (int)(s.u0 - tt * s.nk);
+  kb_hi = s.nk;
+  kind = 2;
+}
+
+// Pairs whose contributor job is in tail tile tt, i.e. whose range ends
+// inside tt: a contiguous run of pairs just before the owner.
+__device__ __forceinline__ int first_contributor(const PairSched& s, long long U, long long tt) {
+  int c = s.cid;
+  while (c > 0) {
+    const long long u1p = U * c / s.ncl;  // end of pair c - 1's range
+    if (u1p <= tt * s.nk) break;
+    --c;
+  }
+  return c;
 }
 
 __device__ __forceinline__ float bits2f(uint32_t u) { return __uint_as_float(u); }
@@ -846,6 +941,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const int tiles_mp = (a.M + 2 * kBM - 1) / (2 * kBM);
   const int num_pt = tiles_mp * a.tiles_n;
   const int cid = (int)ptx::cluster_id_x(), ncl = (int)ptx::nclusters_x();
+  const PairSched sched = make_sched(a, num_pt, nk, cid, ncl);
 
   if (warp >= 8) {
     ptx::setmaxnreg_dec<kPairRegsLow>();
@@ -854,11 +950,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       // ---------------- TMA producer (both CTAs) ----------------
       int stage = 0;
       uint32_t ph = 0, issued = 0, par = 0;
-      for (int pt = cid; pt < num_pt; pt += ncl) {
+      for (int j = 0; j < sched.njobs; ++j) {
+        int pt, kb_lo, kb_hi, kind;
+        job_at(sched, j, pt, kb_lo, kb_hi, kind);
         int mbp, nb;
         pair_tile(a, pt, tiles_mp, mbp, nb);
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = kb_lo; kb < kb_hi; ++kb) {
           if (*abort_flag || !ptx::mbar_wait_cluster(empty(stage), ph ^ 1, a.status)) {
             *abort_flag = 1;
             ok = false;
@@ -887,7 +985,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       constexpr uint32_t idesc = ptx::idesc_bf16(2 * kBM, BN);
       int stage = 0, acc = 0;
       uint32_t ph = 0, aph = 0;
-      for (int pt = cid; pt < num_pt; pt += ncl) {
+      for (int j = 0; j < sched.njobs; ++j) {
+        int pt, kb_lo, kb_hi, kind;
+        job_at(sched, j, pt, kb_lo, kb_hi, kind);
         if (*abort_flag || !ptx::mbar_wait_cluster(tempty(acc), aph ^ 1, a.status)) {
           *abort_flag = 1;
           break;
@@ -895,7 +995,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         ptx::tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(acc * BN);
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = kb_lo; kb < kb_hi; ++kb) {
           if (*abort_flag || !ptx::mbar_wait_cluster(full(stage), ph, a.status)) {
             *abort_flag = 1;
             ok = false;
@@ -906,7 +1006,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           const uint64_t db = ptx::desc_kmajor_sw128(sB(stage));
 #pragma unroll
           for (int k = 0; k < kBK / kUK; ++k)
-            ptx::mma_bf16_ss2(d, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            ptx::mma_bf16_ss2(d, da + 2 * k, db + 2 * k, idesc, (kb != kb_lo || k != 0) ? 1u : 0u);
           ptx::mma_commit2_mc(empty(stage), 0x3);
           if (++stage == S) {
             stage = 0;
@@ -932,20 +1032,27 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     float* stage = epi_stage + ew * Cf::STAGE_FLOATS;
     int acc = 0;
     uint32_t aph = 0;
-    if (cid < num_pt) {
+    if (sched.njobs > 0) {
+      int pt, kb_lo, kb_hi, kind;
+      job_at(sched, 0, pt, kb_lo, kb_hi, kind);
       int mbp, nb;
-      pair_tile(a, cid, tiles_mp, mbp, nb);
+      pair_tile(a, pt, tiles_mp, mbp, nb);
       epilogue_prefetch<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, half, lane);
       epilogue_touch_outputs<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, half, lane);
     }
-    for (int pt = cid; pt < num_pt; pt += ncl) {
+    for (int j = 0; j < sched.njobs; ++j) {
+      int pt, kb_lo, kb_hi, kind;
+      job_at(sched, j, pt, kb_lo, kb_hi, kind);
+      const bool head = kind == 1;  // k-blocks of a tile another pair finishes: write a partial
+      const bool tail = kind == 2;  // finishes a tile: add the earlier pairs' partials
       int mbp, nb;
       pair_tile(a, pt, tiles_mp, mbp, nb);
       const RowPre pre = epilogue_pre<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, half, lane);
-      const int nxt = pt + ncl;
-      if (nxt < num_pt) {
+      if (j + 1 < sched.njobs) {
+        int ptn, kln, khn, kn;
+        job_at(sched, j + 1, ptn, kln, khn, kn);
         int mbn, nbn;
-        pair_tile(a, nxt, tiles_mp, mbn, nbn);
+        pair_tile(a, ptn, tiles_mp, mbn, nbn);
         epilogue_prefetch<BN, MODE>(ep, a, mbn * 2 + (int)rank, nbn, g, half, lane);
       }
       if (*abort_flag || !ptx::mbar_wait_cluster(tfull(acc), aph, a.status)) {
@@ -954,7 +1061,62 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
       ptx::tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(g * 32) << 16) + (uint32_t)(acc * BN);
-      epilogue_tile<BN, MODE>(ep, a, taddr, mbp * 2 + (int)rank, nb, g, half, lane, stage, pre);
+      // this CTA's 128 x 256 partial: column c, row r at slot * 32768 + c * 128 + r
+      const int row = g * 32 + lane;
+      const int col0 = half * (BN / 2);
+      if (head) {
+        float* slot = a.sk_ws + (size_t)(cid * 2 + (int)rank) * (128 * BN);
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+          uint32_t r[32];
+          ptx::tmem_ld32(taddr + (uint32_t)(col0 + c), r);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) slot[(size_t)(col0 + c + i) * 128 + row] = __uint_as_float(r[i]);
+        }
+        // all epilogue warps of this CTA have written their part before the flag
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory");
+        if (warp == 0 && lane == 0) {
+          __threadfence();
+          ptx::st_release_gpu(a.sk_flags + cid * 2 + (int)rank, a.sk_gen);
+        }
+      } else {
+        if (tail) {
+          // add the partials of the pairs before this one that hold the
+          // tile's earlier k-blocks (same CTA rank) into TMEM
+          const long long U = (long long)(num_pt - sched.tail_pt0) * nk;
+          const int c_first = first_contributor(sched, U, (long long)(pt - sched.tail_pt0));
+#pragma unroll 1
+          for (int cp = c_first; cp < cid; ++cp) {
+            if (U * (cp + 1) / ncl == U * cp / ncl) continue;  // pair cp has no tail units
+            const unsigned* flag = a.sk_flags + cp * 2 + (int)rank;
+            bool ready = ptx::ld_acquire_gpu(flag) == a.sk_gen;
+            if (!ready) {
+              const uint64_t t0 = ptx::globaltimer();
+              while (!(ready = ptx::ld_acquire_gpu(flag) == a.sk_gen))
+                if (ptx::globaltimer() - t0 > kWaitLimitNs) break;
+            }
+            if (!__all_sync(0xffffffffu, ready)) {
+              atomicOr(a.status, kStatusTimeout);
+              *abort_flag = 1;
+              break;
+            }
+            const float* slot = a.sk_ws + (size_t)(cp * 2 + (int)rank) * (128 * BN);
+#pragma unroll 1
+            for (int c = 0; c < BN / 2; c += 32) {
+              uint32_t r[32];
+              ptx::tmem_ld32(taddr + (uint32_t)(col0 + c), r);
+              ptx::tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                r[i] = __float_as_uint(__uint_as_float(r[i]) + slot[(size_t)(col0 + c + i) * 128 + row]);
+              ptx::tmem_st32(taddr + (uint32_t)(col0 + c), r);
+            }
+            ptx::tmem_st_wait();
+          }
+        }
+        epilogue_tile<BN, MODE>(ep, a, taddr, mbp * 2 + (int)rank, nb, g, half, lane, stage, pre);
+      }
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive_cluster(ptx::mapa(tempty(acc), 0));
@@ -1069,7 +1231,8 @@ bool make_tmap_4d(CUtensorMap* map, const void* ptr, const uint64_t (&dims)[4],
 int gemm_tc_bn(int N) { return (N % 256 == 0) ? 256 : 128; }
 
 bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int N, int K,
-                    const EpiParams& ep, int* status, int num_sms, cudaStream_t st, bool pair) {
+                    const EpiParams& ep, int* status, int num_sms, cudaStream_t st, bool pair,
+                    const StreamK* sk) {
   const int BN = gemm_tc_bn(N);
   if (pair && BN == 256 && num_sms >= 2) {
     // CTA pairs: each CTA loads 128 rows of A and 128 rows of B per k-slice
@@ -1087,6 +1250,22 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
     a.status = status;
     const int num_pt = ((M + 2 * kBM - 1) / (2 * kBM)) * a.tiles_n;
     const int ncl = num_pt < num_sms / 2 ? num_pt : num_sms / 2;
+    // stream-K when every pair's share spans at least two tiles and the
+    // buffers for the pairs' partial sums are there
+    const int nk = K / kBK;
+    a.streamk = 0;
+    a.sk_ws = nullptr;
+    a.sk_flags = nullptr;
+    a.sk_gen = 0;
+    // (and when the partial wave is at least a quarter full, so that a tile is
+    // cut among a few pairs only)
+    if (sk != nullptr && sk->ws != nullptr && ncl <= sk->max_pairs && ep.mode == EPI_BLOCK_END && nk >= 1 &&
+        num_pt >= ncl && num_pt % ncl != 0 && 4 * (num_pt % ncl) >= ncl) {
+      a.streamk = 1;
+      a.sk_ws = sk->ws;
+      a.sk_flags = sk->flags;
+      a.sk_gen = sk->gen;
+    }
     LaunchScope scope_(KK_GEMM_TC, st);
     return launch_pair(ta, tb, a, ep, ncl, st);
   }
@@ -1102,6 +1281,10 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
   a.num_tiles = a.tiles_m * a.tiles_n;
   a.n_fastest = 0;  // unused by the single-CTA kernel
   a.status = status;
+  a.streamk = 0;
+  a.sk_ws = nullptr;
+  a.sk_flags = nullptr;
+  a.sk_gen = 0;
   const int grid = a.num_tiles < num_sms ? a.num_tiles : num_sms;
   LaunchScope scope_(KK_GEMM_TC, st);
   return BN == 256 ? launch_bn<256>(ta, tb, a, ep, grid, st) : launch_bn<128>(ta, tb, a, ep, grid, st);

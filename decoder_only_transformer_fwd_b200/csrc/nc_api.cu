@@ -104,8 +104,13 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
+// CTA pairs the stream-K buffers of the workspace are sized for (a device
+// with more SMs than 2 * kStreamKPairs runs the GEMMs on the plain schedule)
+constexpr int kStreamKPairs = 96;
+
 struct Layout {
   size_t x, x0, xbo, xn, qkv, o, h, gate, ss, rcos, rsin, rfreq, ce_sum, ce_tgt, logits, tok, tgt, loss;
+  size_t skws, skflags;
   size_t total;
   int ce_tiles;
 };
@@ -154,6 +159,11 @@ Layout layout(const nc_config& c, int max_tokens) {
   L.ce_tgt = take(M * 4);
   const bool simt_head = c.dtype == NC_FP32 || c.gemm_impl != 0;
   L.logits = take(simt_head ? M * (size_t)c.vocab * 4 : 0);
+  // stream-K partial sums of the tcgen05 pair GEMM: one 128 x 256 fp32 tile
+  // per CTA of up to kStreamKPairs CTA pairs, and one flag word per CTA
+  const bool tc = c.dtype == NC_BF16 && c.gemm_impl == 0;
+  L.skws = take(tc ? (size_t)kStreamKPairs * 2 * 128 * 256 * 4 : 0);
+  L.skflags = take(tc ? (size_t)kStreamKPairs * 2 * 4 : 0);
   L.tok = take(M * 4);
   L.tgt = take(M * 4);
   L.loss = take(M * 4);
@@ -168,10 +178,10 @@ T* at(void* base, size_t off) {
 
 // C = A B^T with the given epilogue, on tensor cores (bf16) or CUDA cores.
 bool gemm(const nc_config& c, const DevInfo& d, const void* A, int lda, const void* B, int ldb, int M,
-          int N, int K, const EpiParams& ep, cudaStream_t st) {
+          int N, int K, const EpiParams& ep, cudaStream_t st, const StreamK* sk = nullptr) {
   if (c.dtype == NC_BF16 && c.gemm_impl == 0)
     return launch_gemm_tc((const bf16*)A, lda, (const bf16*)B, ldb, M, N, K, ep, d.status, d.num_sms, st,
-                          c.gemm_pair != 0);
+                          c.gemm_pair != 0, c.gemm_pair == 2 ? sk : nullptr);
   launch_gemm_simt(A, lda, B, ldb, M, N, K, c.dtype == NC_BF16, ep, st);
   return true;
 }
@@ -308,12 +318,25 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
   float* rfreq = at<float>(ws, Lw.rfreq);
   const size_t esz = bf ? 2 : 4;
 
-  int tbits = 1;
-  while ((1 << tbits) < T) ++tbits;
-  launch_rope_table(rcos, rsin, T, D, c.rope_base, st, rfreq, tbits);
   // tensor-core path: RMSNorm is fused into the GEMMs (producers write bf16(x)
   // and per-row sums of squares, consumers scale their rows by 1 / rms)
   const bool tc = bf && c.gemm_impl == 0;
+  // stream-K flags start at 0 each forward; every GEMM launch of the forward
+  // gets its own generation number
+  StreamK sk{nullptr, nullptr, 0u, kStreamKPairs};
+  if (tc) {
+    sk.ws = at<float>(ws, Lw.skws);
+    sk.flags = at<unsigned>(ws, Lw.skflags);
+    if (cudaMemsetAsync(sk.flags, 0, (size_t)kStreamKPairs * 2 * 4, st) != cudaSuccess) return NC_ERR_CUDA;
+  }
+  auto next_sk = [&]() -> const StreamK* {
+    if (!tc) return nullptr;
+    ++sk.gen;
+    return &sk;
+  };
+  int tbits = 1;
+  while ((1 << tbits) < T) ++tbits;
+  launch_rope_table(rcos, rsin, T, D, c.rope_base, st, rfreq, tbits);
   float* ss = at<float>(ws, Lw.ss);
   const int ss_parts = C / (gemm_tc_bn(C) / 2);
   bf16* xb = tc ? static_cast<bf16*>(xn) : nullptr;
@@ -364,7 +387,7 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
       e.n_kv_head = Hkv;
       e.vocab = V;
     }
-    if (!gemm(c, d, xn, C, lp.w_qkv, C, M, nqkv, C, e, st)) return NC_ERR_CUDA;
+    if (!gemm(c, d, xn, C, lp.w_qkv, C, M, nqkv, C, e, st, next_sk())) return NC_ERR_CUDA;
     if (!tc)
       launch_rope_qknorm_ve(qkv, nqkv, B, T, H, Hkv, D, rcos, rsin, c.qk_alpha, c.eps, tokens,
                             ve ? lp.ve : nullptr, gate, V, bf, d.status, st);
@@ -383,14 +406,14 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
     e.x = x;
     e.ldx = C;
     if (tc) norm_out(e);
-    if (!gemm(c, d, o, H * D, lp.w_o, H * D, M, C, H * D, e, st)) return NC_ERR_CUDA;
+    if (!gemm(c, d, o, H * D, lp.w_o, H * D, M, C, H * D, e, st, next_sk())) return NC_ERR_CUDA;
     // MLP sub-block
     if (!tc) launch_rmsnorm(x, xn, M, C, c.eps, bf, nullptr, 0, 0, 0.f, nullptr, st);
     e = epi(EPI_RELU2);
     e.out = h;
     e.ldo = c.mlp_hidden;
     if (tc) norm_in(e);
-    if (!gemm(c, d, xn, C, lp.w_fc1, C, M, c.mlp_hidden, C, e, st)) return NC_ERR_CUDA;
+    if (!gemm(c, d, xn, C, lp.w_fc1, C, M, c.mlp_hidden, C, e, st, next_sk())) return NC_ERR_CUDA;
     e = epi(EPI_BLOCK_END);
     e.x = x;
     e.x0 = x0;
@@ -406,7 +429,8 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
       e.beta = p->backout_lambda;
     }
     if (tc) norm_out(e);  // the next block's (or the head's) normalised input
-    if (!gemm(c, d, h, c.mlp_hidden, lp.w_fc2, c.mlp_hidden, M, C, c.mlp_hidden, e, st)) return NC_ERR_CUDA;
+    if (!gemm(c, d, h, c.mlp_hidden, lp.w_fc2, c.mlp_hidden, M, C, c.mlp_hidden, e, st, next_sk()))
+      return NC_ERR_CUDA;
   }
 
   // final norm, head, softcap, cross-entropy

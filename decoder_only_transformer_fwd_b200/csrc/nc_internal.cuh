@@ -145,8 +145,18 @@ void launch_attn_simt(const void* q, const void* k, const void* v, int ldq, int 
 // tcgen05 GEMM (bf16 only).  Returns false if the tensor maps cannot be built.
 int gemm_tc_bn(int N);  // output tile width the tcgen05 GEMM uses for N columns
 // pair = true selects the CTA-pair (cta_group::2) kernel when N % 256 == 0.
+// With sk given, the pair kernel may use a stream-K schedule: ws holds
+// 2 * max_pairs partial tiles of 128 x 256 floats, flags 2 * max_pairs words
+// that start below gen (gen must differ between launches that share them).
+struct StreamK {
+  float* ws;
+  unsigned* flags;
+  unsigned gen;
+  int max_pairs;
+};
 bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int N, int K,
-                    const EpiParams& ep, int* status, int num_sms, cudaStream_t st, bool pair);
+                    const EpiParams& ep, int* status, int num_sms, cudaStream_t st, bool pair,
+                    const StreamK* sk = nullptr);
 // tcgen05 attention (bf16 only)
 bool launch_attn_tc(const bf16* q, const bf16* k, const bf16* v, int ldq, int ldk, int ldv, bf16* o,
                     int ldo, int B, int T, int H, int Hkv, int window, float scale, int* status,

@@ -69,7 +69,10 @@ typedef struct nc_config {
   int smear;              /* 1 = smear gate on                                  */
   int gemm_impl;          /* 0 = tensor cores (tcgen05) in bf16 mode, 1 = CUDA-core GEMM */
   int attn_impl;          /* 0 = tensor cores (tcgen05) in bf16 mode, 1 = CUDA-core attention */
-  int gemm_pair;          /* 1 = tcgen05 GEMMs on CTA pairs (cta_group::2, 256 x 256 tiles) where N % 256 == 0 */
+  int gemm_pair;          /* 1 = tcgen05 GEMMs on CTA pairs (cta_group::2, 256 x 256 tiles) where N % 256 == 0;
+                            2 = the same, and for the MLP down-projection the k-blocks of its partial last
+                            wave of tiles are split evenly over all CTA pairs (partial sums pass through the
+                            workspace); measured slower than 1 at d24, kept as an option */
   float qk_alpha;         /* 1.15 ([Math] §QK-Norm with Sharpening)              */
   float softmax_scale;    /* 1/sqrt(D)                                          */
   float rope_base;        /* 100000                                             */

@@ -110,11 +110,14 @@ def test_fp32_ragged_window_one():
     _compare(loss, ref_loss, logits, ref_logits, "fp32")
 
 
-@pytest.mark.parametrize("name,rows", [("d12", [0, 5]), ("d24", [2])])
-def test_full_size_sampled_rows(name, rows):
+@pytest.mark.parametrize("name,rows,gemm_pair", [("d12", [0, 5], 1), ("d24", [2], 1), ("d24", [1], 2)])
+def test_full_size_sampled_rows(name, rows, gemm_pair):
+    """gemm_pair = 2 splits the partial last wave of FC2's tiles along K
+    (partial sums through the workspace); at d24 that schedule is in use."""
     w = synth.WORKLOADS[name]
     seed = synth.SEED_BASE + w["index"]
     cfg, ocfg, p, tok, tgt = make_case(w["depth"], w["B"], w["T"], w["short"], w["dtype"], seed)
+    cfg.gemm_pair = gemm_pair
     loss, _, rc, _ = run_gpu(cfg, p, tok, tgt)
     assert rc == 0
     ref_loss, _ = O.forward(ocfg, p, tok, tgt, rows=rows)
