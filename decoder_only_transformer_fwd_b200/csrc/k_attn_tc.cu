@@ -248,24 +248,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto slot_wait = [&](int sc) -> bool {
         return !*abort_flag && ptx::mbar_wait(bar(B_SLF + sc % SLOTS), (uint32_t)(sc / SLOTS) & 1u, a.status);
       };
+      // shared-memory descriptors are built once; the k-steps add constants
+      // to their start-address field (16-byte units): K-major steps of 16
+      // elements are 32 B within a 64-column box and BOX_BYTES between the
+      // two boxes; the MN-major V steps are 16 rows = 2048 B
+      const uint64_t dq0 = ptx::desc_kmajor_sw128(sQ(0)), dq1 = ptx::desc_kmajor_sw128(sQ(1));
+      const uint64_t dk0 = ptx::desc_kmajor_sw128(sSlot(0)), dv0 = ptx::desc_mnmajor_sw128(sSlot(0), BOX_BYTES);
+      auto slot_off = [&](int sc) { return (uint64_t)((sc % SLOTS) * (TILE_BYTES >> 4)); };
       auto qk = [&](int g, int sc) {
         const uint32_t tS = tmem + (uint32_t)(g * 128);
-        const uint32_t k = sSlot(sc % SLOTS);
+        const uint64_t dq = g == 0 ? dq0 : dq1, dk = dk0 + slot_off(sc);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (uint32_t)((kk >> 2) * BOX_BYTES + (kk & 3) * 32);
-          ptx::mma_bf16_ss(tS, ptx::desc_kmajor_sw128(sQ(g) + off), ptx::desc_kmajor_sw128(k + off), idesc_qk,
-                           kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
+          ptx::mma_bf16_ss(tS, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto pv = [&](int g, int sc, bool first) {
         const uint32_t tP = tmem + (uint32_t)(g * 128);  // P_g: packed bf16 over the first 64 columns of S_g
         const uint32_t tO = tmem + 256 + (uint32_t)(g * 128);
-        const uint32_t v = sSlot(sc % SLOTS);
+        const uint64_t dv = dv0 + slot_off(sc);
 #pragma unroll
         for (int kk = 0; kk < kK / 16; ++kk)
-          ptx::mma_bf16_ts(tO, tP + (uint32_t)(kk * 8), ptx::desc_mnmajor_sw128(v + (uint32_t)(kk * 2048), BOX_BYTES),
-                           idesc_pv, (!first || kk > 0) ? 1u : 0u);
+          ptx::mma_bf16_ts(tO, tP + (uint32_t)(kk * 8), dv + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
+                           (!first || kk > 0) ? 1u : 0u);
       };
       bool ok = true;
       int sc = 0, it = 0;
