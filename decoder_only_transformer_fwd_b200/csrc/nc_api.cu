@@ -118,7 +118,7 @@ struct Layout {
 bool config_ok(const nc_config& c) {
   if (c.n_layer <= 0 || c.n_layer > NC_MAX_LAYERS) return false;
   if (c.n_embd <= 0 || c.n_embd % 128 != 0) return false;
-  if (c.head_dim != 128 || c.n_head <= 0 || c.n_kv_head != c.n_head) return false;
+  if (c.head_dim != 128 || c.n_head <= 0 || c.n_kv_head <= 0 || c.n_head % c.n_kv_head != 0) return false;
   if (c.vocab <= 0 || c.vocab_padded < c.vocab || c.vocab_padded % 64 != 0) return false;
   if (c.mlp_hidden <= 0 || c.mlp_hidden % 128 != 0) return false;
   if (c.max_T <= 0 || (c.dtype != NC_BF16 && c.dtype != NC_FP32)) return false;
@@ -516,7 +516,7 @@ int nc_attention(const void* q, const void* k, const void* v, void* out, int B, 
   if (dtype != NC_BF16 && dtype != NC_FP32) return NC_ERR_ARG;
   if (!(softmax_scale > 0.f) || !(eps >= 0.f)) return NC_ERR_ARG;
   if (B <= 0 || T <= 0 || H <= 0 || Hkv <= 0) return NC_ERR_SHAPE;
-  if (D != 128 || Hkv != H) return NC_ERR_SHAPE;
+  if (D != 128 || Hkv <= 0 || H % Hkv != 0) return NC_ERR_SHAPE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return NC_ERR_ALIGN;
   const size_t need = nc_attention_workspace_bytes(B, T, H, Hkv, D, dtype, rope_qknorm);
   if (rope_qknorm && (workspace == nullptr || workspace_bytes < need)) return NC_ERR_WORKSPACE;

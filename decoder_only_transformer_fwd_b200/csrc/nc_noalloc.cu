@@ -56,7 +56,7 @@ extern "C" int nc_attention_noalloc(const void* q, const void* k, const void* v,
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return NC_ERR_ARG;
   if (dtype != NC_BF16 && dtype != NC_FP32) return NC_ERR_ARG;
   if (!(softmax_scale > 0.f) || !(eps >= 0.f)) return NC_ERR_ARG;
-  if (B <= 0 || T <= 0 || H <= 0 || Hkv <= 0 || D != 128 || Hkv != H) return NC_ERR_SHAPE;
+  if (B <= 0 || T <= 0 || H <= 0 || Hkv <= 0 || D != 128 || H % Hkv != 0) return NC_ERR_SHAPE;
   const uintptr_t mis = (reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
                          reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out)) & 15u;
   if (mis) return NC_ERR_ALIGN;

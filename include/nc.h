@@ -55,7 +55,7 @@ typedef struct nc_config {
   int n_layer;            /* L, the depth                                       */
   int n_embd;             /* C = ceil(64 L / 128) * 128 ([Math] §Architecture Overview) */
   int n_head;             /* H = C / 128                                        */
-  int n_kv_head;          /* H_kv (= H; the kernels require H_kv == H)          */
+  int n_kv_head;          /* H_kv, a divisor of H: query head h reads k/v head h / (H / H_kv) */
   int head_dim;           /* D = 128 (the kernels require 128)                  */
   int vocab;              /* V = 32768                                          */
   int vocab_padded;       /* V rounded up to a multiple of 64 ([Source] §5.4)   */
@@ -130,7 +130,7 @@ int nc_params_init(nc_params* p, const nc_config* cfg);
  *   out_logits_opt [B*T, V] fp32 softcapped logits 15 tanh(z/15), or NULL
  *     (when NULL the logits are never written to memory in bf16 mode).
  * Requires B*T <= p->max_tokens, T <= cfg.max_T, C % 128 == 0, D == 128,
- * H_kv == H, all pointers 16-byte aligned. */
+ * H % H_kv == 0, all pointers 16-byte aligned. */
 int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets, int B, int T,
                float* out_loss, float* out_logits_opt, void* stream);
 
@@ -157,7 +157,8 @@ size_t nc_attention_workspace_bytes(int B, int T, int H, int Hkv, int D, int dty
  *   to the workspace; with 0 they are used as given.
  *   o_i = sum_j softmax_j(softmax_scale * qhat_i . khat_j) v_j over j <= i,
  *   i - j < window; window <= 0 or >= T means plain causal.
- * Requires D == 128, H_kv == H, softmax_scale > 0, eps >= 0, 16-byte aligned
+ * Query head h attends with k/v head h / (H / H_kv) (grouped-query attention).
+ * Requires D == 128, H % H_kv == 0, softmax_scale > 0, eps >= 0, 16-byte aligned
  * pointers (NC_ERR_SHAPE / NC_ERR_ARG / NC_ERR_ALIGN otherwise). */
 int nc_attention(const void* q, const void* k, const void* v, void* out, int B, int T, int H,
                  int Hkv, int D, int window, int rope_qknorm, float alpha, float softmax_scale,

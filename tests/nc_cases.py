@@ -6,10 +6,12 @@ from decoder_only_transformer_fwd_b200 import nc, synth
 from oracle import nanochat_fwd as O
 
 
-def make_case(depth, B, T, short, dtype, seed, *, max_T=None, pattern="SSSL", layers=None):
+def make_case(depth, B, T, short, dtype, seed, *, max_T=None, pattern="SSSL", layers=None, n_kv_head=None):
     max_T = T if max_T is None else max_T
     cfg = nc.nc_init_config(depth, max_T, dtype, pattern, short, -1)
-    ocfg = O.make_config(depth, max_T, short, pattern=pattern)
+    if n_kv_head is not None:
+        cfg.n_kv_head = n_kv_head
+    ocfg = O.make_config(depth, max_T, short, pattern=pattern, n_kv_head=n_kv_head)
     params = synth.params(seed, n_layer=cfg.n_layer, n_embd=cfg.n_embd, n_head=cfg.n_head,
                           n_kv_head=cfg.n_kv_head, head_dim=cfg.head_dim, vocab=cfg.vocab,
                           vocab_padded=cfg.vocab_padded, ve_layers=ocfg["ve_layers"],

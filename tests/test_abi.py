@@ -80,7 +80,10 @@ def test_workspace_bytes():
     # bf16 mode never materialises the logits; fp32 mode may
     cfg32 = nc.nc_init_config(24, 2048, "fp32", "SSSL", 1024)
     assert nc.nc_workspace_bytes(cfg32, 8192) > w1 + 8192 * 32768 * 4
-    cfg.n_kv_head = 6            # unsupported: H_kv != H
+    cfg.n_kv_head = 4            # grouped-query attention: 3 query heads per k/v head
+    w_gqa = nc.nc_workspace_bytes(cfg, 8192)
+    assert 0 < w_gqa < w1
+    cfg.n_kv_head = 5            # unsupported: H_kv does not divide H
     assert nc.nc_workspace_bytes(cfg, 8192) == 0
 
 
@@ -128,7 +131,8 @@ def test_attention_rejects_bad_arguments():
                                 a["ws"], a["wsb"], None)
     assert call(args(q=None)) == nc.STATUS_CODES["NC_ERR_ARG"]
     assert call(args(D=64)) == nc.STATUS_CODES["NC_ERR_SHAPE"]
-    assert call(args(Hkv=2, H=4)) == nc.STATUS_CODES["NC_ERR_SHAPE"]
+    assert call(args(Hkv=3, H=4)) == nc.STATUS_CODES["NC_ERR_SHAPE"]  # H_kv must divide H
+    assert call(args(Hkv=0, H=4)) == nc.STATUS_CODES["NC_ERR_SHAPE"]
     assert call(args(T=0)) == nc.STATUS_CODES["NC_ERR_SHAPE"]
     assert call(args(dt=5)) == nc.STATUS_CODES["NC_ERR_ARG"]
     assert call(args(scale=0.0)) == nc.STATUS_CODES["NC_ERR_ARG"]

@@ -52,6 +52,19 @@ def test_attention_small(B, T, H, window, dtype):
         assert err <= tol, (b, err)
 
 
+@pytest.mark.parametrize("B,T,H,Hkv,window,dtype", [
+    (2, 300, 4, 2, 96, "bf16"), (1, 200, 6, 3, 0, "bf16"), (2, 257, 4, 1, 1, "bf16"), (2, 130, 4, 2, 129, "fp32")])
+def test_attention_grouped_query(B, T, H, Hkv, window, dtype):
+    """H_kv < H: query head h attends with k/v head h / (H / H_kv)."""
+    q, k, v = synth.attention_inputs(700 + T, B, T, H, 128, Hkv=Hkv, bf16=(dtype == "bf16"))
+    out = _run(q, k, v, window, dtype)
+    tol = 2e-2 if dtype == "bf16" else 1e-4
+    for b in range(B):
+        ref = _ref(q[b], k[b], v[b], window)
+        err = np.max(np.abs(out[b] - ref))
+        assert err <= tol, (b, err)
+
+
 @pytest.mark.parametrize("T,window", synth.ATTN_SWEEP["cases"])
 def test_attention_sweep_sampled(T, window):
     s = synth.ATTN_SWEEP

@@ -78,6 +78,18 @@ def test_d4_bf16_full(gemm_impl, attn_impl, gemm_pair):
     _compare(loss, ref_all, dtype="bf16")
 
 
+@pytest.mark.parametrize("depth,B,T,short,n_kv_head", [(4, 2, 512, 256, 1), (12, 1, 384, 128, 2), (12, 1, 256, 64, 3)])
+def test_grouped_query_attention_forward(depth, B, T, short, n_kv_head):
+    """H_kv < H: query head h reads k/v head h / (H / H_kv); the k/v and
+    value-embedding widths shrink with H_kv (d4: H = 2; d12: H = 6)."""
+    cfg, ocfg, p, tok, tgt = make_case(depth, B, T, short, "bf16", 300 + n_kv_head, n_kv_head=n_kv_head)
+    assert cfg.n_kv_head == n_kv_head < cfg.n_head
+    loss, logits, rc, _ = run_gpu(cfg, p, tok, tgt, want_logits=True)
+    assert rc == 0
+    ref_loss, ref_logits = O.forward(ocfg, p, tok, tgt, rows=[0], want_logits=True)
+    _compare(loss[:1], ref_loss, logits[:1], ref_logits, "bf16")
+
+
 def test_tc_gemm_matches_cuda_core_gemm():
     """The tcgen05 and CUDA-core GEMMs round at the same points but sum in a
     different order; in bf16 that alone moves per-token losses by the bf16
