@@ -5,9 +5,9 @@
 // with Sliding Window: query i sees key j iff j <= i and i - j < w;
 // o_i = sum_j softmax_j(scale q_i . k_j) v_j.
 //
-// Persistent: one CTA per SM walks work items, heaviest first.  An item is a
-// pair of adjacent 128-query tiles (A, B) of one head, which share one stream
-// of 128-key K/V tiles:
+// Persistent: one CTA per SM walks work items, heaviest first, in rounds of
+// alternating direction.  An item is a pair of adjacent 128-query tiles
+// (A, B) of one head, which share one stream of 128-key K/V tiles:
 //   warps 0..3  softmax of tile A, one query row per thread (its TMEM lane);
 //   warps 4..7  softmax of tile B;
 //   warp 8      TMA: the item's two Q tiles, then K_t and V_t for every key
@@ -105,6 +105,15 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, int i) {
   return it;
 }
 
+// The k-th item of this CTA.  Rounds of gridDim.x items alternate direction
+// (forward, then backward over the CTAs), so with items ordered heaviest first
+// the CTA that took the heaviest item of one round takes the lightest of the
+// next: per-CTA totals stay close to the mean without any atomics.
+__device__ __forceinline__ int item_of(int k) {
+  const int g = (int)gridDim.x, c = (int)blockIdx.x;
+  return k * g + ((k & 1) ? g - 1 - c : c);
+}
+
 __device__ __forceinline__ bool active(const Item& it, int g, int t) {
   return g == 0 ? (t >= it.lo0 && t <= it.hi0) : (it.has_b && t >= it.lo1 && t <= it.hi1);
 }
@@ -200,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t issued = 0, par = 0, qpar = 0;
       bool qissued = false, ok = true;
       int sc = 0, it = 0;
-      for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x, ++it) {
+      for (int item = item_of(0); ok && item < a.n_items; ++it, item = item_of(it)) {
         const Item w = decode_item(a, item);
         const int row_base = w.b * a.T;
         const int qcol = w.h * kD, kcol = (w.h / (a.H / a.Hkv)) * kD;
@@ -276,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       int sc = 0, it = 0;
       int pc0 = 0, pc1 = 0, ic0 = 0, ic1 = 0;  // P phases consumed, items finished, per group
-      for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x, ++it) {
+      for (int item = item_of(0); ok && item < a.n_items; ++it, item = item_of(it)) {
         const Item w = decode_item(a, item);
         if (*abort_flag || !ptx::mbar_wait(bar(B_QF), it & 1, a.status)) { ok = false; break; }
         ptx::tc_fence_after();
@@ -345,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = a.scale_log2;
     bool ok = true;
     int cnt = 0, icnt = 0;
-    for (int item = blockIdx.x; ok && item < a.n_items; item += gridDim.x) {
+    for (int k = 0, item = item_of(0); ok && item < a.n_items; ++k, item = item_of(k)) {
       const Item w = decode_item(a, item);
       if (g == 1 && !w.has_b) continue;
       const int qg = w.q0 + g * kQ;  // first query of this group's tile
