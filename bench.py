@@ -210,6 +210,51 @@ def attention_sweep(args, dev, stream):
     return out
 
 
+def generation_step(args, model, cfg, tok, B, T, stream, peaks):
+    """One generation step at the bench workload's sizes (nc_generate_next):
+    the forward over [B, T], the last-position logits, one token per row drawn
+    with temperature 0.8 and top-k 50.  Device time per step (CUDA events), and
+    per-launch times of the two kernels that are specific to it."""
+    import torch
+
+    from decoder_only_transformer_fwd_b200 import nc, synth
+    tau, k = 0.8, 50
+    u = torch.from_numpy(synth.uniforms(synth.SEED_BASE, B)).to(tok.device)
+    nxt = torch.empty(B, dtype=torch.int32, device=tok.device)
+    z = torch.empty(B, cfg.vocab, dtype=torch.float32, device=tok.device)
+    call = lambda: nc.nc_generate_next(model.params, tok, tau, k, u, nxt, z, stream)
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    per_call = nc.nc_last_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    timer = nc.LaunchTimer(args.steps * 2, kinds=["last_logits", "sample"])
+    with timer:
+        for _ in range(args.steps):
+            call()
+    torch.cuda.synchronize()
+    pk = timer.per_kind()
+    n_ll, ms_ll = pk.get("last_logits", (0, 0.0))
+    n_s, ms_s = pk.get("sample", (0, 0.0))
+    us_ll = 1e3 * ms_ll / max(n_ll, 1)
+    # algorithmic bytes of one k_last_logits launch: W_U [V, C] bf16 once, the
+    # B final residual rows (fp32) and the B x V fp32 logits written
+    nbytes = cfg.vocab * cfg.n_embd * 2 + B * cfg.n_embd * 4 + B * cfg.vocab * 4
+    gbs = nbytes / (us_ll * 1e-6) / 1e9 if us_ll > 0 else None
+    return {"workload": f"next-token step: forward over B={B} x T={T}, head on the last position only, "
+                        f"temperature {tau}, top-k {k}",
+            "ms_per_step": ms, "tokens_per_s": B / (ms / 1e3), "launches_per_step": per_call,
+            "last_logits_us": us_ll, "sample_us": 1e3 * ms_s / max(n_s, 1),
+            "last_logits_roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                     "frac": gbs / peaks["hbm_gbs"] if gbs else None, "bytes_per_launch": nbytes}}
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -315,6 +360,9 @@ def run_ours(args):
         nc.nc_forward_host(model.params, h_tok, h_tgt, h_loss, stream)
     e2e_s = max_over_ranks(time.perf_counter() - t0)
     attn = None if args.no_attention_sweep else attention_sweep(args, dev, stream)
+    gen = None
+    if not args.no_generation and not args.layers:
+        gen = generation_step(args, model, cfg, tok, B, T, stream, load_peaks()[0])
     clk = clocks.stop()
     rc, bits = nc.nc_get_status(stream)
     if rc != 0:
@@ -344,6 +392,15 @@ def run_ours(args):
         "launches": n_gemm, "avg_launch_us": 1e3 * gemm_ms / max(n_gemm, 1),
         "share_of_step": gemm_ms / ms_total if ms_total > 0 else None,
     }
+
+    # the embedding kernel is HBM-bound: per launch it gathers M rows of W_E
+    # (bf16) and writes x, x0 (fp32) and bf16(x) for the first norm
+    n_emb, ms_emb = per_kind.get("embed_norm_smear", (0, 0.0))
+    emb_bytes = M * cfg.n_embd * (2 + 4 + 4 + 2)
+    emb_gbs = emb_bytes / (ms_emb / max(n_emb, 1) / 1e3) / 1e9 if ms_emb > 0 else None
+    embed_roofline = {"kernel": "k_embed", "bound": "hbm", "achieved": emb_gbs, "peak": peaks["hbm_gbs"],
+                      "unit": "GB/s", "frac": emb_gbs / peaks["hbm_gbs"] if emb_gbs else None,
+                      "bytes_per_launch": emb_bytes}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -381,7 +438,9 @@ def run_ours(args):
             # region B's step time minus the summed kernel times: launch gaps,
             # pipeline fill/drain between kernels and the timing events themselves
             "gap_ms_per_step": ms_step_b - sum(v[1] for v in per_kind.values()) / args.steps,
+            "embed_roofline": embed_roofline,
             "attention_sweep": attn,
+            "generation": gen,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -399,6 +458,7 @@ def main():
     ap.add_argument("--cpu-tokens", type=int, default=1024)
     ap.add_argument("--rows", type=int, default=0, help="rows per step (default: the workload's B = 4)")
     ap.add_argument("--no-attention-sweep", action="store_true")
+    ap.add_argument("--no-generation", action="store_true", help="skip the generation-step measurement")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling only: keep the first N blocks of the d24 stack (1..24)")
     args = ap.parse_args()

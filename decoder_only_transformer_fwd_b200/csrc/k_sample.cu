@@ -1,0 +1,481 @@
+// Next-token step of generation: the softcapped logits of the last position
+// of each row, then one token per row drawn from them.
+//
+// "The Mathematics of Karpathy's nanochat", §Inference: Generating Text: a
+// forward pass gives the logits z in R^V at the last position only; §Sampling
+// Controls: top-k keeps the entries z_v >= (k-th largest z), temperature tau
+// divides them, P(v) = exp(z_v / tau) / sum_v' exp(z_v' / tau), one index is
+// drawn from P; tau = 0 is greedy decoding (argmax).  §Logit Softcap:
+// z = cap * tanh(x_L W_U^T / cap) with x_L = RMSNorm(final residual).
+//
+// The draw takes its uniform number u in [0, 1) from the caller: the index is
+// the first v (vocabulary order) whose cumulative weight exceeds u * sum.
+#include "nc_internal.cuh"
+#include "ptx.cuh"
+
+namespace nc {
+
+namespace {
+
+constexpr int kLastRows = 8;      // rows of one k_last_logits launch
+constexpr int kMaxLastC = 4096;   // widest model row it stages (8 x 4096 fp32 = 128 KB)
+
+// W_U and the staged rows of x share one element type: bf16 in bf16 mode
+// (x rounded to bf16, as the head GEMM of the full forward rounds it), fp32
+// otherwise.  A 16-byte chunk holds 8 or 4 of them, unpacked to fp32 pairs.
+template <typename TW> struct Chunk;
+template <> struct Chunk<bf16> {
+  static constexpr int kN = 8;
+  __device__ static void unpack(const uint4& u, float2* f) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+  }
+  __device__ static bf16 round(float v) { return __float2bfloat16_rn(v); }
+};
+template <> struct Chunk<float> {
+  static constexpr int kN = 4;
+  __device__ static void unpack(const uint4& u, float2* f) {
+    f[0] = make_float2(__uint_as_float(u.x), __uint_as_float(u.y));
+    f[1] = make_float2(__uint_as_float(u.z), __uint_as_float(u.w));
+  }
+  __device__ static float round(float v) { return v; }
+};
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+// k_last_logits: warps 0..7 multiply, warp 8 streams W_U into the ring
+constexpr int kLastConsumers = 8;
+constexpr int kLastThreads = 32 * (kLastConsumers + 1);
+constexpr int kLastR = 2;  // vocabulary rows a consumer warp multiplies together
+
+// The ring geometry for rows of `row_bytes`: `rows` vocabulary rows per stage
+// (about 48 KB), `stages` stages, and the shared-memory bytes of the launch
+// (ring, staged x rows, barriers).
+struct LastGeom {
+  int rows, stages;
+  size_t stage_bytes, x_bytes, smem;
+};
+inline LastGeom last_geom(int C, int esz, int nb) {
+  LastGeom g;
+  const size_t row_bytes = (size_t)C * esz;
+  g.rows = (int)(49152 / row_bytes);
+  g.rows = g.rows < 1 ? 1 : (g.rows > 32 ? 32 : g.rows);
+  g.stage_bytes = (size_t)g.rows * row_bytes;
+  g.x_bytes = (size_t)nb * row_bytes;
+  const size_t budget = 220 * 1024 - g.x_bytes - 1024;
+  g.stages = (int)(budget / g.stage_bytes);
+  g.stages = g.stages > 4 ? 4 : g.stages;
+  g.smem = g.stages * g.stage_bytes + g.x_bytes + 2 * 4 * 8 + 128;
+  return g;
+}
+
+// logits[b0 + j][v] = cap * tanh(rs_j * (x_j . W_U[v]) / cap) for the NB rows
+// x_j = x[(b0 + j) T + T - 1], rs_j = 1 / sqrt(mean(x_j^2) + eps).  One CTA
+// per SM; CTA c takes the blocks of `rows` consecutive vocabulary rows
+// c, c + G, c + 2G, ...  One thread copies each block (contiguous in W_U)
+// into a ring of shared-memory stages with a bulk copy; the consumer warps
+// multiply two rows at a time against the staged x rows and release the stage.
+template <typename TW, int NB>
+__global__ void __launch_bounds__(kLastThreads, 1)
+k_last_logits(const float* __restrict__ x, int ldx, int T, int b0, const TW* __restrict__ W, int V, int C,
+              float cap, float eps, float* __restrict__ out, int ldo, int rows, int stages, int* status) {
+  pdl_launch_dependents();
+  extern __shared__ __align__(16) unsigned char sh_raw[];
+  const size_t row_bytes = (size_t)C * sizeof(TW);
+  const size_t stage_bytes = (size_t)rows * row_bytes;
+  unsigned char* ring = sh_raw;
+  TW* xs = reinterpret_cast<TW*>(sh_raw + stages * stage_bytes);  // [NB][C]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sh_raw + stages * stage_bytes + NB * row_bytes);
+  __shared__ float red[32];
+  __shared__ float rs[NB];
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto full = [&](int s) { return ptx::smem_u32(bars + s); };
+  auto empty = [&](int s) { return ptx::smem_u32(bars + 4 + s); };
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      ptx::mbar_init(full(s), 1);
+      ptx::mbar_init(empty(s), kLastConsumers);
+    }
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_wait();
+  const int nblk = (V + rows - 1) / rows;
+  if (warp == kLastConsumers) {
+    if (lane == 0) {
+      int k = 0;
+      for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x, ++k) {
+        const int s = k % stages;
+        const uint32_t ph = (uint32_t)(k / stages) & 1u;
+        if (abort_flag || !ptx::mbar_wait(empty(s), ph ^ 1u, status)) { abort_flag = 1; break; }
+        const int r0 = blk * rows;
+        const int nr = V - r0 < rows ? V - r0 : rows;
+        const uint32_t bytes = (uint32_t)(nr * row_bytes);
+        ptx::mbar_arrive_expect_tx(full(s), bytes);
+        ptx::bulk_load(ptx::smem_u32(ring + s * stage_bytes), W + (size_t)r0 * C, bytes, full(s));
+      }
+      // every copy this thread issued has landed before the CTA may exit
+      const int issued = k;
+      for (int q = issued - stages > 0 ? issued - stages : 0; q < issued; ++q)
+        ptx::mbar_wait(full(q % stages), (uint32_t)(q / stages) & 1u, status);
+    }
+    return;
+  }
+  // consumers: stage the NB rows of x (while the first blocks stream in)
+#pragma unroll 1
+  for (int j = 0; j < NB; ++j) {
+    const float* xr = x + ((size_t)(b0 + j) * T + (T - 1)) * ldx;
+    float sq = 0.f;
+    for (int c = threadIdx.x; c < C; c += 32 * kLastConsumers) {
+      const float v = xr[c];
+      sq += v * v;
+      xs[(size_t)j * C + c] = Chunk<TW>::round(v);
+    }
+    sq = warp_sum(sq);
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * kLastConsumers));
+    if (lane == 0) red[warp] = sq;
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * kLastConsumers));
+    if (threadIdx.x == 0) {
+      float t = 0.f;
+      for (int w = 0; w < kLastConsumers; ++w) t += red[w];
+      rs[j] = rsqrtf(t / (float)C + eps);
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(32 * kLastConsumers));
+  constexpr int kN = Chunk<TW>::kN;
+  const int nchunks = C / kN;
+  const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
+  int k = 0;
+  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x, ++k) {
+    const int s = k % stages;
+    if (abort_flag || !ptx::mbar_wait(full(s), (uint32_t)(k / stages) & 1u, status)) { abort_flag = 1; break; }
+    const int r0 = blk * rows;
+    const int nr = V - r0 < rows ? V - r0 : rows;
+    const uint4* st4 = reinterpret_cast<const uint4*>(ring + s * stage_bytes);
+    for (int r = kLastR * warp; r < nr; r += kLastR * kLastConsumers) {
+      const bool two = r + 1 < nr;
+      float2 acc[kLastR][NB];
+#pragma unroll
+      for (int q = 0; q < kLastR; ++q)
+#pragma unroll
+        for (int j = 0; j < NB; ++j) acc[q][j] = make_float2(0.f, 0.f);
+#pragma unroll 2
+      for (int ci = lane; ci < nchunks; ci += 32) {
+        float2 wf[kLastR][kN / 2];
+        Chunk<TW>::unpack(st4[(size_t)r * nchunks + ci], wf[0]);
+        Chunk<TW>::unpack(two ? st4[(size_t)(r + 1) * nchunks + ci] : make_uint4(0u, 0u, 0u, 0u), wf[1]);
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+          float2 xf[kN / 2];
+          Chunk<TW>::unpack(xs4[(size_t)j * nchunks + ci], xf);
+#pragma unroll
+          for (int q = 0; q < kLastR; ++q)
+#pragma unroll
+            for (int e = 0; e < kN / 2; ++e) acc[q][j] = ffma2(wf[q][e], xf[e], acc[q][j]);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < kLastR; ++q) {
+        float mine = 0.f;
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+          const float sj = warp_sum(acc[q][j].x + acc[q][j].y);
+          if (lane == j) mine = sj;
+        }
+        if (lane < NB && (q == 0 || two)) out[(size_t)(b0 + lane) * ldo + r0 + r + q] = cap * tanhf(mine * rs[lane] / cap);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(empty(s));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// sampling, one CTA of 1024 threads per row
+// ---------------------------------------------------------------------------
+
+constexpr int kSampleThreads = 1024;
+// a row of up to this many bytes of logits is staged in shared memory
+constexpr size_t kSampleSmemMax = 160 * 1024;
+
+// order-preserving map of a float to an unsigned key (larger float, larger
+// key); -0 maps with +0, as the two compare equal
+__device__ __forceinline__ uint32_t fkey(float f) {
+  uint32_t u = __float_as_uint(f);
+  u = (u == 0x80000000u) ? 0u : u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float unkey(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+__global__ void __launch_bounds__(kSampleThreads, 1)
+k_sample(const float* __restrict__ logits, int V, int ldl, float temperature, int top_k,
+         const float* __restrict__ uniforms, int32_t* __restrict__ out, int in_smem, int* status) {
+  pdl_launch_dependents();
+  pdl_wait();
+  extern __shared__ __align__(16) unsigned char sh_raw[];
+  float* zsh = reinterpret_cast<float*>(sh_raw);
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t whist[32][256];  // one digit histogram per warp
+  __shared__ uint32_t s_key[32];
+  __shared__ int s_idx[32];
+  __shared__ float wtot[32];
+  __shared__ uint32_t s_sel[2];
+  __shared__ int s_pick;
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const float* zg = logits + (size_t)b * ldl;
+  const float* z = zg;
+  if (in_smem) {
+    for (int i = tid; i < V; i += kSampleThreads) zsh[i] = zg[i];
+    __syncthreads();
+    z = zsh;
+  }
+  // the largest entry (greedy answer; lowest index among equal maxima)
+  uint32_t bk = 0u;
+  int bi = 0x7fffffff;
+  for (int i = tid; i < V; i += kSampleThreads) {
+    const uint32_t k = fkey(z[i]);
+    if (k > bk || (k == bk && i < bi)) { bk = k; bi = i; }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint32_t k2 = __shfl_xor_sync(0xffffffffu, bk, o);
+    const int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (k2 > bk || (k2 == bk && i2 < bi)) { bk = k2; bi = i2; }
+  }
+  if (lane == 0) { s_key[wid] = bk; s_idx[wid] = bi; }
+  __syncthreads();
+  if (wid == 0) {
+    bk = s_key[lane];
+    bi = s_idx[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint32_t k2 = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (k2 > bk || (k2 == bk && i2 < bi)) { bk = k2; bi = i2; }
+    }
+    if (lane == 0) { s_key[0] = bk; s_idx[0] = bi; }
+  }
+  __syncthreads();
+  const uint32_t kmax = s_key[0];
+  const int imax = s_idx[0];
+  if (!(temperature > 0.f)) {
+    if (tid == 0) out[b] = imax;
+    return;
+  }
+  // top-k threshold: the key of the k-th largest entry (ties counted), found
+  // digit by digit from the most significant byte
+  uint32_t thr = 0u;
+  if (top_k > 0 && top_k < V) {
+    uint32_t prefix = 0u, pmask = 0u, rank = (uint32_t)top_k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 32 * 256; i += kSampleThreads) (&whist[0][0])[i] = 0u;
+      __syncthreads();
+      for (int i0 = 0; i0 < V; i0 += kSampleThreads) {
+        const int i = i0 + tid;
+        const uint32_t k = i < V ? fkey(z[i]) : 0u;
+        const bool in = i < V && (k & pmask) == prefix;
+        if (__any_sync(0xffffffffu, in)) {
+          const uint32_t d = in ? (k >> shift) & 255u : 0xffffffffu;  // lanes out form one group
+          // lanes with the same digit add once, through their leader, into
+          // this warp's own histogram (no contention between warps)
+          const uint32_t peers = __match_any_sync(0xffffffffu, d);
+          if (in && (__ffs(peers) - 1) == lane) whist[wid][d] += (uint32_t)__popc(peers);
+        }
+      }
+      __syncthreads();
+      if (tid < 256) {
+        uint32_t t = 0u;
+#pragma unroll 8
+        for (int w = 0; w < 32; ++w) t += whist[w][tid];
+        hist[tid] = t;
+      }
+      __syncthreads();
+      if (wid == 0) {
+        // lane l owns digits 255 - 8 l down to 248 - 8 l
+        uint32_t cnt[8], tot = 0u;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          cnt[e] = hist[255 - 8 * lane - e];
+          tot += cnt[e];
+        }
+        uint32_t incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += n;
+        }
+        const uint32_t excl = incl - tot;
+        if (excl < rank && rank <= incl) {
+          uint32_t c = excl;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (c + cnt[e] >= rank) {
+              s_sel[0] = (uint32_t)(255 - 8 * lane - e);
+              s_sel[1] = rank - c;
+              break;
+            }
+            c += cnt[e];
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= s_sel[0] << shift;
+      pmask |= 255u << shift;
+      rank = s_sel[1];
+      __syncthreads();
+    }
+    thr = prefix;
+  }
+  // weights w_i = exp((z_i - z_max) / tau) over the kept entries.  Warp w owns
+  // the contiguous indices [w bw, (w + 1) bw) and walks them 32 at a time
+  // (lane l reads index i0 + l: conflict-free); the warp's running sum adds
+  // one butterfly row sum per step, in index order.
+  const float zmax = unkey(kmax);
+  const float itau = 1.0f / temperature;
+  const int nw = kSampleThreads / 32;
+  const int bw = ((V + nw - 1) / nw + 31) & ~31;
+  const int wlo = min(wid * bw, V), whi = min(wlo + bw, V);
+  auto weight = [&](int i) -> float {
+    if (i >= whi) return 0.f;
+    const float zi = z[i];
+    return fkey(zi) >= thr ? expf((zi - zmax) * itau) : 0.f;
+  };
+  float run = 0.f;
+  int lastpos = -1;  // last index of this warp's block with a positive weight
+  for (int i0 = wlo; i0 < whi; i0 += 32) {
+    const float wi = weight(i0 + lane);
+    run += warp_sum(wi);
+    const uint32_t pos = __ballot_sync(0xffffffffu, wi > 0.f);
+    if (pos) lastpos = i0 + 31 - __clz(pos);
+  }
+  if (lane == 0) { wtot[wid] = run; s_idx[wid] = lastpos; }
+  __syncthreads();
+  float u = uniforms[b];
+  if (!(u >= 0.f && u < 1.f)) {
+    if (tid == 0) atomicOr(status, kStatusData);
+    u = fminf(fmaxf(u, 0.f), 0.99999994f);
+  }
+  if (tid == 0) {
+    // warp prefixes in warp order; the draw falls in the first warp (with a
+    // positive sum) whose inclusive prefix exceeds u * total
+    float total = 0.f;
+    for (int w = 0; w < nw; ++w) total += wtot[w];
+    const float target = u * total;
+    float c = 0.f;
+    int pick_w = -1, last_w = -1;
+    for (int w = 0; w < nw; ++w) {
+      if (wtot[w] > 0.f) {
+        last_w = w;
+        if (pick_w < 0 && c + wtot[w] > target) {
+          pick_w = w;
+          s_sel[1] = __float_as_uint(c);  // prefix before the drawing warp
+        }
+      }
+      c += wtot[w];
+    }
+    s_sel[0] = __float_as_uint(target);
+    // none passes (u * total at the very top, by rounding): the last token
+    // with a positive weight
+    s_pick = pick_w >= 0 ? -1 - pick_w : (last_w >= 0 ? s_idx[last_w] : imax);
+  }
+  __syncthreads();
+  if (s_pick < 0 && wid == -1 - s_pick) {
+    const float target = __uint_as_float(s_sel[0]);
+    float c = __uint_as_float(s_sel[1]);
+    int pick = lastpos;
+    for (int i0 = wlo; i0 < whi; i0 += 32) {
+      const float wi = weight(i0 + lane);
+      // inclusive prefix within the row, then the first lane past the target
+      float inc = wi;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += n;
+      }
+      const uint32_t past = __ballot_sync(0xffffffffu, wi > 0.f && c + inc > target);
+      if (past) {
+        pick = i0 + __ffs(past) - 1;
+        break;
+      }
+      c += warp_sum(wi);
+    }
+    if (lane == 0) out[b] = pick;
+  } else if (s_pick >= 0 && tid == 0) {
+    out[b] = s_pick;
+  }
+}
+
+template <typename TW, int NB>
+void launch_last_logits_nb(const float* x, int ldx, int T, int b0, const TW* W, int V, int C, float cap, float eps,
+                           float* out, int ldo, int num_sms, int* status, cudaStream_t st) {
+  const LastGeom g = last_geom(C, (int)sizeof(TW), NB);
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(k_last_logits<TW, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
+    attr = true;
+  }
+  launch_pdl(k_last_logits<TW, NB>, dim3(num_sms), dim3(kLastThreads), g.smem, st, 1, x, ldx, T, b0, W, V, C, cap,
+             eps, out, ldo, g.rows, g.stages, status);
+}
+
+template <typename TW>
+void launch_last_logits_t(const float* x, int ldx, int B, int T, const TW* W, int V, int C, float cap, float eps,
+                          float* out, int ldo, int num_sms, int* status, cudaStream_t st) {
+  for (int b0 = 0; b0 < B; b0 += kLastRows) {
+    const int nb = B - b0 < kLastRows ? B - b0 : kLastRows;
+    LaunchScope scope_(KK_LAST_LOGITS, st);
+    switch (nb) {
+      case 1: launch_last_logits_nb<TW, 1>(x, ldx, T, b0, W, V, C, cap, eps, out, ldo, num_sms, status, st); break;
+      case 2: launch_last_logits_nb<TW, 2>(x, ldx, T, b0, W, V, C, cap, eps, out, ldo, num_sms, status, st); break;
+      case 3: launch_last_logits_nb<TW, 3>(x, ldx, T, b0, W, V, C, cap, eps, out, ldo, num_sms, status, st); break;
+      case 4: launch_last_logits_nb<TW, 4>(x, ldx, T, b0, W, V, C, cap, eps, out, ldo, num_sms, status, st); break;
+      case 5: launch_last_logits_nb<TW, 5>(x, ldx, T, b0, W, V, C, cap, eps, out, ldo, num_sms, status, st); break;
+      case 6: launch_last_logits_nb<TW, 6>(x, ldx, T, b0, W, V, C, cap, eps, out, ldo, num_sms, status, st); break;
+      case 7: launch_last_logits_nb<TW, 7>(x, ldx, T, b0, W, V, C, cap, eps, out, ldo, num_sms, status, st); break;
+      default: launch_last_logits_nb<TW, 8>(x, ldx, T, b0, W, V, C, cap, eps, out, ldo, num_sms, status, st); break;
+    }
+  }
+}
+
+}  // namespace
+
+void launch_last_logits(const float* x, int ldx, int B, int T, const void* W, int V, int C, bool bf, float cap,
+                        float eps, float* out, int ldo, int num_sms, int* status, cudaStream_t st) {
+  if (bf)
+    launch_last_logits_t(x, ldx, B, T, static_cast<const bf16*>(W), V, C, cap, eps, out, ldo, num_sms, status, st);
+  else
+    launch_last_logits_t(x, ldx, B, T, static_cast<const float*>(W), V, C, cap, eps, out, ldo, num_sms, status, st);
+}
+
+int last_logits_max_c() { return kMaxLastC; }
+
+bool sample_in_smem(int V) { return (size_t)V * 4 <= kSampleSmemMax; }
+
+void launch_sample(const float* logits, int B, int V, int ldl, float temperature, int top_k,
+                   const float* uniforms, int32_t* out, int* status, cudaStream_t st) {
+  LaunchScope scope_(KK_SAMPLE, st);
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(k_sample, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSampleSmemMax);
+    attr = true;
+  }
+  const bool sm = sample_in_smem(V);
+  launch_pdl(k_sample, dim3(B), dim3(kSampleThreads), sm ? (size_t)V * 4 : 0, st, 1, logits, V, ldl, temperature,
+             top_k, uniforms, out, sm ? 1 : 0, status);
+}
+
+}  // namespace nc

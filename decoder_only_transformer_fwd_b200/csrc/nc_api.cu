@@ -9,6 +9,7 @@
 // residual add, RMSNorm, FC1 + ReLU^2, FC2 with the residual add; then backout,
 // the final RMSNorm, the head with softcap and the cross-entropy.
 #include <stdio.h>
+#include <cmath>
 #include <string.h>
 
 #include <mutex>
@@ -272,10 +273,17 @@ int nc_params_init(nc_params* p, const nc_config* cfg) {
   return NC_OK;
 }
 
-int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets, int B, int T,
-               float* out_loss, float* out_logits, void* stream) {
+namespace {
+
+// The forward pass over tokens [B, T].  With last_only, the head runs on the
+// last position of each row only and writes its softcapped logits to
+// out_logits [B, V] (no targets, no loss); otherwise it is the full head with
+// per-token cross-entropy.
+int forward_impl(const nc_params* p, const int32_t* tokens, const int32_t* targets, int B, int T,
+                 float* out_loss, float* out_logits, void* stream, bool last_only) {
   t_launches = 0;
-  if (p == nullptr || tokens == nullptr || targets == nullptr || out_loss == nullptr) return NC_ERR_ARG;
+  if (p == nullptr || tokens == nullptr) return NC_ERR_ARG;
+  if (last_only ? out_logits == nullptr : (targets == nullptr || out_loss == nullptr)) return NC_ERR_ARG;
   const nc_config& c = p->cfg;
   if (!config_ok(c)) return NC_ERR_SHAPE;
   if (B <= 0 || T <= 0 || T > c.max_T || (long long)B * T > (long long)p->max_tokens) return NC_ERR_SHAPE;
@@ -290,9 +298,11 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
         (lp.ve && !aligned16(lp.ve)))
       return NC_ERR_ALIGN;
   }
-  if (!aligned16(p->wte) || !aligned16(p->lm_head) || !aligned16(tokens) || !aligned16(targets) ||
-      !aligned16(out_loss) || (out_logits && !aligned16(out_logits)) || !aligned16(p->workspace))
+  if (!aligned16(p->wte) || !aligned16(p->lm_head) || !aligned16(tokens) ||
+      (!last_only && (!aligned16(targets) || !aligned16(out_loss))) || (out_logits && !aligned16(out_logits)) ||
+      !aligned16(p->workspace))
     return NC_ERR_ALIGN;
+  if (last_only && c.n_embd > last_logits_max_c()) return NC_ERR_SHAPE;
   const Layout Lw = layout(c, p->max_tokens);
   if (p->workspace == nullptr || p->workspace_bytes < Lw.total) return NC_ERR_WORKSPACE;
   if (c.dtype == NC_BF16 && c.gemm_impl == 0 && c.vocab_padded % 128 != 0) return NC_ERR_SHAPE;
@@ -434,7 +444,9 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
   }
 
   // final norm, head, softcap, cross-entropy
-  if (tc) {
+  if (last_only) {
+    launch_last_logits(x, C, B, T, p->lm_head, V, C, bf, c.softcap, c.eps, out_logits, V, d.num_sms, d.status, st);
+  } else if (tc) {
     const int bn = gemm_tc_bn(c.vocab_padded);
     const int tiles = 2 * ((c.vocab_padded + bn - 1) / bn);  // two epilogue halves per tile
     EpiParams e = epi(EPI_CE);
@@ -460,7 +472,45 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
     launch_gemm_simt(xn, C, p->lm_head, C, M, c.vocab_padded, C, bf, e, st);
     launch_ce_rows(logits, V, targets, M, V, out_loss, d.status, st);
   }
-  return check_launch("nc_forward");
+  return check_launch(last_only ? "nc_last_logits" : "nc_forward");
+}
+
+}  // namespace
+
+int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets, int B, int T,
+               float* out_loss, float* out_logits, void* stream) {
+  return forward_impl(p, tokens, targets, B, T, out_loss, out_logits, stream, false);
+}
+
+int nc_last_logits(const nc_params* p, const int32_t* tokens, int B, int T, float* out_logits, void* stream) {
+  return forward_impl(p, tokens, nullptr, B, T, nullptr, out_logits, stream, true);
+}
+
+int nc_sample(const float* logits, int B, int V, int ldl, float temperature, int top_k, const float* uniforms,
+              int32_t* out_next, void* stream) {
+  t_launches = 0;
+  if (logits == nullptr || uniforms == nullptr || out_next == nullptr) return NC_ERR_ARG;
+  if (B <= 0 || V <= 0 || ldl < V || top_k < 0 || !(temperature >= 0.f) || !std::isfinite(temperature))
+    return NC_ERR_SHAPE;
+  DevInfo d;
+  if (!dev_info(&d)) return NC_ERR_CUDA;
+  launch_sample(logits, B, V, ldl, temperature, top_k, uniforms, out_next, d.status,
+                static_cast<cudaStream_t>(stream));
+  return check_launch("nc_sample");
+}
+
+int nc_generate_next(const nc_params* p, const int32_t* tokens, int B, int T, float temperature, int top_k,
+                     const float* uniforms, int32_t* out_next, float* out_logits, void* stream) {
+  if (uniforms == nullptr || out_next == nullptr || out_logits == nullptr) return NC_ERR_ARG;
+  if (top_k < 0 || !(temperature >= 0.f) || !std::isfinite(temperature)) return NC_ERR_SHAPE;
+  const int rc = forward_impl(p, tokens, nullptr, B, T, nullptr, out_logits, stream, true);
+  if (rc != NC_OK) return rc;
+  const int V = p->cfg.vocab;
+  DevInfo d;
+  if (!dev_info(&d)) return NC_ERR_CUDA;
+  launch_sample(out_logits, B, V, V, temperature, top_k, uniforms, out_next, d.status,
+                static_cast<cudaStream_t>(stream));
+  return check_launch("nc_generate_next");
 }
 
 int nc_forward_host(const nc_params* p, const int32_t* h_tokens, const int32_t* h_targets, int B,
@@ -603,7 +653,8 @@ int nc_launch_timing_count(void) { return t_timing.n; }
 const char* nc_kernel_name(int kind) {
   static const char* names[KK_COUNT] = {
       "embed_norm_smear", "rmsnorm", "rope_table", "rope_qknorm", "gemm_tcgen05", "gemm_cuda_core",
-      "attention_tcgen05", "attention_cuda_core", "ce_combine", "ce_rows", "loss_mean"};
+      "attention_tcgen05", "attention_cuda_core", "ce_combine", "ce_rows", "loss_mean", "last_logits",
+      "sample"};
   return (kind >= 0 && kind < KK_COUNT) ? names[kind] : "unknown";
 }
 

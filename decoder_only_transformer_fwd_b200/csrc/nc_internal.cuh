@@ -133,6 +133,14 @@ void launch_ce_rows(const float* logits, int ldl, const int32_t* targets, int M,
 void launch_ce_combine(const float* ce_sum, const float* ce_tgt, int n_tiles, float offset,
                        const int32_t* targets, int M, int V, float* loss, int* status, cudaStream_t st);
 void launch_loss_mean(const float* loss, const int32_t* targets, int n, float* out, cudaStream_t st);
+// generation: softcapped logits of the last position of each of B rows
+// (x: the final fp32 residual [B T, ldx]; W: lm_head [V_padded, C], bf16 or
+// fp32), and one token per row drawn from logits [B, ldl]
+void launch_last_logits(const float* x, int ldx, int B, int T, const void* W, int V, int C, bool bf, float cap,
+                        float eps, float* out, int ldo, int num_sms, int* status, cudaStream_t st);
+int last_logits_max_c();
+void launch_sample(const float* logits, int B, int V, int ldl, float temperature, int top_k,
+                   const float* uniforms, int32_t* out, int* status, cudaStream_t st);
 
 // CUDA-core GEMM: C[M, N] = A[M, K] B[N, K]^T, fp32 accumulate
 void launch_gemm_simt(const void* A, int lda, const void* Bm, int ldb, int M, int N, int K,
@@ -165,7 +173,7 @@ bool launch_attn_tc(const bf16* q, const bf16* k, const bf16* v, int ldq, int ld
 // Kernel kinds, for the launch counter and the optional per-launch timing.
 enum KernelKind : int {
   KK_EMBED = 0, KK_RMSNORM, KK_ROPE_TABLE, KK_ROPE_QKNORM, KK_GEMM_TC, KK_GEMM_SIMT, KK_ATTN_TC,
-  KK_ATTN_SIMT, KK_CE_COMBINE, KK_CE_ROWS, KK_LOSS_MEAN, KK_COUNT
+  KK_ATTN_SIMT, KK_CE_COMBINE, KK_CE_ROWS, KK_LOSS_MEAN, KK_LAST_LOGITS, KK_SAMPLE, KK_COUNT
 };
 // Every launcher holds one of these around its kernel launch: it counts the
 // launch (per host thread) and, when the caller enabled timing for this kind,

@@ -61,6 +61,11 @@ _SIGS = {
     "nc_forward_host": (C.c_int, [C.POINTER(nc_params), C.c_void_p, C.c_void_p, C.c_int, C.c_int,
                                   C.c_void_p, C.c_void_p]),
     "nc_loss_mean": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
+    "nc_last_logits": (C.c_int, [C.POINTER(nc_params), C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]),
+    "nc_sample": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_float, C.c_int, C.c_void_p, C.c_void_p,
+                            C.c_void_p]),
+    "nc_generate_next": (C.c_int, [C.POINTER(nc_params), C.c_void_p, C.c_int, C.c_int, C.c_float, C.c_int,
+                                   C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     "nc_attention_workspace_bytes": (C.c_size_t, [C.c_int] * 7),
     "nc_attention": (C.c_int, [C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int, C.c_int,
                                C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_float, C.c_float,
@@ -81,7 +86,7 @@ _SIGS = {
 
 KERNEL_KINDS = ["embed_norm_smear", "rmsnorm", "rope_table", "rope_qknorm", "gemm_tcgen05",
                 "gemm_cuda_core", "attention_tcgen05", "attention_cuda_core", "ce_combine", "ce_rows",
-                "loss_mean"]
+                "loss_mean", "last_logits", "sample"]
 
 
 class LaunchTimer:
@@ -179,6 +184,29 @@ def nc_forward(params: nc_params, tokens, targets, out_loss, out_logits=None, st
     B, T = tokens.shape
     _check(lib().nc_forward(C.byref(params), _ptr(tokens), _ptr(targets), B, T, _ptr(out_loss),
                             _ptr(out_logits), _stream(stream)), "nc_forward")
+
+
+def nc_last_logits(params: nc_params, tokens, out_logits, stream=None):
+    """Softcapped logits [B, V] of the last position of each row of tokens [B, T]."""
+    B, T = tokens.shape
+    _check(lib().nc_last_logits(C.byref(params), _ptr(tokens), B, T, _ptr(out_logits), _stream(stream)),
+           "nc_last_logits")
+
+
+def nc_sample(logits, temperature: float, top_k: int, uniforms, out_next, stream=None):
+    """One token per row of logits [B, V] (device fp32, rows may be strided),
+    drawn with the row's uniform u in [0, 1) (uniforms: device fp32 [B])."""
+    B, V = logits.shape
+    _check(lib().nc_sample(_ptr(logits), B, V, logits.stride(0), float(temperature), int(top_k), _ptr(uniforms),
+                           _ptr(out_next), _stream(stream)), "nc_sample")
+
+
+def nc_generate_next(params: nc_params, tokens, temperature: float, top_k: int, uniforms, out_next, out_logits,
+                     stream=None):
+    B, T = tokens.shape
+    _check(lib().nc_generate_next(C.byref(params), _ptr(tokens), B, T, float(temperature), int(top_k),
+                                  _ptr(uniforms), _ptr(out_next), _ptr(out_logits), _stream(stream)),
+           "nc_generate_next")
 
 
 def nc_forward_host(params: nc_params, tokens: np.ndarray, targets: np.ndarray, out_loss: np.ndarray,
@@ -284,3 +312,12 @@ class NcModel:
                   if want_logits else None)
         nc_forward(self.params, tokens, targets, loss, logits, stream)
         return loss, logits
+
+    def generate_next(self, tokens, uniforms, temperature: float = 1.0, top_k: int = 0, stream=None):
+        """One generation step: (next tokens [B] int32, last-position logits [B, V])."""
+        import torch
+        B = tokens.shape[0]
+        nxt = torch.empty(B, dtype=torch.int32, device=self.device)
+        logits = torch.empty(B, self.cfg.vocab, dtype=torch.float32, device=self.device)
+        nc_generate_next(self.params, tokens, temperature, top_k, uniforms, nxt, logits, stream)
+        return nxt, logits

@@ -29,6 +29,7 @@ SEED_BASE = 20260  # seed of workload i is SEED_BASE + i
 # tensor ids for the per-tensor streams
 _ID_TOKENS, _ID_TARGETS, _ID_WTE, _ID_HEAD, _ID_SMEAR = 1, 2, 3, 4, 5
 _ID_Q, _ID_K, _ID_V = 11, 12, 13
+_ID_UNIFORM, _ID_LOGITS = 21, 22
 _LAYER_BASE = 1000  # layer l uses ids _LAYER_BASE + 16*l + j
 
 
@@ -71,6 +72,27 @@ def tokens(seed: int, B: int, T: int, V: int) -> np.ndarray:
 
 def targets(seed: int, B: int, T: int, V: int) -> np.ndarray:
     return _gen(seed, _ID_TARGETS).integers(0, V, size=(B, T), dtype=np.int64).astype(np.int32)
+
+
+def uniforms(seed: int, B: int) -> np.ndarray:
+    """float32 u_b in [0, 1): the random number each row's sampling step draws."""
+    u = _gen(seed, _ID_UNIFORM).random(size=B, dtype=np.float32)
+    return np.minimum(u, np.float32(0.99999994))
+
+
+def sampling_logits(seed: int, B: int, V: int, cap: float = 15.0, ties: int = 0) -> np.ndarray:
+    """float32 logits in the range of a softcapped head's output: a N(0, 2^2)
+    bulk clipped to [-cap, cap], plus 8 entries per row drawn from [6, 8); with
+    `ties`, that many entries of each row repeat the row's 5th-largest value."""
+    g = _gen(seed, _ID_LOGITS)
+    z = np.clip(g.standard_normal(size=(B, V)) * 2.0, -cap, cap).astype(np.float32)
+    for b in range(B):
+        hot = g.choice(V, size=min(V, 8), replace=False)
+        z[b, hot] = (6.0 + 2.0 * g.random(len(hot))).astype(np.float32)
+        if ties and V > 5:
+            fifth = np.sort(z[b])[::-1][4]
+            z[b, g.choice(V, size=min(ties, V), replace=False)] = fifth
+    return z
 
 
 def params(seed: int, *, n_layer: int, n_embd: int, n_head: int, n_kv_head: int,

@@ -141,6 +141,43 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
 int nc_forward_host(const nc_params* p, const int32_t* h_tokens, const int32_t* h_targets, int B,
                     int T, float* h_out_loss, void* stream);
 
+/* Generation ([Math] §Inference: Generating Text, step 2): the forward pass
+ * over tokens [B, T] (device int32, ids in [0, V)), then the head on the last
+ * position of each row only:
+ *   out_logits [B, V] fp32 (device), out_logits[b] = 15 tanh(z/15) with
+ *   z = RMSNorm(x_L[b, T-1]) W_U^T (in bf16 mode the normalised row is
+ *   rounded to bf16 before the product, as in nc_forward).
+ * Same requirements as nc_forward, plus C <= 4096; no targets, no loss.
+ * Status codes as nc_forward (NC_ERR_ARG for a NULL tokens/out_logits). */
+int nc_last_logits(const nc_params* p, const int32_t* tokens, int B, int T, float* out_logits,
+                   void* stream);
+
+/* One token per row drawn from logits ([Math] §Sampling Controls):
+ *   logits   [B, ldl] fp32 (device), first V entries of each row used
+ *   uniforms [B] fp32 (device), u_b in [0, 1): the row's random number
+ *   out_next [B] int32 (device)
+ * temperature == 0: out_next[b] = argmax_v logits[b, v], the lowest index
+ *   among equal maxima (greedy decoding).
+ * temperature > 0: with top_k > 0 (and < V) the entries below the top_k-th
+ *   largest value (ties counted) are dropped, so ties at that value are all
+ *   kept; top_k == 0 or >= V keeps everything.  Weights
+ *   w_v = exp((z_v - max z) / temperature); out_next[b] is the first v (in
+ *   vocabulary order) whose cumulative weight exceeds u_b * sum_v w_v, i.e. a
+ *   draw from P(v) = w_v / sum w by inversion of u_b.
+ * fp32 throughout; a u_b outside [0, 1) sets NC_ERR_DATA in the status word
+ * and is clamped.  NC_ERR_SHAPE: B <= 0, V <= 0, ldl < V, top_k < 0,
+ * temperature < 0 or not finite.  No workspace; a row of V <= 40960 is staged
+ * in shared memory, longer rows are read from global memory. */
+int nc_sample(const float* logits, int B, int V, int ldl, float temperature, int top_k,
+              const float* uniforms, int32_t* out_next, void* stream);
+
+/* nc_last_logits() then nc_sample() on its logits (ldl = V): one generation
+ * step.  out_logits [B, V] fp32 (device) is required and holds the logits
+ * afterwards. */
+int nc_generate_next(const nc_params* p, const int32_t* tokens, int B, int T, float temperature,
+                     int top_k, const float* uniforms, int32_t* out_next, float* out_logits,
+                     void* stream);
+
 /* Mean of loss[i] over i with targets[i] != -1 ([Math] §Cross-Entropy Loss),
  * written to *out_mean (device fp32); NaN when no target is valid.  n >= 0. */
 int nc_loss_mean(const float* loss, const int32_t* targets, int n, float* out_mean, void* stream);

@@ -292,12 +292,13 @@ def block(cfg: dict, lp: dict, layer: int, x: np.ndarray, tok: np.ndarray, lam: 
 
 
 def forward(cfg: dict, params: dict, tokens: np.ndarray, targets: np.ndarray | None = None,
-            rows=None, want_logits: bool = False):
+            rows=None, want_logits: bool = False, positions=None):
     """Per-token loss (and optionally the softcapped logits) for the given rows.
 
     tokens/targets are [B, T] int arrays; rows are independent sequences, so
-    `rows` selects which ones to evaluate.  Returns (loss [R, T], logits
-    [R, T, V] or None).
+    `rows` selects which ones to evaluate.  `positions` (default: all) limits
+    the head to those positions of each row; the blocks still run over the
+    whole row.  Returns (loss [R, P], logits [R, P, V] or None).
     """
     tokens = np.asarray(tokens)
     B, T = tokens.shape
@@ -319,10 +320,11 @@ def forward(cfg: dict, params: dict, tokens: np.ndarray, targets: np.ndarray | N
                 x_bo = x.copy()
         if x_bo is not None:
             x = x - beta * x_bo
-        z = rmsnorm(x, cfg["eps"]) @ head.T
+        pos = np.arange(T) if positions is None else np.asarray(positions, dtype=np.int64)
+        z = rmsnorm(x[pos], cfg["eps"]) @ head.T
         zh = softcap(z, cfg["softcap"])
         if targets is not None:
-            losses.append(cross_entropy_per_token(zh, np.asarray(targets)[b]))
+            losses.append(cross_entropy_per_token(zh, np.asarray(targets)[b][pos]))
         if want_logits:
             logits.append(zh)
     loss = np.stack(losses) if losses else None

@@ -143,6 +143,35 @@ def test_attention_rejects_bad_arguments():
     assert nc.nc_attention_workspace_bytes(2, 8, 4, 4, 128, "bf16", 0) == 0
 
 
+def test_generation_entry_points_reject_bad_arguments():
+    lib = nc.lib()
+    buf = (C.c_byte * 4096)()
+    a16 = C.c_void_p((C.addressof(buf) + 15) & ~15)
+    ARG, SHAPE = nc.STATUS_CODES["NC_ERR_ARG"], nc.STATUS_CODES["NC_ERR_SHAPE"]
+    # nc_sample(logits, B, V, ldl, temperature, top_k, uniforms, out_next, stream)
+    assert lib.nc_sample(None, 1, 8, 8, 1.0, 0, a16, a16, None) == ARG
+    assert lib.nc_sample(a16, 1, 8, 8, 1.0, 0, None, a16, None) == ARG
+    assert lib.nc_sample(a16, 0, 8, 8, 1.0, 0, a16, a16, None) == SHAPE
+    assert lib.nc_sample(a16, 1, 0, 8, 1.0, 0, a16, a16, None) == SHAPE
+    assert lib.nc_sample(a16, 1, 8, 7, 1.0, 0, a16, a16, None) == SHAPE
+    assert lib.nc_sample(a16, 1, 8, 8, 1.0, -1, a16, a16, None) == SHAPE
+    assert lib.nc_sample(a16, 1, 8, 8, -0.5, 0, a16, a16, None) == SHAPE
+    assert lib.nc_sample(a16, 1, 8, 8, float("inf"), 0, a16, a16, None) == SHAPE
+    assert lib.nc_sample(a16, 1, 8, 8, float("nan"), 0, a16, a16, None) == SHAPE
+    cfg = nc.nc_init_config(1, 256, "fp32", "L", 256)
+    p = nc.nc_params()
+    assert lib.nc_params_init(C.byref(p), C.byref(cfg)) == 0
+    assert lib.nc_last_logits(C.byref(p), a16, 1, 8, None, None) == ARG
+    assert lib.nc_last_logits(C.byref(p), None, 1, 8, a16, None) == ARG
+    assert lib.nc_last_logits(C.byref(p), a16, 1, 8, a16, None) == SHAPE  # max_tokens == 0
+    p.max_tokens = 8
+    assert lib.nc_last_logits(C.byref(p), a16, 1, 8, a16, None) == ARG    # no weights set
+    assert lib.nc_generate_next(C.byref(p), a16, 1, 8, 1.0, 0, None, a16, a16, None) == ARG
+    assert lib.nc_generate_next(C.byref(p), a16, 1, 8, 1.0, 0, a16, a16, None, None) == ARG
+    assert lib.nc_generate_next(C.byref(p), a16, 1, 8, 1.0, -2, a16, a16, a16, None) == SHAPE
+    assert lib.nc_generate_next(C.byref(p), a16, 1, 8, -1.0, 0, a16, a16, a16, None) == SHAPE
+
+
 def test_status_strings():
     lib = nc.lib()
     for code in range(8):
