@@ -361,7 +361,7 @@ def run_ours(args):
     e2e_s = max_over_ranks(time.perf_counter() - t0)
     attn = None if args.no_attention_sweep else attention_sweep(args, dev, stream)
     gen = None
-    if not args.no_generation and not args.layers:
+    if not args.no_generation:
         gen = generation_step(args, model, cfg, tok, B, T, stream, load_peaks()[0])
     clk = clocks.stop()
     rc, bits = nc.nc_get_status(stream)
