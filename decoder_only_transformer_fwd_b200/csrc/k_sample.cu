@@ -17,8 +17,7 @@ namespace nc {
 
 namespace {
 
-constexpr int kLastRows = 8;      // rows of one k_last_logits launch
-constexpr int kMaxLastC = 4096;   // widest model row it stages (8 x 4096 fp32 = 128 KB)
+constexpr int kLastRows = 8;  // rows of one k_last_logits launch
 
 // W_U and the staged rows of x share one element type: bf16 in bf16 mode
 // (x rounded to bf16, as the head GEMM of the full forward rounds it), fp32
@@ -52,14 +51,15 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   return d;
 }
 
-// k_last_logits: warps 0..7 multiply, warp 8 streams W_U into the ring
-constexpr int kLastConsumers = 8;
+// k_last_logits: warps 0..15 multiply (two groups of 8 that take alternate
+// stages), warp 16 streams W_U into the ring
+constexpr int kLastGroupWarps = 8;
+constexpr int kLastConsumers = 2 * kLastGroupWarps;
 constexpr int kLastThreads = 32 * (kLastConsumers + 1);
 constexpr int kLastR = 2;  // vocabulary rows a consumer warp multiplies together
 
-// The ring geometry for rows of `row_bytes`: `rows` vocabulary rows per stage
-// (about 48 KB), `stages` stages, and the shared-memory bytes of the launch
-// (ring, staged x rows, barriers).
+// The ring geometry for rows of `row_bytes`: kLastGroupWarps * kLastR rows
+// per stage, 4 or 2 stages, as fit next to the staged x rows (fp32).
 struct LastGeom {
   int rows, stages;
   size_t stage_bytes, x_bytes, smem;
@@ -67,35 +67,69 @@ struct LastGeom {
 inline LastGeom last_geom(int C, int esz, int nb) {
   LastGeom g;
   const size_t row_bytes = (size_t)C * esz;
-  g.rows = (int)(49152 / row_bytes);
-  g.rows = g.rows < 1 ? 1 : (g.rows > 32 ? 32 : g.rows);
+  g.rows = kLastGroupWarps * kLastR;
   g.stage_bytes = (size_t)g.rows * row_bytes;
-  g.x_bytes = (size_t)nb * row_bytes;
+  g.x_bytes = (size_t)nb * C * 4;
   const size_t budget = 220 * 1024 - g.x_bytes - 1024;
   g.stages = (int)(budget / g.stage_bytes);
-  g.stages = g.stages > 4 ? 4 : g.stages;
+  // an even count, so that every block a stage holds belongs to the same
+  // consumer group: each group then waits on consecutive phases of its stages
+  g.stages = g.stages >= 4 ? 4 : (g.stages >= 2 ? 2 : 0);
   g.smem = g.stages * g.stage_bytes + g.x_bytes + 2 * 4 * 8 + 128;
   return g;
 }
 
+// Sums 2^K values across the warp at once (a transposing butterfly): on
+// return, lane l holds the warp-wide total of value index
+// v(l) = sum_r ((l >> (4 - r)) & 1) << (K - 1 - r), r < K.
+template <int K>
+__device__ __forceinline__ float warp_reduce_many(float (&a)[1 << K], int lane) {
+#pragma unroll
+  for (int r = 0; r < K; ++r) {
+    const int bit = 4 - r, half = 1 << (K - 1 - r);
+    const bool hi = (lane >> bit) & 1;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = hi ? a[i] : a[i + half];
+      const float keep = hi ? a[i + half] : a[i];
+      a[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1 << bit);
+    }
+  }
+  float d = a[0];
+#pragma unroll
+  for (int bit = 4 - K; bit >= 0; --bit) d += __shfl_xor_sync(0xffffffffu, d, 1 << bit);
+  return d;
+}
+
 // logits[b0 + j][v] = cap * tanh(rs_j * (x_j . W_U[v]) / cap) for the NB rows
-// x_j = x[(b0 + j) T + T - 1], rs_j = 1 / sqrt(mean(x_j^2) + eps).  One CTA
-// per SM; CTA c takes the blocks of `rows` consecutive vocabulary rows
-// c, c + G, c + 2G, ...  One thread copies each block (contiguous in W_U)
-// into a ring of shared-memory stages with a bulk copy; the consumer warps
-// multiply two rows at a time against the staged x rows and release the stage.
+// x_j = x[(b0 + j) T + T - 1], rs_j = 1 / sqrt(mean(x_j^2) + eps).  In bf16
+// mode x_j is rounded to bf16 (as the head GEMM of the full forward rounds
+// it) and held as fp32.  One CTA per SM; CTA c takes the blocks of `rows`
+// consecutive vocabulary rows c, c + G, c + 2G, ...  One thread copies each
+// block (contiguous in W_U) into a ring of shared-memory stages with a bulk
+// copy; the two groups of consumer warps take alternate blocks, each warp
+// multiplies two rows against the staged x rows, and the group releases the
+// stage.
 template <typename TW, int NB>
 __global__ void __launch_bounds__(kLastThreads, 1)
 k_last_logits(const float* __restrict__ x, int ldx, int T, int b0, const TW* __restrict__ W, int V, int C,
-              float cap, float eps, float* __restrict__ out, int ldo, int rows, int stages, int* status) {
+              float cap, float eps, float* __restrict__ out, int ldo, int stages, int* status) {
   pdl_launch_dependents();
+  constexpr int kN = Chunk<TW>::kN;  // elements of a 16-byte chunk of W_U
+  constexpr int kH = kN / 4;         // float4s of x per chunk
+  constexpr int kNV = NB <= 4 ? 4 : 8;
+  constexpr int kK = NB <= 4 ? 3 : 4;  // log2(kLastR * kNV)
+  constexpr int rows = kLastGroupWarps * kLastR;
   extern __shared__ __align__(16) unsigned char sh_raw[];
   const size_t row_bytes = (size_t)C * sizeof(TW);
   const size_t stage_bytes = (size_t)rows * row_bytes;
+  const int nchunks = C / kN;
   unsigned char* ring = sh_raw;
-  TW* xs = reinterpret_cast<TW*>(sh_raw + stages * stage_bytes);  // [NB][C]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sh_raw + stages * stage_bytes + NB * row_bytes);
-  __shared__ float red[32];
+  // x as fp32: plane (j, h) holds float4 h of every chunk of row j, so a warp
+  // reading consecutive chunks reads consecutive 16-byte words
+  float4* xq = reinterpret_cast<float4*>(sh_raw + stages * stage_bytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sh_raw + stages * stage_bytes + (size_t)NB * C * 4);
+  __shared__ float red[kLastConsumers];
   __shared__ float rs[NB];
   __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -104,7 +138,7 @@ k_last_logits(const float* __restrict__ x, int ldx, int T, int b0, const TW* __r
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       ptx::mbar_init(full(s), 1);
-      ptx::mbar_init(empty(s), kLastConsumers);
+      ptx::mbar_init(empty(s), kLastGroupWarps);
     }
     abort_flag = 0;
     ptx::fence_mbar_init();
@@ -133,6 +167,7 @@ k_last_logits(const float* __restrict__ x, int ldx, int T, int b0, const TW* __r
     return;
   }
   // consumers: stage the NB rows of x (while the first blocks stream in)
+  float* xf = reinterpret_cast<float*>(xq);
 #pragma unroll 1
   for (int j = 0; j < NB; ++j) {
     const float* xr = x + ((size_t)(b0 + j) * T + (T - 1)) * ldx;
@@ -140,7 +175,8 @@ k_last_logits(const float* __restrict__ x, int ldx, int T, int b0, const TW* __r
     for (int c = threadIdx.x; c < C; c += 32 * kLastConsumers) {
       const float v = xr[c];
       sq += v * v;
-      xs[(size_t)j * C + c] = Chunk<TW>::round(v);
+      const int ci = c / kN, e = c % kN;
+      xf[(((size_t)j * kH + e / 4) * nchunks + ci) * 4 + (e & 3)] = static_cast<float>(Chunk<TW>::round(v));
     }
     sq = warp_sum(sq);
     asm volatile("bar.sync 1, %0;" ::"r"(32 * kLastConsumers));
@@ -153,18 +189,18 @@ k_last_logits(const float* __restrict__ x, int ldx, int T, int b0, const TW* __r
     }
   }
   asm volatile("bar.sync 1, %0;" ::"r"(32 * kLastConsumers));
-  constexpr int kN = Chunk<TW>::kN;
-  const int nchunks = C / kN;
-  const uint4* xs4 = reinterpret_cast<const uint4*>(xs);
-  int k = 0;
-  for (int blk = blockIdx.x; blk < nblk; blk += gridDim.x, ++k) {
+  const int grp = warp / kLastGroupWarps, gw = warp % kLastGroupWarps;
+  const int r = kLastR * gw;  // this warp's rows within a block
+  int k = grp;
+  for (int blk = blockIdx.x + grp * gridDim.x; blk < nblk; blk += 2 * gridDim.x, k += 2) {
     const int s = k % stages;
     if (abort_flag || !ptx::mbar_wait(full(s), (uint32_t)(k / stages) & 1u, status)) { abort_flag = 1; break; }
     const int r0 = blk * rows;
     const int nr = V - r0 < rows ? V - r0 : rows;
-    const uint4* st4 = reinterpret_cast<const uint4*>(ring + s * stage_bytes);
-    for (int r = kLastR * warp; r < nr; r += kLastR * kLastConsumers) {
+    if (r < nr) {
       const bool two = r + 1 < nr;
+      const uint4* w0 = reinterpret_cast<const uint4*>(ring + s * stage_bytes + (size_t)r * row_bytes);
+      const uint4* w1 = reinterpret_cast<const uint4*>(ring + s * stage_bytes + (size_t)(two ? r + 1 : r) * row_bytes);
       float2 acc[kLastR][NB];
 #pragma unroll
       for (int q = 0; q < kLastR; ++q)
@@ -173,28 +209,35 @@ k_last_logits(const float* __restrict__ x, int ldx, int T, int b0, const TW* __r
 #pragma unroll 2
       for (int ci = lane; ci < nchunks; ci += 32) {
         float2 wf[kLastR][kN / 2];
-        Chunk<TW>::unpack(st4[(size_t)r * nchunks + ci], wf[0]);
-        Chunk<TW>::unpack(two ? st4[(size_t)(r + 1) * nchunks + ci] : make_uint4(0u, 0u, 0u, 0u), wf[1]);
+        Chunk<TW>::unpack(w0[ci], wf[0]);
+        Chunk<TW>::unpack(w1[ci], wf[1]);
 #pragma unroll
         for (int j = 0; j < NB; ++j) {
-          float2 xf[kN / 2];
-          Chunk<TW>::unpack(xs4[(size_t)j * nchunks + ci], xf);
 #pragma unroll
-          for (int q = 0; q < kLastR; ++q)
+          for (int h = 0; h < kH; ++h) {
+            const float4 xv = xq[((size_t)j * kH + h) * nchunks + ci];
 #pragma unroll
-            for (int e = 0; e < kN / 2; ++e) acc[q][j] = ffma2(wf[q][e], xf[e], acc[q][j]);
+            for (int q = 0; q < kLastR; ++q) {
+              acc[q][j] = ffma2(wf[q][2 * h], make_float2(xv.x, xv.y), acc[q][j]);
+              acc[q][j] = ffma2(wf[q][2 * h + 1], make_float2(xv.z, xv.w), acc[q][j]);
+            }
+          }
         }
       }
+      // value index q * kNV + j; lane l ends up with the total of one of them
+      float vals[1 << kK];
 #pragma unroll
-      for (int q = 0; q < kLastR; ++q) {
-        float mine = 0.f;
+      for (int q = 0; q < kLastR; ++q)
 #pragma unroll
-        for (int j = 0; j < NB; ++j) {
-          const float sj = warp_sum(acc[q][j].x + acc[q][j].y);
-          if (lane == j) mine = sj;
-        }
-        if (lane < NB && (q == 0 || two)) out[(size_t)(b0 + lane) * ldo + r0 + r + q] = cap * tanhf(mine * rs[lane] / cap);
-      }
+        for (int j = 0; j < kNV; ++j) vals[q * kNV + j] = j < NB ? acc[q][j].x + acc[q][j].y : 0.f;
+      const float tot = warp_reduce_many<kK>(vals, lane);
+      int vi = 0;
+#pragma unroll
+      for (int rr = 0; rr < kK; ++rr) vi |= ((lane >> (4 - rr)) & 1) << (kK - 1 - rr);
+      const int q = vi / kNV, j = vi % kNV;
+      const bool writer = (lane & ((1 << (5 - kK)) - 1)) == 0;
+      if (writer && j < NB && (q == 0 || two))
+        out[(size_t)(b0 + j) * ldo + r0 + r + q] = cap * tanhf(tot * rs[j] / cap);
     }
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(empty(s));
@@ -220,34 +263,37 @@ __device__ __forceinline__ float unkey(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
+// keys of the top digit's bin kept for the lower digits of the radix select
+constexpr int kCand = 4096;
+
 __global__ void __launch_bounds__(kSampleThreads, 1)
 k_sample(const float* __restrict__ logits, int V, int ldl, float temperature, int top_k,
          const float* __restrict__ uniforms, int32_t* __restrict__ out, int in_smem, int* status) {
   pdl_launch_dependents();
   pdl_wait();
   extern __shared__ __align__(16) unsigned char sh_raw[];
-  float* zsh = reinterpret_cast<float*>(sh_raw);
+  uint32_t* cand = reinterpret_cast<uint32_t*>(sh_raw);       // [kCand]
+  float* zsh = reinterpret_cast<float*>(sh_raw + kCand * 4);  // [V] when the row is staged
   __shared__ uint32_t hist[256];
   __shared__ uint32_t whist[32][256];  // one digit histogram per warp
   __shared__ uint32_t s_key[32];
   __shared__ int s_idx[32];
   __shared__ float wtot[32];
   __shared__ uint32_t s_sel[2];
+  __shared__ uint32_t s_ncand;
   __shared__ int s_pick;
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const float* zg = logits + (size_t)b * ldl;
-  const float* z = zg;
-  if (in_smem) {
-    for (int i = tid; i < V; i += kSampleThreads) zsh[i] = zg[i];
-    __syncthreads();
-    z = zsh;
-  }
-  // the largest entry (greedy answer; lowest index among equal maxima)
+  const float* z = in_smem ? zsh : zg;
+  // stage the row and find its largest entry (greedy answer; lowest index
+  // among equal maxima) in one pass
   uint32_t bk = 0u;
   int bi = 0x7fffffff;
   for (int i = tid; i < V; i += kSampleThreads) {
-    const uint32_t k = fkey(z[i]);
+    const float zi = zg[i];
+    if (in_smem) zsh[i] = zi;
+    const uint32_t k = fkey(zi);
     if (k > bk || (k == bk && i < bi)) { bk = k; bi = i; }
   }
 #pragma unroll
@@ -280,14 +326,19 @@ k_sample(const float* __restrict__ logits, int V, int ldl, float temperature, in
   // digit by digit from the most significant byte
   uint32_t thr = 0u;
   if (top_k > 0 && top_k < V) {
-    uint32_t prefix = 0u, pmask = 0u, rank = (uint32_t)top_k;
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    // histogram of digit (key >> shift) & 255 over the keys with
+    // (key & pmask) == prefix, taken from the row or from the candidate list
+    auto count = [&](int shift, uint32_t prefix, uint32_t pmask, bool from_cand, int n) {
       for (int i = tid; i < 32 * 256; i += kSampleThreads) (&whist[0][0])[i] = 0u;
       __syncthreads();
-      for (int i0 = 0; i0 < V; i0 += kSampleThreads) {
+      for (int i0 = 0; i0 < n; i0 += kSampleThreads) {
         const int i = i0 + tid;
-        const uint32_t k = i < V ? fkey(z[i]) : 0u;
-        const bool in = i < V && (k & pmask) == prefix;
+        uint32_t k = 0u;
+        bool in = false;
+        if (i < n) {
+          k = from_cand ? cand[i] : fkey(z[i]);
+          in = (k & pmask) == prefix;
+        }
         if (__any_sync(0xffffffffu, in)) {
           const uint32_t d = in ? (k >> shift) & 255u : 0xffffffffu;  // lanes out form one group
           // lanes with the same digit add once, through their leader, into
@@ -304,6 +355,9 @@ k_sample(const float* __restrict__ logits, int V, int ldl, float temperature, in
         hist[tid] = t;
       }
       __syncthreads();
+    };
+    // the digit whose bin holds the rank-th largest key, and the rank within it
+    auto select = [&](uint32_t rank) {
       if (wid == 0) {
         // lane l owns digits 255 - 8 l down to 248 - 8 l
         uint32_t cnt[8], tot = 0u;
@@ -333,6 +387,36 @@ k_sample(const float* __restrict__ logits, int V, int ldl, float temperature, in
         }
       }
       __syncthreads();
+    };
+    count(24, 0u, 0u, false, V);
+    select((uint32_t)top_k);
+    uint32_t prefix = s_sel[0] << 24, pmask = 0xff000000u, rank = s_sel[1];
+    const uint32_t nbin = hist[s_sel[0]];
+    const bool use_cand = nbin <= (uint32_t)kCand;
+    __syncthreads();
+    if (use_cand) {
+      // compact the keys of the selected bin (warp-aggregated slots)
+      if (tid == 0) s_ncand = 0u;
+      __syncthreads();
+      for (int i0 = 0; i0 < V; i0 += kSampleThreads) {
+        const int i = i0 + tid;
+        const uint32_t k = i < V ? fkey(z[i]) : 0u;
+        const bool in = i < V && (k & pmask) == prefix;
+        const uint32_t m = __ballot_sync(0xffffffffu, in);
+        if (m) {
+          const int leader = __ffs(m) - 1;
+          uint32_t base = 0u;
+          if (lane == leader) base = atomicAdd(&s_ncand, (uint32_t)__popc(m));
+          base = __shfl_sync(0xffffffffu, base, leader);
+          if (in) cand[base + __popc(m & ((1u << lane) - 1u))] = k;
+        }
+      }
+      __syncthreads();
+    }
+    const int n = use_cand ? (int)nbin : V;
+    for (int shift = 16; shift >= 0; shift -= 8) {
+      count(shift, prefix, pmask, use_cand, n);
+      select(rank);
       prefix |= s_sel[0] << shift;
       pmask |= 255u << shift;
       rank = s_sel[1];
@@ -342,26 +426,27 @@ k_sample(const float* __restrict__ logits, int V, int ldl, float temperature, in
   }
   // weights w_i = exp((z_i - z_max) / tau) over the kept entries.  Warp w owns
   // the contiguous indices [w bw, (w + 1) bw) and walks them 32 at a time
-  // (lane l reads index i0 + l: conflict-free); the warp's running sum adds
-  // one butterfly row sum per step, in index order.
+  // (lane l reads index i0 + l: conflict-free); steps with no kept entry cost
+  // one ballot.
   const float zmax = unkey(kmax);
   const float itau = 1.0f / temperature;
   const int nw = kSampleThreads / 32;
   const int bw = ((V + nw - 1) / nw + 31) & ~31;
   const int wlo = min(wid * bw, V), whi = min(wlo + bw, V);
-  auto weight = [&](int i) -> float {
-    if (i >= whi) return 0.f;
-    const float zi = z[i];
-    return fkey(zi) >= thr ? expf((zi - zmax) * itau) : 0.f;
-  };
-  float run = 0.f;
+  float acc = 0.f;
   int lastpos = -1;  // last index of this warp's block with a positive weight
   for (int i0 = wlo; i0 < whi; i0 += 32) {
-    const float wi = weight(i0 + lane);
-    run += warp_sum(wi);
-    const uint32_t pos = __ballot_sync(0xffffffffu, wi > 0.f);
-    if (pos) lastpos = i0 + 31 - __clz(pos);
+    const int i = i0 + lane;
+    const float zi = i < whi ? z[i] : 0.f;
+    const bool kept = i < whi && fkey(zi) >= thr;
+    if (__ballot_sync(0xffffffffu, kept)) {
+      const float wi = kept ? expf((zi - zmax) * itau) : 0.f;
+      acc += wi;
+      const uint32_t pos = __ballot_sync(0xffffffffu, wi > 0.f);
+      if (pos) lastpos = i0 + 31 - __clz(pos);
+    }
   }
+  const float run = warp_sum(acc);
   if (lane == 0) { wtot[wid] = run; s_idx[wid] = lastpos; }
   __syncthreads();
   float u = uniforms[b];
@@ -394,17 +479,23 @@ k_sample(const float* __restrict__ logits, int V, int ldl, float temperature, in
   }
   __syncthreads();
   if (s_pick < 0 && wid == -1 - s_pick) {
+    // walk the drawing warp's block again, step by step, and pick the first
+    // lane whose running prefix passes the target; if rounding leaves none,
+    // the block's last token with a positive weight
     const float target = __uint_as_float(s_sel[0]);
     float c = __uint_as_float(s_sel[1]);
     int pick = lastpos;
     for (int i0 = wlo; i0 < whi; i0 += 32) {
-      const float wi = weight(i0 + lane);
-      // inclusive prefix within the row, then the first lane past the target
+      const int i = i0 + lane;
+      const float zi = i < whi ? z[i] : 0.f;
+      const bool kept = i < whi && fkey(zi) >= thr;
+      if (!__ballot_sync(0xffffffffu, kept)) continue;
+      const float wi = kept ? expf((zi - zmax) * itau) : 0.f;
       float inc = wi;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const float n = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += n;
+        const float nb = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += nb;
       }
       const uint32_t past = __ballot_sync(0xffffffffu, wi > 0.f && c + inc > target);
       if (past) {
@@ -429,7 +520,7 @@ void launch_last_logits_nb(const float* x, int ldx, int T, int b0, const TW* W, 
     attr = true;
   }
   launch_pdl(k_last_logits<TW, NB>, dim3(num_sms), dim3(kLastThreads), g.smem, st, 1, x, ldx, T, b0, W, V, C, cap,
-             eps, out, ldo, g.rows, g.stages, status);
+             eps, out, ldo, g.stages, status);
 }
 
 template <typename TW>
@@ -461,7 +552,10 @@ void launch_last_logits(const float* x, int ldx, int B, int T, const void* W, in
     launch_last_logits_t(x, ldx, B, T, static_cast<const float*>(W), V, C, cap, eps, out, ldo, num_sms, status, st);
 }
 
-int last_logits_max_c() { return kMaxLastC; }
+bool last_logits_supported(int C, bool bf) {
+  // at least two ring stages next to eight staged rows of x
+  return C > 0 && last_geom(C, bf ? 2 : 4, kLastRows).stages >= 2;
+}
 
 bool sample_in_smem(int V) { return (size_t)V * 4 <= kSampleSmemMax; }
 
@@ -470,11 +564,12 @@ void launch_sample(const float* logits, int B, int V, int ldl, float temperature
   LaunchScope scope_(KK_SAMPLE, st);
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(k_sample, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSampleSmemMax);
+    cudaFuncSetAttribute(k_sample, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(kSampleSmemMax + kCand * 4));
     attr = true;
   }
   const bool sm = sample_in_smem(V);
-  launch_pdl(k_sample, dim3(B), dim3(kSampleThreads), sm ? (size_t)V * 4 : 0, st, 1, logits, V, ldl, temperature,
+  launch_pdl(k_sample, dim3(B), dim3(kSampleThreads), (size_t)kCand * 4 + (sm ? (size_t)V * 4 : 0), st, 1, logits, V,
+             ldl, temperature,
              top_k, uniforms, out, sm ? 1 : 0, status);
 }
 

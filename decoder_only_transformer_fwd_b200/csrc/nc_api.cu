@@ -302,7 +302,7 @@ int forward_impl(const nc_params* p, const int32_t* tokens, const int32_t* targe
       (!last_only && (!aligned16(targets) || !aligned16(out_loss))) || (out_logits && !aligned16(out_logits)) ||
       !aligned16(p->workspace))
     return NC_ERR_ALIGN;
-  if (last_only && c.n_embd > last_logits_max_c()) return NC_ERR_SHAPE;
+  if (last_only && !last_logits_supported(c.n_embd, c.dtype == NC_BF16)) return NC_ERR_SHAPE;
   const Layout Lw = layout(c, p->max_tokens);
   if (p->workspace == nullptr || p->workspace_bytes < Lw.total) return NC_ERR_WORKSPACE;
   if (c.dtype == NC_BF16 && c.gemm_impl == 0 && c.vocab_padded % 128 != 0) return NC_ERR_SHAPE;

@@ -138,7 +138,7 @@ void launch_loss_mean(const float* loss, const int32_t* targets, int n, float* o
 // fp32), and one token per row drawn from logits [B, ldl]
 void launch_last_logits(const float* x, int ldx, int B, int T, const void* W, int V, int C, bool bf, float cap,
                         float eps, float* out, int ldo, int num_sms, int* status, cudaStream_t st);
-int last_logits_max_c();
+bool last_logits_supported(int C, bool bf);  // C <= 2304 (bf16) / 1280 (fp32)
 void launch_sample(const float* logits, int B, int V, int ldl, float temperature, int top_k,
                    const float* uniforms, int32_t* out, int* status, cudaStream_t st);
 
