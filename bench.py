@@ -14,7 +14,9 @@ Prints one JSON line (rank 0).  With N > 1 (launched by torch.distributed.run)
 every rank runs an independent replica on its own 4 rows: the rows of a batch
 are independent sequences and the forward pass has no exchange step, so there
 is no data-path collective (weak scaling); the ranks only meet at the timing
-barriers and the max-over-ranks reduction of the elapsed time.
+barriers, the max-over-ranks reduction of the elapsed time and, after the
+timed steps, one all-reduce of (loss sum, valid count) for the mean loss of
+the global batch (reported as mean_loss).
 
 --impl reference times the CPU oracle (fp64 numpy) on the host cores instead:
 each step is a bounded sample of the same workload (the first 256 positions
@@ -259,7 +261,7 @@ def run_ours(args):
     import numpy as np
     import torch
 
-    from decoder_only_transformer_fwd_b200 import flops, nc, synth
+    from decoder_only_transformer_fwd_b200 import flops, nc, replicas, synth
 
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
@@ -286,8 +288,8 @@ def run_ours(args):
                           n_kv_head=cfg.n_kv_head, head_dim=cfg.head_dim, vocab=cfg.vocab,
                           vocab_padded=cfg.vocab_padded, ve_layers=ve_layers, bf16=True)
     # each rank processes its own batch of B rows (rank-dependent tokens)
-    tok_h = synth.tokens(seed + 1000 * rank, B, T, cfg.vocab)
-    tgt_h = synth.targets(seed + 1000 * rank, B, T, cfg.vocab)
+    tok_h = synth.tokens(replicas.rank_seed(seed, rank), B, T, cfg.vocab)
+    tgt_h = synth.targets(replicas.rank_seed(seed, rank), B, T, cfg.vocab)
     model = nc.NcModel(cfg, params, M, device=dev)
     tok = torch.from_numpy(tok_h).to(dev)
     tgt = torch.from_numpy(tgt_h).to(dev)
@@ -301,12 +303,7 @@ def run_ours(args):
         if world > 1:
             torch.distributed.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+    max_over_ranks = replicas.max_over_ranks
 
     for _ in range(args.warmup):
         step()
@@ -368,13 +365,16 @@ def run_ours(args):
     if rc != 0:
         raise RuntimeError(f"device status after the timed steps: {nc.STATUS.get(rc)} bits={bits}")
     assert np.all(np.isfinite(h_loss.numpy()))
+    # mean loss of the global batch: every rank's (sum, count), one all-reduce
+    valid = tgt_h.reshape(-1) >= 0
+    mean_loss = replicas.global_mean_loss(float(h_loss.numpy().astype(np.float64)[valid].sum()), int(valid.sum()))
 
     peaks, peak_src = load_peaks()
     windows = list(cfg.window[:cfg.n_layer])
     f_tok = flops.forward_flops_per_token(cfg.n_layer, cfg.n_embd, cfg.vocab, windows, T)
     ms_step = ms_total / args.steps
     tokens_all = M * world
-    value = tokens_all * args.steps / (ms_total / 1e3)
+    value = replicas.aggregate_throughput(M, world, args.steps, ms_total / 1e3)
     tflops = f_tok * M / (ms_step / 1e3) / 1e12
 
     gemm_flops_step = flops.gemm_flops_per_token(cfg.n_layer, cfg.n_embd, cfg.vocab) * M
@@ -422,12 +422,13 @@ def run_ours(args):
             "data": "synthetic",
             "config": {"workload": workload_desc(cfg, B, T), "global_batch": B * world, "seq_len": T,
                        "tokens_per_step": tokens_all,
-                       "parallelism": f"replicas x{world} (independent rows, no collective)",
+                       "parallelism": f"replicas x{world} (independent rows; no collective on the data path)",
                        "l2": "inputs larger than L2 (1.46 GB bf16 weights + 0.33 GB gathered rows per step)",
                        "seed": seed},
             "tflops": tflops, "pct_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
             "pct_bf16_peak_sustained": 100.0 * tflops / peaks["bf16_tflops_sustained"],
             "flops_per_token": f_tok,
+            "mean_loss": mean_loss,
             "clocks": clk,
             "roofline": roofline,
             "cpu_baseline": cpu,
