@@ -111,13 +111,21 @@ def dist_setup():
     return world, rank, local
 
 
-def workload_desc(cfg, B, T):
-    head = "d24 nanochat GPT forward+CE" if cfg.n_layer == 24 else \
-        f"profiling case: d24 dimensions cut to {cfg.n_layer} blocks, forward+CE"
-    return (f"{head}: depth {cfg.n_layer}, C={cfg.n_embd}, {cfg.n_head}x{cfg.head_dim} "
-            f"heads, MLP {cfg.mlp_hidden} ReLU^2, V={cfg.vocab}, SSSL windows "
-            f"{cfg.window[0]}/{cfg.max_T} (last block full), value embeddings on odd blocks, "
-            f"backout from block {cfg.backout_layer}, softcap {cfg.softcap:g}, B={B}, T={T}")
+def workload_desc(n_layer, C, H, D, V, short_window, max_T, backout_layer, softcap, B, T):
+    """The workload as the bench line names it; both arms describe it from
+    their own configuration (plain numbers)."""
+    head = "d24 nanochat GPT forward+CE" if n_layer == 24 else \
+        f"profiling case: d24 dimensions cut to {n_layer} blocks, forward+CE"
+    return (f"{head}: depth {n_layer}, C={C}, {H}x{D} heads, MLP {4 * C} ReLU^2, V={V}, SSSL windows "
+            f"{short_window}/{max_T} (last block full), value embeddings on odd blocks, "
+            f"backout from block {backout_layer}, softcap {softcap:g}, B={B}, T={T}")
+
+
+def workload_config(desc, B, T, world, seed):
+    return {"workload": desc, "global_batch": B * world, "seq_len": T, "tokens_per_step": B * T * world,
+            "parallelism": f"replicas x{world} (independent rows; no collective on the data path)",
+            "l2": "inputs larger than L2 (1.46 GB bf16 weights + 0.33 GB gathered rows per step)",
+            "seed": seed}
 
 
 def cpu_oracle_run(cfg_o, params, tok, tgt, ntok):
@@ -161,8 +169,10 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": "d24 nanochat GPT forward+CE (CPU oracle, bounded sample)",
-                   "tokens_per_step": CPU_SAMPLE_TOKENS, "seq_len": w["T"]},
+        "config": workload_config(
+            workload_desc(ocfg["n_layer"], ocfg["n_embd"], ocfg["n_head"], ocfg["head_dim"], ocfg["vocab"],
+                          ocfg["windows"][0], w["T"], ocfg["backout_layer"], ocfg["softcap"], w["B"], w["T"]),
+            w["B"], w["T"], world, seed),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -420,11 +430,10 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": {"workload": workload_desc(cfg, B, T), "global_batch": B * world, "seq_len": T,
-                       "tokens_per_step": tokens_all,
-                       "parallelism": f"replicas x{world} (independent rows; no collective on the data path)",
-                       "l2": "inputs larger than L2 (1.46 GB bf16 weights + 0.33 GB gathered rows per step)",
-                       "seed": seed},
+            "config": workload_config(
+                workload_desc(cfg.n_layer, cfg.n_embd, cfg.n_head, cfg.head_dim, cfg.vocab, cfg.window[0],
+                              cfg.max_T, cfg.backout_layer, cfg.softcap, B, T),
+                B, T, world, seed),
             "tflops": tflops, "pct_bf16_peak": 100.0 * tflops / peaks["bf16_tflops"],
             "pct_bf16_peak_sustained": 100.0 * tflops / peaks["bf16_tflops_sustained"],
             "flops_per_token": f_tok,
