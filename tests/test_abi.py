@@ -99,6 +99,10 @@ def test_forward_rejects_bad_arguments_without_launching():
     assert lib.nc_forward(C.byref(p), None, a16, 1, 8, a16, None, None) == nc.STATUS_CODES["NC_ERR_ARG"]
     # shape beyond capacity (max_tokens == 0)
     assert lib.nc_forward(C.byref(p), a16, a16, 1, 8, a16, None, None) == nc.STATUS_CODES["NC_ERR_SHAPE"]
+    # empty batches
+    for B, T in ((0, 8), (1, 0), (-1, 8)):
+        assert lib.nc_forward(C.byref(p), a16, a16, B, T, a16, None, None) == nc.STATUS_CODES["NC_ERR_SHAPE"]
+        assert lib.nc_last_logits(C.byref(p), a16, B, T, a16, None) == nc.STATUS_CODES["NC_ERR_SHAPE"]
     p.max_tokens = 8
     assert lib.nc_forward(C.byref(p), a16, a16, 1, 300, a16, None, None) == nc.STATUS_CODES["NC_ERR_SHAPE"]
     # missing parameters
