@@ -6,7 +6,9 @@
  * nanochat" (§High-Level Forward Pass and the sections it links), extended by
  * the smear gate and backout of the "nanochat depth sweep" model card
  * (Architecture list) and "Reading nanochat Source" (§5, Forward pass, shape
- * by shape).
+ * by shape).  The generation step of the same page (§Inference: Generating
+ * Text, §Sampling Controls) runs on it: the logits of the last position only,
+ * then a greedy or top-k / temperature draw.
  *
  * Conventions for every call:
  *  - Pointers are DEVICE pointers unless the argument says "host".
@@ -42,7 +44,8 @@ typedef enum {
   NC_ERR_SHAPE = 2,      /* unsupported or inconsistent sizes                */
   NC_ERR_ALIGN = 3,      /* pointer or stride not 16-byte aligned            */
   NC_ERR_CUDA = 4,       /* a CUDA runtime call failed (see nc_last_error)   */
-  NC_ERR_DATA = 5,       /* device-side: token/target id out of range        */
+  NC_ERR_DATA = 5,       /* device-side: token/target id out of range, or a
+                            sampling uniform outside [0, 1)                   */
   NC_ERR_TIMEOUT = 6,    /* device-side: a bounded wait inside a kernel ran out */
   NC_ERR_WORKSPACE = 7   /* workspace missing or smaller than required       */
 } nc_status;
