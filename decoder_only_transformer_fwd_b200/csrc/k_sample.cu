@@ -19,9 +19,10 @@ namespace {
 
 constexpr int kLastRows = 8;  // rows of one k_last_logits launch
 
-// W_U and the staged rows of x share one element type: bf16 in bf16 mode
-// (x rounded to bf16, as the head GEMM of the full forward rounds it), fp32
-// otherwise.  A 16-byte chunk holds 8 or 4 of them, unpacked to fp32 pairs.
+// W_U's element type: bf16 in bf16 mode, fp32 otherwise.  A 16-byte chunk
+// holds 8 or 4 elements, unpacked to fp32 pairs.  round() gives the value an
+// x element takes in the product: rounded to bf16 in bf16 mode, as the head
+// GEMM of the full forward rounds it (the staged copy is held as fp32).
 template <typename TW> struct Chunk;
 template <> struct Chunk<bf16> {
   static constexpr int kN = 8;
@@ -557,7 +558,7 @@ bool last_logits_supported(int C, bool bf) {
   return C > 0 && last_geom(C, bf ? 2 : 4, kLastRows).stages >= 2;
 }
 
-bool sample_in_smem(int V) { return (size_t)V * 4 <= kSampleSmemMax; }
+static bool sample_in_smem(int V) { return (size_t)V * 4 <= kSampleSmemMax; }
 
 void launch_sample(const float* logits, int B, int V, int ldl, float temperature, int top_k,
                    const float* uniforms, int32_t* out, int* status, cudaStream_t st) {
