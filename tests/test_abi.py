@@ -176,6 +176,29 @@ def test_generation_entry_points_reject_bad_arguments():
     assert lib.nc_generate_next(C.byref(p), a16, 1, 8, -1.0, 0, a16, a16, a16, None) == SHAPE
 
 
+@pytest.mark.parametrize("dtype,C_ok,C_bad", [("bf16", 2304, 2432), ("fp32", 1280, 1408)])
+def test_last_logits_width_limit(dtype, C_ok, C_bad):
+    """The last-position head stages eight rows of x next to two stages of 16
+    W_U rows in 220 KB of shared memory: C <= 2304 in bf16, <= 1280 in fp32.
+    Past the limit the call is rejected before any launch; at the limit it
+    gets as far as the (missing) workspace."""
+    lib = nc.lib()
+    buf = (C.c_byte * 4096)()
+    a16 = C.c_void_p((C.addressof(buf) + 15) & ~15)
+    for width, want in ((C_bad, "NC_ERR_SHAPE"), (C_ok, "NC_ERR_WORKSPACE")):
+        cfg = nc.nc_init_config(1, 256, dtype, "L", 256)
+        cfg.n_embd, cfg.n_head, cfg.n_kv_head = width, width // 128, width // 128
+        cfg.mlp_hidden = 4 * width
+        p = nc.nc_params()
+        assert lib.nc_params_init(C.byref(p), C.byref(cfg)) == 0
+        p.max_tokens = 8
+        for name in ("wte", "lm_head", "smear_gate", "resid_lambdas", "x0_lambdas"):
+            setattr(p, name, a16.value)
+        L = p.layer[0]
+        L.w_qkv = L.w_o = L.w_fc1 = L.w_fc2 = L.ve = L.ve_gate = a16.value
+        assert lib.nc_last_logits(C.byref(p), a16, 1, 8, a16, None) == nc.STATUS_CODES[want], (width, want)
+
+
 def test_status_strings():
     lib = nc.lib()
     for code in range(8):
