@@ -183,9 +183,11 @@ def run_reference(args):
 
 def attention_sweep(args, dev, stream):
     """The single attention layer sweep (RoPE + QK-norm, then causal sliding-window
-    attention; B = 8, H = 12, D = 128): per case the attention kernel's own
-    device time (launch events, averaged over `steps` calls) and its
-    algorithmic TFLOP/s, plus the whole nc_attention call."""
+    attention; B = 8, H = 12, D = 128) on the seeded inputs of the parity tests:
+    per case the attention kernel's own device time (launch events, averaged
+    over `steps` calls) and its algorithmic TFLOP/s, the RoPE + QK-norm
+    kernel's time and GB/s (q and k read and written once, bf16, plus the
+    cos/sin rows), and the whole nc_attention call."""
     import torch
 
     from decoder_only_transformer_fwd_b200 import flops, nc, synth
@@ -194,15 +196,15 @@ def attention_sweep(args, dev, stream):
     B, H, D = s["B"], s["H"], s["D"]
     out = []
     for T, window in s["cases"]:
-        g = torch.Generator(device=dev).manual_seed(synth.SEED_BASE + s["index"])
-        q, k, v = (torch.randn(B, T, H, D, device=dev, generator=g).to(torch.bfloat16) for _ in range(3))
+        q, k, v = (torch.from_numpy(a).to(dev).to(torch.bfloat16)
+                   for a in synth.attention_inputs(synth.SEED_BASE + s["index"], B, T, H, D))
         o = torch.empty_like(q)
         ws = torch.empty(nc.nc_attention_workspace_bytes(B, T, H, H, D, "bf16", 1), dtype=torch.uint8,
                          device=dev)
         call = lambda: nc.nc_attention(q, k, v, o, window, 1, 1.15, D ** -0.5, 100000.0, 1e-6, ws, stream)
         for _ in range(3):
             call()
-        timer = nc.LaunchTimer(args.steps, kinds=["attention_tcgen05"])
+        timer = nc.LaunchTimer(2 * args.steps, kinds=["attention_tcgen05", "rope_qknorm"])
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         e0.record(stream)
@@ -211,14 +213,90 @@ def attention_sweep(args, dev, stream):
                 call()
         e1.record(stream)
         torch.cuda.synchronize()
-        n, kms = timer.per_kind().get("attention_tcgen05", (0, 0.0))
+        pk = timer.per_kind()
+        n, kms = pk.get("attention_tcgen05", (0, 0.0))
+        nr, rms_ = pk.get("rope_qknorm", (0, 0.0))
         f = flops.attention_layer_flops(B, T, H, D, window)
         us = 1e3 * kms / max(n, 1)
         tf = f / (us * 1e-6) / 1e12
+        rope_us = 1e3 * rms_ / max(nr, 1)
+        rope_bytes = 2 * (2 * B * T * H * D * 2) + 2 * T * (D // 2) * 4
+        rope_gbs = rope_bytes / (rope_us * 1e-6) / 1e9 if rope_us > 0 else None
         out.append({"T": T, "window": window if window > 0 else "full", "kernel_us": us,
                     "call_us": 1e3 * e0.elapsed_time(e1) / args.steps, "gflop": f / 1e9, "tflops": tf,
-                    "pct_bf16_peak": 100.0 * tf / peaks["bf16_tflops"]})
+                    "pct_bf16_peak": 100.0 * tf / peaks["bf16_tflops"],
+                    "rope_qknorm": {"us": rope_us, "bytes": rope_bytes, "achieved_gbs": rope_gbs,
+                                    "frac": rope_gbs / peaks["hbm_gbs"] if rope_gbs else None}})
         del q, k, v, o, ws
+    return out
+
+
+def head_backward_step(args, model, cfg, tok, tgt, M, stream, peaks):
+    """The head backward (nc_head_backward) after a forward at the bench
+    workload's sizes: device time per call and the TFLOP/s of its three head
+    GEMMs (logits recomputed, dL/dxn, dL/dW_U: 3 x 2 M V C FLOPs)."""
+    import torch
+
+    from decoder_only_transformer_fwd_b200 import nc
+    loss = torch.empty(M, dtype=torch.float32, device=tok.device)
+    dx = torch.empty(M, cfg.n_embd, dtype=torch.float32, device=tok.device)
+    dw = torch.empty(cfg.vocab, cfg.n_embd, dtype=torch.float32, device=tok.device)
+    ws = torch.empty(nc.nc_head_backward_workspace_bytes(cfg, M), dtype=torch.uint8, device=tok.device)
+    nc.nc_forward(model.params, tok, tgt, loss, None, stream)
+    for _ in range(3):
+        nc.nc_head_backward(model.params, tgt, dx, dw, ws, stream)
+    torch.cuda.synchronize()
+    timer = nc.LaunchTimer(8 * args.steps, kinds=["gemm_tcgen05_bwd", "head_bwd_rows"])
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    with timer:
+        for _ in range(args.steps):
+            nc.nc_head_backward(model.params, tgt, dx, dw, ws, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    pk = timer.per_kind()
+    ng, gms = pk.get("gemm_tcgen05_bwd", (0, 0.0))
+    gemm_flops = 3 * 2.0 * M * cfg.vocab_padded * cfg.n_embd
+    tf = gemm_flops * args.steps / (gms / 1e3) / 1e12 if gms > 0 else None
+    return {"workload": f"head backward after the forward: dL/dx [{M}, {cfg.n_embd}] and dL/dW_U "
+                        f"[{cfg.vocab}, {cfg.n_embd}] of the mean CE, B*T = {M}",
+            "ms_per_call": e0.elapsed_time(e1) / args.steps, "gemm_ms_per_call": gms / args.steps,
+            "gemm_tflops": tf, "gemm_frac_of_burst": tf / peaks["bf16_tflops"] if tf else None,
+            "launches_per_call": nc.nc_last_launch_count()}
+
+
+def routing_sweep(args, dev, stream, peaks):
+    """The pass-2 routing attention (nc_routing_attention; 256-wide QK, 128-wide
+    PV) at B = 8, H = 12, T = 2048, window 1024 and full: kernel time and
+    algorithmic TFLOP/s (6 B T H D meankeys)."""
+    import torch
+
+    from decoder_only_transformer_fwd_b200 import flops, nc, synth
+    s = synth.ATTN_SWEEP
+    B, H, D = s["B"], s["H"], s["D"]
+    out = []
+    for T, window in [(2048, 1024), (2048, 0)]:
+        t = [torch.from_numpy(a).to(dev).to(torch.bfloat16)
+             for seed in (synth.SEED_BASE + s["index"], synth.SEED_BASE + s["index"] + 1)
+             for a in synth.attention_inputs(seed, B, T, H, D)]
+        q2, k2, v2, q1, k1 = t[0], t[1], t[2], t[3], t[4]
+        o = torch.empty_like(q2)
+        call = lambda: nc.nc_routing_attention(q2, k2, v2, q1, k1, o, window, 0.5, stream=stream)
+        for _ in range(3):
+            call()
+        timer = nc.LaunchTimer(2 * args.steps, kinds=["attention_tcgen05"])
+        torch.cuda.synchronize()
+        with timer:
+            for _ in range(args.steps):
+                call()
+        torch.cuda.synchronize()
+        n, kms = timer.per_kind().get("attention_tcgen05", (0, 0.0))
+        us = 1e3 * kms / max(n, 1)
+        f = 1.5 * flops.attention_layer_flops(B, T, H, D, window)
+        tf = f / (us * 1e-6) / 1e12
+        out.append({"T": T, "window": window if window > 0 else "full", "kernel_us": us, "gflop": f / 1e9,
+                    "tflops": tf, "pct_bf16_peak": 100.0 * tf / peaks["bf16_tflops"]})
+        del t, q2, k2, v2, q1, k1, o
     return out
 
 
@@ -370,6 +448,10 @@ def run_ours(args):
     gen = None
     if not args.no_generation:
         gen = generation_step(args, model, cfg, tok, B, T, stream, load_peaks()[0])
+    bwd = route = None
+    if not args.no_variants:
+        bwd = head_backward_step(args, model, cfg, tok, tgt, M, stream, load_peaks()[0])
+        route = routing_sweep(args, dev, stream, load_peaks()[0])
     clk = clocks.stop()
     rc, bits = nc.nc_get_status(stream)
     if rc != 0:
@@ -392,9 +474,10 @@ def run_ours(args):
     achieved = (gemm_flops_step * args.steps) / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else None
     roofline = {
         "kernel": "gemm_tcgen05 (k_gemm_tc: QKV, O, FC1, FC2, head+CE)",
-        "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
-        "peak_kind": f"bf16 dense, sustained ({peak_src})", "unit": "TFLOP/s",
-        "frac": (achieved / peaks["bf16_tflops_sustained"]) if achieved else None,
+        "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+        "peak_kind": f"bf16 dense, burst ({peak_src}): the step is milliseconds long", "unit": "TFLOP/s",
+        "frac": (achieved / peaks["bf16_tflops"]) if achieved else None,
+        "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]) if achieved else None,
         "traffic": GEMM_DRAM_BYTES_PER_LAUNCH,
         "traffic_note": "cold-cache DRAM bytes (read + write) per GEMM launch, ncu capture of each GEMM "
                         "mode at d24 sizes weighted by the step's launch mix (12 QKV + 12 QKV-with-VE, "
@@ -408,9 +491,17 @@ def run_ours(args):
     n_emb, ms_emb = per_kind.get("embed_norm_smear", (0, 0.0))
     emb_bytes = M * cfg.n_embd * (2 + 4 + 4 + 2)
     emb_gbs = emb_bytes / (ms_emb / max(n_emb, 1) / 1e3) / 1e9 if ms_emb > 0 else None
-    embed_roofline = {"kernel": "k_embed", "bound": "hbm", "achieved": emb_gbs, "peak": peaks["hbm_gbs"],
+    embed_roofline = {"kernel": "k_embed_vec", "bound": "hbm", "achieved": emb_gbs, "peak": peaks["hbm_gbs"],
                       "unit": "GB/s", "frac": emb_gbs / peaks["hbm_gbs"] if emb_gbs else None,
                       "bytes_per_launch": emb_bytes}
+    # the CE combine reads one partial sum per (row, 128-column tile half) and
+    # the target logit, and writes the loss and the log-sum-exp of each row
+    n_ce, ms_ce = per_kind.get("ce_combine", (0, 0.0))
+    ce_bytes = M * (2 * ((cfg.vocab_padded + 127) // 128) * 4 + 4 + 4 + 4 + 4)
+    ce_gbs = ce_bytes / (ms_ce / max(n_ce, 1) / 1e3) / 1e9 if ms_ce > 0 else None
+    ce_roofline = {"kernel": "k_ce_combine", "bound": "hbm", "achieved": ce_gbs, "peak": peaks["hbm_gbs"],
+                   "unit": "GB/s", "frac": ce_gbs / peaks["hbm_gbs"] if ce_gbs else None,
+                   "bytes_per_launch": ce_bytes, "us": 1e3 * ms_ce / max(n_ce, 1)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -449,8 +540,11 @@ def run_ours(args):
             # pipeline fill/drain between kernels and the timing events themselves
             "gap_ms_per_step": ms_step_b - sum(v[1] for v in per_kind.values()) / args.steps,
             "embed_roofline": embed_roofline,
+            "ce_combine_roofline": ce_roofline,
             "attention_sweep": attn,
             "generation": gen,
+            "head_backward": bwd,
+            "routing_attention": route,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -469,6 +563,8 @@ def main():
     ap.add_argument("--rows", type=int, default=0, help="rows per step (default: the workload's B = 4)")
     ap.add_argument("--no-attention-sweep", action="store_true")
     ap.add_argument("--no-generation", action="store_true", help="skip the generation-step measurement")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the head-backward and routing-attention measurements")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling only: keep the first N blocks of the d24 stack (1..24)")
     args = ap.parse_args()

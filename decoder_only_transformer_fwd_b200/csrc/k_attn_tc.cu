@@ -34,7 +34,7 @@
 // are counted over the CTA's whole sequence.  Every wait is bounded; on a
 // timeout the CTA records NC_ERR_TIMEOUT and returns after its copies and
 // MMAs have landed.
-#include <mutex>
+#include <stdlib.h>
 
 #include "nc_internal.cuh"
 #include "ptx.cuh"
@@ -86,7 +86,10 @@ struct Item {
 __device__ __forceinline__ int first_key_tile(const AttnArgs& a, int q0) { return max(0, q0 - a.window + 1) / kK; }
 __device__ __forceinline__ int last_key_tile(const AttnArgs& a, int q0) { return min(q0 + kQ - 1, a.T - 1) / kK; }
 
-// item i: query-tile pair n_pairs - 1 - i / (B H) (heaviest first), head-batch i % (B H)
+// item i: query-tile pair n_pairs - 1 - i / (B H) (heaviest first), head-batch i % (B H).
+// With ROUTE an item is a single query tile (tile A only): its two Q halves
+// take both Q buffers.
+template <bool ROUTE>
 __device__ __forceinline__ Item decode_item(const AttnArgs& a, int i) {
   Item it;
   const int bh = a.B * a.H;
@@ -94,8 +97,8 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, int i) {
   const int r = i % bh;
   it.b = r / a.H;
   it.h = r % a.H;
-  it.q0 = 2 * p * kQ;
-  it.has_b = (2 * p + 1) < a.n_qblocks;
+  it.q0 = (ROUTE ? 1 : 2) * p * kQ;
+  it.has_b = !ROUTE && (2 * p + 1) < a.n_qblocks;
   it.lo0 = first_key_tile(a, it.q0);
   it.hi0 = last_key_tile(a, it.q0);
   it.lo1 = first_key_tile(a, it.q0 + kQ);
@@ -120,24 +123,31 @@ __device__ __forceinline__ bool active(const Item& it, int g, int t) {
 
 using ptx::ex2;
 
-// Packed fp32 pairs (the f32x2 forms of add / fma on this architecture).
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-  return d;
-}
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
+// Packed fp32 pairs (the f32x2 add / fma of this architecture).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+// 2^e on the FMA and integer pipes, for a share of the exponentials, so that
+// the special-function unit (16 results per clock per SM, the same rate at
+// which the tensor core consumes them at D = 128) is not the bound.  Range
+// reduction e = n + f with n = rint(e), f in [-0.5, 0.5]: adding 1.5 * 2^23
+// leaves n in the low mantissa bits of t; 2^f by a cubic fitted to minimise
+// the relative error on [-0.5, 0.5] (max 7.5e-5, far below the bf16 step
+// 2^-8 that p is rounded to); n is added to the exponent field.  e is
+// clamped at -125 so that the result stays a normal number (2^-125 for masked
+// entries, which no output can see next to the row's maximum term 2^0..2^8).
+__device__ __forceinline__ float2 exp2_poly(float2 e) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  e.x = fmaxf(e.x, -125.0f);
+  e.y = fmaxf(e.y, -125.0f);
+  const float2 t = __fadd2_rn(e, make_float2(kShift, kShift));
+  const float2 n = __fadd2_rn(t, make_float2(-kShift, -kShift));
+  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), e);
+  float2 q = __ffma2_rn(make_float2(0.05517132f, 0.05517132f), f, make_float2(0.24261054f, 0.24261054f));
+  q = __ffma2_rn(q, f, make_float2(0.69326099f, 0.69326099f));
+  q = __ffma2_rn(q, f, make_float2(0.99992811f, 0.99992811f));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
@@ -150,9 +160,18 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// ROUTE: the pass-2 attention of the looped model ("looped-nanochat-d24"
+// card, routing loop): the logits gain a prior g q1 . k1 from the pass-1
+// features, computed as one QK^T over the augmented width 256, [q2 | g q1] .
+// [k2 | k1] (the card's own construction).  Q2 and the pre-scaled Q1 fill the
+// two Q buffers (so an item is one query tile), and each key tile takes three
+// ring slots: K2, K1, V.
+template <int POLY, bool ROUTE>
 __global__ void __launch_bounds__(kThreads, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-              const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ1,
+              const __grid_constant__ CUtensorMap tmK1, const AttnArgs a) {
+  constexpr int PER_TILE = ROUTE ? 3 : 2;  // ring slots per key tile
   pdl_launch_dependents();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -188,6 +207,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::prefetch_tmap(&tmQ);
     ptx::prefetch_tmap(&tmK);
     ptx::prefetch_tmap(&tmV);
+    if (ROUTE) {
+      ptx::prefetch_tmap(&tmQ1);
+      ptx::prefetch_tmap(&tmK1);
+    }
   }
   if (warp == kWarpMma) {
     ptx::tmem_alloc(ptx::smem_u32(tmem_slot), TMEM_COLS);
@@ -210,17 +233,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool qissued = false, ok = true;
       int sc = 0, it = 0;
       for (int item = item_of(0); ok && item < a.n_items; ++it, item = item_of(it)) {
-        const Item w = decode_item(a, item);
+        const Item w = decode_item<ROUTE>(a, item);
         const int row_base = w.b * a.T;
         const int qcol = w.h * kD, kcol = (w.h / (a.H / a.Hkv)) * kD;
-        // K_t then V_t into the next ring slots
+        // K_t (ROUTE: K2_t, K1_t) then V_t into the next ring slots
         auto load_kv = [&](int t) -> bool {
           const int krow = row_base + t * kK;
-          for (int kv = 0; kv < 2; ++kv, ++sc) {
+          for (int kv = 0; kv < PER_TILE; ++kv, ++sc) {
             const int s = sc % SLOTS;
             const uint32_t ph = (uint32_t)(sc / SLOTS) & 1u;
             if (*abort_flag || !ptx::mbar_wait(bar(B_SLE + s), ph ^ 1, a.status)) return false;
-            const void* tm = kv == 0 ? (const void*)&tmK : (const void*)&tmV;
+            const void* tm = kv == 0 ? (const void*)&tmK
+                                     : (kv == PER_TILE - 1 ? (const void*)&tmV : (const void*)&tmK1);
             ptx::mbar_arrive_expect_tx(bar(B_SLF + s), TILE_BYTES);
             ptx::tma_load_2d(sSlot(s), tm, bar(B_SLF + s), kcol, krow);
             ptx::tma_load_2d(sSlot(s) + BOX_BYTES, tm, bar(B_SLF + s), kcol + 64, krow);
@@ -233,10 +257,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!load_kv(w.lo)) { ok = false; break; }
         // the previous item's QK MMAs have finished reading the Q buffers
         if (*abort_flag || !ptx::mbar_wait(bar(B_QE), (it & 1) ^ 1, a.status)) { ok = false; break; }
-        ptx::mbar_arrive_expect_tx(bar(B_QF), (w.has_b ? 2 : 1) * TILE_BYTES);
-        for (int g = 0; g < (w.has_b ? 2 : 1); ++g) {
-          ptx::tma_load_2d(sQ(g), &tmQ, bar(B_QF), qcol, row_base + w.q0 + g * kQ);
-          ptx::tma_load_2d(sQ(g) + BOX_BYTES, &tmQ, bar(B_QF), qcol + 64, row_base + w.q0 + g * kQ);
+        ptx::mbar_arrive_expect_tx(bar(B_QF), (ROUTE || w.has_b ? 2 : 1) * TILE_BYTES);
+        if (ROUTE) {
+          // Q2 into the first buffer, the pre-scaled Q1 into the second
+          for (int g = 0; g < 2; ++g) {
+            const void* tq = g == 0 ? (const void*)&tmQ : (const void*)&tmQ1;
+            ptx::tma_load_2d(sQ(g), tq, bar(B_QF), qcol, row_base + w.q0);
+            ptx::tma_load_2d(sQ(g) + BOX_BYTES, tq, bar(B_QF), qcol + 64, row_base + w.q0);
+          }
+        } else {
+          for (int g = 0; g < (w.has_b ? 2 : 1); ++g) {
+            ptx::tma_load_2d(sQ(g), &tmQ, bar(B_QF), qcol, row_base + w.q0 + g * kQ);
+            ptx::tma_load_2d(sQ(g) + BOX_BYTES, &tmQ, bar(B_QF), qcol + 64, row_base + w.q0 + g * kQ);
+          }
         }
         qissued = true;
         qpar = it & 1;
@@ -264,13 +297,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dq0 = ptx::desc_kmajor_sw128(sQ(0)), dq1 = ptx::desc_kmajor_sw128(sQ(1));
       const uint64_t dk0 = ptx::desc_kmajor_sw128(sSlot(0)), dv0 = ptx::desc_mnmajor_sw128(sSlot(0), BOX_BYTES);
       auto slot_off = [&](int sc) { return (uint64_t)((sc % SLOTS) * (TILE_BYTES >> 4)); };
+      // S_g = Q_g K^T; with ROUTE (group 0 only) S = Q2 K2^T + (g Q1) K1^T, the
+      // second half of the 256-wide contraction continuing the same accumulation
       auto qk = [&](int g, int sc) {
         const uint32_t tS = tmem + (uint32_t)(g * 128);
-        const uint64_t dq = g == 0 ? dq0 : dq1, dk = dk0 + slot_off(sc);
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint64_t off = (uint64_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
-          ptx::mma_bf16_ss(tS, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+        for (int half = 0; half < (ROUTE ? 2 : 1); ++half) {
+          const uint64_t dq = (g == 0 && half == 0) ? dq0 : dq1, dk = dk0 + slot_off(sc + half);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint64_t off = (uint64_t)((kk >> 2) * (BOX_BYTES >> 4) + (kk & 3) * 2);
+            ptx::mma_bf16_ss(tS, dq + off, dk + off, idesc_qk, (half > 0 || kk > 0) ? 1u : 0u);
+          }
         }
       };
       auto pv = [&](int g, int sc, bool first) {
@@ -286,11 +324,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int sc = 0, it = 0;
       int pc0 = 0, pc1 = 0, ic0 = 0, ic1 = 0;  // P phases consumed, items finished, per group
       for (int item = item_of(0); ok && item < a.n_items; ++it, item = item_of(it)) {
-        const Item w = decode_item(a, item);
+        const Item w = decode_item<ROUTE>(a, item);
         if (*abort_flag || !ptx::mbar_wait(bar(B_QF), it & 1, a.status)) { ok = false; break; }
         ptx::tc_fence_after();
         // K_lo feeds the first S of every group that sees key tile lo
-        if (!slot_wait(sc)) { ok = false; break; }
+        if (!slot_wait(sc) || (ROUTE && !slot_wait(sc + 1))) { ok = false; break; }
         ptx::tc_fence_after();
 #pragma unroll
         for (int g = 0; g < 2; ++g)
@@ -300,10 +338,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         if (w.lo == w.hi) ptx::mma_commit(bar(B_QE));
         ptx::mma_commit(bar(B_SLE + sc % SLOTS));
+        if (ROUTE) ptx::mma_commit(bar(B_SLE + (sc + 1) % SLOTS));
         for (int t = w.lo; ok && t <= w.hi; ++t) {
-          const int scV = sc + 2 * (t - w.lo) + 1, scK1 = scV + 1;
+          const int scV = sc + PER_TILE * (t - w.lo) + PER_TILE - 1, scK1 = scV + 1;
           const bool more = t < w.hi;
-          if (!slot_wait(scV) || (more && !slot_wait(scK1))) { ok = false; break; }
+          if (!slot_wait(scV) || (more && !slot_wait(scK1)) || (ROUTE && more && !slot_wait(scK1 + 1))) {
+            ok = false;
+            break;
+          }
           ptx::tc_fence_after();
 #pragma unroll
           for (int g = 0; g < 2; ++g) {
@@ -332,10 +374,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (t + 1 == w.hi) ptx::mma_commit(bar(B_QE));  // the item's last QKs are issued
           ptx::mma_commit(bar(B_SLE + scV % SLOTS));
           if (more) ptx::mma_commit(bar(B_SLE + scK1 % SLOTS));
+          if (ROUTE && more) ptx::mma_commit(bar(B_SLE + (scK1 + 1) % SLOTS));
         }
         ++ic0;
         if (w.has_b) ++ic1;
-        sc += 2 * (w.hi - w.lo + 1);
+        sc += PER_TILE * (w.hi - w.lo + 1);
       }
       if (!ok) *abort_flag = 1;
       ptx::mma_commit(bar(B_DONE));
@@ -355,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     int cnt = 0, icnt = 0;
     for (int k = 0, item = item_of(0); ok && item < a.n_items; ++k, item = item_of(k)) {
-      const Item w = decode_item(a, item);
+      const Item w = decode_item<ROUTE>(a, item);
       if (g == 1 && !w.has_b) continue;
       const int qg = w.q0 + g * kQ;  // first query of this group's tile
       const int qi = qg + r;         // query position
@@ -413,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float2 e = ffma2(make_float2(x[32 * qd + 2 * i], x[32 * qd + 2 * i + 1]), c2, mc2);
-            const float2 p = make_float2(ex2(e.x), ex2(e.y));
+            const float2 p = (POLY > 0 && i % POLY == POLY - 1) ? exp2_poly(e) : make_float2(ex2(e.x), ex2(e.y));
             sm[i & 3] = fadd2(sm[i & 3], p);
             pk[i] = pack_bf16(p.x, p.y);
           }
@@ -453,25 +496,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++icnt;
       ptx::tc_fence_after();
       const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;
-      const bool store = qi < a.T;
-      bf16* dst = a.o + (size_t)(w.b * a.T + qi) * a.ldo + w.h * kD;
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t u[32];
-        ptx::tmem_ld32(tO + (uint32_t)(cc * 32), u);
-        ptx::tmem_ld_wait();
-        if (store) {
-          uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            d4[q] = make_uint4(pack_bf16(__uint_as_float(u[8 * q + 0]) * inv, __uint_as_float(u[8 * q + 1]) * inv),
-                               pack_bf16(__uint_as_float(u[8 * q + 2]) * inv, __uint_as_float(u[8 * q + 3]) * inv),
-                               pack_bf16(__uint_as_float(u[8 * q + 4]) * inv, __uint_as_float(u[8 * q + 5]) * inv),
-                               pack_bf16(__uint_as_float(u[8 * q + 6]) * inv, __uint_as_float(u[8 * q + 7]) * inv));
-        }
-      }
+      // read all of O_g, release it to the next item's P V, then store
+      uint32_t o0[32], o1[32], o2[32], o3[32];
+      ptx::tmem_ld32(tO, o0);
+      ptx::tmem_ld32(tO + 32, o1);
+      ptx::tmem_ld32(tO + 64, o2);
+      ptx::tmem_ld32(tO + 96, o3);
+      ptx::tmem_ld_wait();
       ptx::tc_fence_before();
       __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(B_OE + g));
+      if (qi < a.T) {
+        uint4* d4 = reinterpret_cast<uint4*>(a.o + (size_t)(w.b * a.T + qi) * a.ldo + w.h * kD);
+        auto put = [&](int q0, const uint32_t (&u)[32]) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            d4[q0 + q] = make_uint4(pack_bf16(__uint_as_float(u[8 * q + 0]) * inv, __uint_as_float(u[8 * q + 1]) * inv),
+                                    pack_bf16(__uint_as_float(u[8 * q + 2]) * inv, __uint_as_float(u[8 * q + 3]) * inv),
+                                    pack_bf16(__uint_as_float(u[8 * q + 4]) * inv, __uint_as_float(u[8 * q + 5]) * inv),
+                                    pack_bf16(__uint_as_float(u[8 * q + 6]) * inv, __uint_as_float(u[8 * q + 7]) * inv));
+        };
+        put(0, o0);
+        put(4, o1);
+        put(8, o2);
+        put(12, o3);
+      }
       if (lane == 0) ptx::mbar_arrive(bar(B_OE + g));
     }
     if (!ok) *abort_flag = 1;
@@ -485,14 +534,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-bool launch_attn_tc(const bf16* q, const bf16* k, const bf16* v, int ldq, int ldk, int ldv, bf16* o,
-                    int ldo, int B, int T, int H, int Hkv, int window, float scale, int* status,
-                    int num_sms, cudaStream_t st) {
+namespace {
+
+bool launch_attn_common(const bf16* q, const bf16* k, const bf16* v, const bf16* q1, const bf16* k1, int ldq,
+                        int ldk, int ldv, bf16* o, int ldo, int B, int T, int H, int Hkv, int window, float scale,
+                        int* status, int num_sms, cudaStream_t st) {
+  const bool route = q1 != nullptr;
   const int M = B * T;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, tq1, tk1;
   if (!make_tmap_2d(&tq, q, M, H * kD, ldq, kQ, 64)) return false;
   if (!make_tmap_2d(&tk, k, M, Hkv * kD, ldk, kK, 64)) return false;
   if (!make_tmap_2d(&tv, v, M, Hkv * kD, ldv, kK, 64)) return false;
+  if (!make_tmap_2d(&tq1, route ? q1 : q, M, H * kD, ldq, kQ, 64)) return false;
+  if (!make_tmap_2d(&tk1, route ? k1 : k, M, Hkv * kD, ldk, kK, 64)) return false;
   AttnArgs a;
   a.B = B;
   a.T = T;
@@ -501,18 +555,37 @@ bool launch_attn_tc(const bf16* q, const bf16* k, const bf16* v, int ldq, int ld
   a.window = (window <= 0 || window > T) ? T : window;
   a.ldo = ldo;
   a.n_qblocks = (T + kQ - 1) / kQ;
-  a.n_pairs = (a.n_qblocks + 1) / 2;
+  a.n_pairs = route ? a.n_qblocks : (a.n_qblocks + 1) / 2;
   a.n_items = a.n_pairs * B * H;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.o = o;
   a.status = status;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaFuncSetAttribute(k_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  });
+  static const int poly = getenv("NC_ATTN_POLY") ? atoi(getenv("NC_ATTN_POLY")) : 0;
+  void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, AttnArgs) =
+      route ? k_attn_tc<0, true>
+            : (poly == 2 ? k_attn_tc<2, false>
+                         : poly == 3 ? k_attn_tc<3, false>
+                                     : poly == 4 ? k_attn_tc<4, false> : poly == 8 ? k_attn_tc<8, false> : k_attn_tc<0, false>);
+  if (!smem_optin(kern, SMEM_BYTES)) return false;
   LaunchScope scope_(KK_ATTN_TC, st);
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
-  return launch_pdl(k_attn_tc, dim3(grid), dim3(kThreads), SMEM_BYTES, st, 1, tq, tk, tv, a) == cudaSuccess;
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), SMEM_BYTES, st, 1, tq, tk, tv, tq1, tk1, a) == cudaSuccess;
+}
+
+}  // namespace
+
+bool launch_attn_tc(const bf16* q, const bf16* k, const bf16* v, int ldq, int ldk, int ldv, bf16* o,
+                    int ldo, int B, int T, int H, int Hkv, int window, float scale, int* status,
+                    int num_sms, cudaStream_t st) {
+  return launch_attn_common(q, k, v, nullptr, nullptr, ldq, ldk, ldv, o, ldo, B, T, H, Hkv, window, scale, status,
+                            num_sms, st);
+}
+
+bool launch_attn_route_tc(const bf16* q2, const bf16* k2, const bf16* v2, const bf16* q1s, const bf16* k1, bf16* o,
+                          int B, int T, int H, int Hkv, int window, float scale, int* status, int num_sms,
+                          cudaStream_t st) {
+  return launch_attn_common(q2, k2, v2, q1s, k1, H * kD, Hkv * kD, Hkv * kD, o, H * kD, B, T, H, Hkv, window, scale,
+                            status, num_sms, st);
 }
 
 }  // namespace nc

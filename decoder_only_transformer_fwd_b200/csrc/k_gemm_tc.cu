@@ -25,6 +25,8 @@
 // unless asked.
 #include <cudaTypedefs.h>
 
+#include <string.h>
+
 #include <mutex>
 
 #include "epilogue.cuh"
@@ -59,11 +61,15 @@ struct TcArgs {
   int* status;
   // pair kernel, stream-K schedule (see PairSched); sk_ws holds one fp32
   // partial accumulator per CTA (128 x 256, column-major), sk_flags one word
-  // per CTA, set to sk_gen once that CTA's partial is written
+  // per CTA, set to sk_gen once that CTA's partial is written; a finishing
+  // pair waits (at most sk_wait_ns) until its contributors' flags equal
+  // sk_expect, which is sk_gen except under the timeout test hook
   int streamk;
   float* sk_ws;
   unsigned* sk_flags;
   unsigned sk_gen;
+  unsigned sk_expect;
+  unsigned long long sk_wait_ns;
 };
 
 // Pair tile pt -> (row-pair block, column tile).  Column-fastest order keeps
@@ -169,6 +175,18 @@ __device__ __forceinline__ int first_contributor(const PairSched& s, long long U
 }
 
 __device__ __forceinline__ float bits2f(uint32_t u) { return __uint_as_float(u); }
+
+// Per-row values of a tile that do not depend on its accumulator.  They are
+// loaded before the epilogue waits for the accumulator, so their memory
+// latency overlaps the tile's MMAs; the rows the epilogue will read later are
+// pulled into L2 at the same time.
+struct RowPre {
+  float rscale;  // 1 / rms of the A row (fused RMSNorm); 1 when unused
+  float gate;    // QKV value heads: the value-embedding gate
+  int y;         // CE / DZ: the row's target id, or -1
+  int tok;       // QKV value heads: the row's token id, clamped
+  float lse;     // DZ: the row's log-sum-exp
+};
 
 // The 32 x 32 chunk epilogues below receive the accumulator one row per lane
 // (TMEM lane = row) and stage it in the warp's shared-memory buffer (row
@@ -327,6 +345,68 @@ __device__ __forceinline__ void epi_store_chunk(const EpiParams& ep, const TcArg
   __syncwarp();
 }
 
+// EPI_DZ / EPI_F32: each lane first turns its row's 32 accumulator values
+// into the output value (for EPI_DZ the gradient of the mean softcapped
+// cross-entropy with respect to z, scaled by the row's 1 / rms), stages them,
+// and the transposed pass stores 8-byte bf16 or 16-byte fp32 quads.
+template <int MODE>
+__device__ __forceinline__ void epi_bwd_chunk(const EpiParams& ep, const TcArgs& a, float* stage, int row0, int n,
+                                              const uint32_t (&r)[32], int lane, const RowPre& pre, float ginv) {
+  if constexpr (MODE == EPI_DZ) {
+    // zhat = c tanh(z / c) = c - 2c / (e^{2z/c} + 1); p = e^{zhat - lse};
+    // d loss_mean / d z = (p - [n == y]) (1 - (zhat / c)^2) / count
+    const float k1 = 2.0f * 1.4426950408889634f / ep.cap;
+    const float c2 = -2.0f * ep.cap, inv_cap = 1.0f / ep.cap;
+    const float lse2 = pre.lse * 1.4426950408889634f;
+    const float scale = pre.y >= 0 ? pre.rscale * ginv : 0.f;  // ignored rows get no gradient
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float q = ptx::rcp(ptx::ex2(__uint_as_float(r[i]) * (pre.rscale * k1)) + 1.0f);
+      const float zh = fmaf(c2, q, ep.cap);
+      const float p = ptx::ex2(fmaf(zh, 1.4426950408889634f, -lse2));
+      const float th = zh * inv_cap;
+      const float d = (p - ((n + i == pre.y) ? 1.0f : 0.0f)) * (1.0f - th * th);
+      stage[lane * 33 + i] = (n + i < ep.vocab) ? d * scale : 0.f;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = __uint_as_float(r[i]);
+  }
+  __syncwarp();
+  const int q = lane >> 3, c4 = lane & 7;
+  const int col = n + 4 * c4;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int rr = 4 * i + q;
+    const int m = row0 + rr;
+    const float* sr = stage + rr * 33 + 4 * c4;
+    if (m < a.M) {
+      if constexpr (MODE == EPI_DZ) {
+        bf16* dst = reinterpret_cast<bf16*>(ep.out) + (size_t)m * ep.ldo + col;
+        if (col + 3 < a.N) {
+          const __nv_bfloat162 b0 = __floats2bfloat162_rn(sr[0], sr[1]), b1 = __floats2bfloat162_rn(sr[2], sr[3]);
+          *reinterpret_cast<uint2*>(dst) =
+              make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (col + e < a.N) dst[e] = __float2bfloat16_rn(sr[e]);
+        }
+      } else {
+        float* dst = reinterpret_cast<float*>(ep.out) + (size_t)m * ep.ldo + col;
+        if (col + 3 < a.N) {
+          *reinterpret_cast<float4*>(dst) = make_float4(sr[0], sr[1], sr[2], sr[3]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (col + e < a.N) dst[e] = sr[e];
+        }
+      }
+    }
+  }
+  __syncwarp();
+}
+
 // Fused QKV epilogue for the 128 columns of one head held in TMEM at taddr,
 // rows m0 .. m0 + 31 (one per lane): q and k heads get RoPE (position m % T)
 // and alpha * RMSNorm over the head; v heads get gate * VE[tok] added; one
@@ -466,16 +546,6 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
   }
 }
 
-// Per-row values of a tile that do not depend on its accumulator.  They are
-// loaded before the epilogue waits for the accumulator, so their memory
-// latency overlaps the tile's MMAs; the rows the epilogue will read later are
-// pulled into L2 at the same time.
-struct RowPre {
-  float rscale;  // 1 / rms of the A row (fused RMSNorm); 1 when unused
-  float gate;    // QKV value heads: the value-embedding gate
-  int y;         // CE: the row's target id, or -1
-  int tok;       // QKV value heads: the row's token id, clamped
-};
 
 template <int BN, int MODE>
 __device__ __forceinline__ RowPre epilogue_pre(const EpiParams& ep, const TcArgs& a, int mb, int nb, int g,
@@ -483,9 +553,9 @@ __device__ __forceinline__ RowPre epilogue_pre(const EpiParams& ep, const TcArgs
   constexpr int HALF = BN / 2;
   const int m = mb * kBM + g * 32 + lane;
   const int n_lo = nb * BN + half * HALF;
-  RowPre p{1.f, 0.f, -1, 0};
+  RowPre p{1.f, 0.f, -1, 0, 0.f};
   if (m >= a.M) return p;
-  if constexpr (MODE == EPI_QKV || MODE == EPI_RELU2 || MODE == EPI_CE) {
+  if constexpr (MODE == EPI_QKV || MODE == EPI_RELU2 || MODE == EPI_CE || MODE == EPI_DZ) {
     if (ep.ss_in != nullptr) {
       const float* sp = ep.ss_in + (size_t)m * ep.ss_in_parts;
       float t = 0.f;
@@ -516,10 +586,11 @@ __device__ __forceinline__ RowPre epilogue_pre(const EpiParams& ep, const TcArgs
         p.gate = ep.gate_scale / (1.0f + __expf(-p.rscale * d));
       }
     }
-  } else if constexpr (MODE == EPI_CE) {
+  } else if constexpr (MODE == EPI_CE || MODE == EPI_DZ) {
     int y = ep.targets[m];
     if (y != -1) y = min(max(y, 0), ep.vocab - 1);  // out-of-range ids are flagged by the combine
     p.y = y;
+    if constexpr (MODE == EPI_DZ) p.lse = ep.lse[m];
   }
   return p;
 }
@@ -626,6 +697,19 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs&
       ep.ce_sum[(size_t)m * ep.ce_tiles + nb * 2 + half] = sum;
       if (y >= n_lo && y < n_lo + HALF) ep.ce_tgt[m] = tgt;
     }
+  } else if constexpr (MODE == EPI_DZ || MODE == EPI_F32) {
+    const float ginv = MODE == EPI_DZ ? *ep.inv_count : 0.f;
+    uint32_t r[32];
+    ptx::tmem_ld32(taddr + (uint32_t)c_lo, r);
+#pragma unroll 1
+    for (int c = 0; c < HALF; c += 32) {
+      ptx::tmem_ld_wait();
+      uint32_t rc[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) rc[i] = r[i];
+      if (c + 32 < HALF) ptx::tmem_ld32(taddr + (uint32_t)(c_lo + c + 32), r);
+      epi_bwd_chunk<MODE>(ep, a, stage, mb * kBM + g * 32, n_lo + c, rc, lane, pre, ginv);
+    }
   } else if constexpr (MODE == EPI_RESID) {
     float ssr[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     const int row0 = mb * kBM + g * 32;
@@ -690,7 +774,12 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs&
   }
 }
 
-template <int BN, int MODE>
+// AMN / BMN = 1: that operand is stored MN-major (the transpose of the
+// K-major layout), loaded as 64 x 64 boxes (64 MN elements = one 128-byte
+// swizzled row, 64 k rows) placed 8 KB apart, and read by the MMA through an
+// MN-major descriptor (leading offset 8 KB between 64-wide MN blocks, a
+// 16-row k step = 2 KB).
+template <int BN, int MODE, int AMN = 0, int BMN = 0>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const TcArgs a, const EpiParams ep) {
@@ -738,7 +827,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int nk = a.K / kBK;
+  const int nk = (a.K + kBK - 1) / kBK;  // k beyond K reads zeros (tensor-map bounds)
   pdl_wait();  // the operands and the epilogue's inputs come from earlier kernels
 
   if (warp == 0) {
@@ -756,8 +845,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           ptx::mbar_arrive_expect_tx(full(stage), Cf::STAGE_BYTES);
-          ptx::tma_load_2d(sA(stage), &tmA, full(stage), kb * kBK, mb * kBM);
-          ptx::tma_load_2d(sB(stage), &tmB, full(stage), kb * kBK, nb * BN);
+          if constexpr (AMN) {
+#pragma unroll
+            for (int j = 0; j < kBM / 64; ++j)
+              ptx::tma_load_2d(sA(stage) + j * 8192, &tmA, full(stage), mb * kBM + 64 * j, kb * kBK);
+          } else {
+            ptx::tma_load_2d(sA(stage), &tmA, full(stage), kb * kBK, mb * kBM);
+          }
+          if constexpr (BMN) {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              ptx::tma_load_2d(sB(stage) + j * 8192, &tmB, full(stage), nb * BN + 64 * j, kb * kBK);
+          } else {
+            ptx::tma_load_2d(sB(stage), &tmB, full(stage), kb * kBK, nb * BN);
+          }
           issued |= 1u << stage;
           par = (par & ~(1u << stage)) | (ph << stage);
           if (++stage == S) {
@@ -774,7 +875,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (ptx::elect_one()) {
       // ---------------- MMA issuer ----------------
-      constexpr uint32_t idesc = ptx::idesc_bf16(kBM, BN);
+      constexpr uint32_t idesc = ptx::idesc_bf16(kBM, BN, AMN, BMN);
       int stage = 0, acc = 0;
       uint32_t ph = 0, aph = 0;
       for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
@@ -792,11 +893,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           ptx::tc_fence_after();
-          const uint64_t da = ptx::desc_kmajor_sw128(sA(stage));
-          const uint64_t db = ptx::desc_kmajor_sw128(sB(stage));
+          const uint64_t da = AMN ? ptx::desc_mnmajor_sw128(sA(stage), 8192) : ptx::desc_kmajor_sw128(sA(stage));
+          const uint64_t db = BMN ? ptx::desc_mnmajor_sw128(sB(stage), 8192) : ptx::desc_kmajor_sw128(sB(stage));
+          // a k step of 16 is 32 bytes along a K-major row, 16 rows (2 KB) of an MN-major box
+          constexpr uint64_t ka = AMN ? (2048 >> 4) : 2, kb16 = BMN ? (2048 >> 4) : 2;
 #pragma unroll
           for (int k = 0; k < kBK / kUK; ++k)
-            ptx::mma_bf16_ss(d, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            ptx::mma_bf16_ss(d, da + ka * k, db + kb16 * k, idesc, (kb | k) != 0 ? 1u : 0u);
           ptx::mma_commit(empty(stage));
           if (++stage == S) {
             stage = 0;
@@ -1090,11 +1193,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           for (int cp = c_first; cp < cid; ++cp) {
             if (U * (cp + 1) / ncl == U * cp / ncl) continue;  // pair cp has no tail units
             const unsigned* flag = a.sk_flags + cp * 2 + (int)rank;
-            bool ready = ptx::ld_acquire_gpu(flag) == a.sk_gen;
+            bool ready = ptx::ld_acquire_gpu(flag) == a.sk_expect;
             if (!ready) {
               const uint64_t t0 = ptx::globaltimer();
-              while (!(ready = ptx::ld_acquire_gpu(flag) == a.sk_gen))
-                if (ptx::globaltimer() - t0 > kWaitLimitNs) break;
+              while (!(ready = ptx::ld_acquire_gpu(flag) == a.sk_expect))
+                if (ptx::globaltimer() - t0 > a.sk_wait_ns) break;
             }
             if (!__all_sync(0xffffffffu, ready)) {
               atomicOr(a.status, kStatusTimeout);
@@ -1151,34 +1254,38 @@ EncodeTiledFn get_encode() {
 }
 
 template <int BN, int MODE>
-void launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep, int grid,
+bool launch_mode(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep, int grid,
                  cudaStream_t st) {
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaFuncSetAttribute(k_gemm_tc<BN, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<BN>::SMEM);
-  });
-  launch_pdl(k_gemm_tc<BN, MODE>, dim3(grid), dim3(kThreads), TcCfg<BN>::SMEM, st, 1, ta, tb, a, ep);
+  if (!smem_optin(k_gemm_tc<BN, MODE>, TcCfg<BN>::SMEM)) return false;
+  return launch_pdl(k_gemm_tc<BN, MODE>, dim3(grid), dim3(kThreads), TcCfg<BN>::SMEM, st, 1, ta, tb, a, ep) ==
+         cudaSuccess;
+}
+
+template <int MODE, int AMN, int BMN>
+bool launch_layout_mode(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep, int grid,
+                        cudaStream_t st) {
+  if (!smem_optin(k_gemm_tc<256, MODE, AMN, BMN>, TcCfg<256>::SMEM)) return false;
+  return launch_pdl(k_gemm_tc<256, MODE, AMN, BMN>, dim3(grid), dim3(kThreads), TcCfg<256>::SMEM, st, 1, ta, tb, a,
+                    ep) == cudaSuccess;
 }
 
 template <int MODE>
-void launch_pair_mode(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep,
+bool launch_pair_mode(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep,
                       int nclusters, cudaStream_t st) {
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaFuncSetAttribute(k_gemm_tc2<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, PairCfg::SMEM);
-  });
-  launch_pdl(k_gemm_tc2<MODE>, dim3(2 * nclusters), dim3(kPairThreads), PairCfg::SMEM, st, 2, ta, tb, a, ep);
+  if (!smem_optin(k_gemm_tc2<MODE>, PairCfg::SMEM)) return false;
+  return launch_pdl(k_gemm_tc2<MODE>, dim3(2 * nclusters), dim3(kPairThreads), PairCfg::SMEM, st, 2, ta, tb, a,
+                    ep) == cudaSuccess;
 }
 
 bool launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep, int nclusters,
                  cudaStream_t st) {
   switch (ep.mode) {
-    case EPI_STORE: launch_pair_mode<EPI_STORE>(ta, tb, a, ep, nclusters, st); return true;
-    case EPI_RELU2: launch_pair_mode<EPI_RELU2>(ta, tb, a, ep, nclusters, st); return true;
-    case EPI_RESID: launch_pair_mode<EPI_RESID>(ta, tb, a, ep, nclusters, st); return true;
-    case EPI_BLOCK_END: launch_pair_mode<EPI_BLOCK_END>(ta, tb, a, ep, nclusters, st); return true;
-    case EPI_CE: launch_pair_mode<EPI_CE>(ta, tb, a, ep, nclusters, st); return true;
-    case EPI_QKV: launch_pair_mode<EPI_QKV>(ta, tb, a, ep, nclusters, st); return true;
+    case EPI_STORE: return launch_pair_mode<EPI_STORE>(ta, tb, a, ep, nclusters, st);
+    case EPI_RELU2: return launch_pair_mode<EPI_RELU2>(ta, tb, a, ep, nclusters, st);
+    case EPI_RESID: return launch_pair_mode<EPI_RESID>(ta, tb, a, ep, nclusters, st);
+    case EPI_BLOCK_END: return launch_pair_mode<EPI_BLOCK_END>(ta, tb, a, ep, nclusters, st);
+    case EPI_CE: return launch_pair_mode<EPI_CE>(ta, tb, a, ep, nclusters, st);
+    case EPI_QKV: return launch_pair_mode<EPI_QKV>(ta, tb, a, ep, nclusters, st);
     default: return false;
   }
 }
@@ -1187,12 +1294,12 @@ template <int BN>
 bool launch_bn(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep, int grid,
                cudaStream_t st) {
   switch (ep.mode) {
-    case EPI_STORE: launch_mode<BN, EPI_STORE>(ta, tb, a, ep, grid, st); return true;
-    case EPI_RELU2: launch_mode<BN, EPI_RELU2>(ta, tb, a, ep, grid, st); return true;
-    case EPI_RESID: launch_mode<BN, EPI_RESID>(ta, tb, a, ep, grid, st); return true;
-    case EPI_BLOCK_END: launch_mode<BN, EPI_BLOCK_END>(ta, tb, a, ep, grid, st); return true;
-    case EPI_CE: launch_mode<BN, EPI_CE>(ta, tb, a, ep, grid, st); return true;
-    case EPI_QKV: launch_mode<BN, EPI_QKV>(ta, tb, a, ep, grid, st); return true;
+    case EPI_STORE: return launch_mode<BN, EPI_STORE>(ta, tb, a, ep, grid, st);
+    case EPI_RELU2: return launch_mode<BN, EPI_RELU2>(ta, tb, a, ep, grid, st);
+    case EPI_RESID: return launch_mode<BN, EPI_RESID>(ta, tb, a, ep, grid, st);
+    case EPI_BLOCK_END: return launch_mode<BN, EPI_BLOCK_END>(ta, tb, a, ep, grid, st);
+    case EPI_CE: return launch_mode<BN, EPI_CE>(ta, tb, a, ep, grid, st);
+    case EPI_QKV: return launch_mode<BN, EPI_QKV>(ta, tb, a, ep, grid, st);
     default: return false;
   }
 }
@@ -1230,6 +1337,31 @@ bool make_tmap_4d(CUtensorMap* map, const void* ptr, const uint64_t (&dims)[4],
 
 int gemm_tc_bn(int N) { return (N % 256 == 0) ? 256 : 128; }
 
+bool launch_gemm_tc_layout(const bf16* A, int lda, int a_mn, const bf16* Bm, int ldb, int b_mn, int M, int N, int K,
+                           const EpiParams& ep, int* status, int num_sms, cudaStream_t st) {
+  constexpr int BN = 256;
+  CUtensorMap ta, tb;
+  // K-major: [rows, K] with boxes of 64 k x rows; MN-major: [K, MN] with 64 x 64 boxes
+  if (!(a_mn ? make_tmap_2d(&ta, A, K, M, lda, 64, 64) : make_tmap_2d(&ta, A, M, K, lda, kBM, kBK))) return false;
+  if (!(b_mn ? make_tmap_2d(&tb, Bm, K, N, ldb, 64, 64) : make_tmap_2d(&tb, Bm, N, K, ldb, BN, kBK))) return false;
+  TcArgs a;
+  memset(&a, 0, sizeof(a));
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.tiles_m = (M + kBM - 1) / kBM;
+  a.tiles_n = (N + BN - 1) / BN;
+  a.num_tiles = a.tiles_m * a.tiles_n;
+  a.status = status;
+  a.sk_wait_ns = kWaitLimitNs;
+  const int grid = a.num_tiles < num_sms ? a.num_tiles : num_sms;
+  LaunchScope scope_(KK_GEMM_TC_BWD, st);
+  if (ep.mode == EPI_DZ && !a_mn && !b_mn) return launch_layout_mode<EPI_DZ, 0, 0>(ta, tb, a, ep, grid, st);
+  if (ep.mode == EPI_F32 && !a_mn && b_mn) return launch_layout_mode<EPI_F32, 0, 1>(ta, tb, a, ep, grid, st);
+  if (ep.mode == EPI_F32 && a_mn && b_mn) return launch_layout_mode<EPI_F32, 1, 1>(ta, tb, a, ep, grid, st);
+  return false;
+}
+
 bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int N, int K,
                     const EpiParams& ep, int* status, int num_sms, cudaStream_t st, bool pair,
                     const StreamK* sk) {
@@ -1257,6 +1389,8 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
     a.sk_ws = nullptr;
     a.sk_flags = nullptr;
     a.sk_gen = 0;
+    a.sk_expect = 0;
+    a.sk_wait_ns = kWaitLimitNs;
     // (and when the partial wave is at least a quarter full, so that a tile is
     // cut among a few pairs only)
     if (sk != nullptr && sk->ws != nullptr && ncl <= sk->max_pairs && ep.mode == EPI_BLOCK_END && nk >= 1 &&
@@ -1265,6 +1399,9 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
       a.sk_ws = sk->ws;
       a.sk_flags = sk->flags;
       a.sk_gen = sk->gen;
+      unsigned skew = 0;
+      flag_wait_test(&a.sk_wait_ns, &skew);
+      a.sk_expect = sk->gen + skew;
     }
     LaunchScope scope_(KK_GEMM_TC, st);
     return launch_pair(ta, tb, a, ep, ncl, st);
@@ -1285,6 +1422,8 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
   a.sk_ws = nullptr;
   a.sk_flags = nullptr;
   a.sk_gen = 0;
+  a.sk_expect = 0;
+  a.sk_wait_ns = kWaitLimitNs;
   const int grid = a.num_tiles < num_sms ? a.num_tiles : num_sms;
   LaunchScope scope_(KK_GEMM_TC, st);
   return BN == 256 ? launch_bn<256>(ta, tb, a, ep, grid, st) : launch_bn<128>(ta, tb, a, ep, grid, st);

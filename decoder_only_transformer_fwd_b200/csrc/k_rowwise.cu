@@ -93,6 +93,125 @@ __global__ void k_embed(const T* __restrict__ wte, const int32_t* __restrict__ t
   }
 }
 
+// bf16 tables, C = 32 * EPL: one warp walks a run of `run` consecutive
+// positions of one row.  Lane l holds elements [(k * 32 + l) * VW, + VW) of
+// every row for k < EPL / VW, so each load and store is a 16- or 8-byte vector
+// and consecutive lanes touch consecutive bytes.  The normalised embedding of
+// the position before the run is loaded once and then carried in registers
+// from one position to the next (it is what smear mixes in).  Same outputs as
+// k_embed: x0, x = (lam0 + mu0) x0, bf16(x) and its sum of squares.
+template <int EPL>
+__global__ void __launch_bounds__(128) k_embed_vec(
+    const bf16* __restrict__ wte, const int32_t* __restrict__ tokens, const float* __restrict__ smear_gate,
+    int smear, int gc, const float* __restrict__ lam0p, const float* __restrict__ mu0p, float eps, int B, int T_,
+    int C, int V, int run, float* __restrict__ x, float* __restrict__ x0, bf16* __restrict__ xb,
+    float* __restrict__ ss, int ss_parts, int* status) {
+  constexpr int VW = (EPL % 8 == 0) ? 8 : 4;  // elements per vector access
+  constexpr int NCH = EPL / VW;
+  pdl_launch_dependents();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int wid = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int runs_per_row = (T_ + run - 1) / run;
+  if (wid >= B * runs_per_row) return;
+  const int b = wid / runs_per_row;
+  const int t0 = (wid % runs_per_row) * run;
+  const int t1 = min(T_, t0 + run);
+  const float inv_c = 1.0f / (float)C;
+  // the normalised embedding row of token `tok` into v
+  auto load_norm = [&](int tok, float (&v)[EPL]) {
+    const bf16* row = wte + (size_t)tok * C;
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+      const int e0 = (k * 32 + lane) * VW;
+      if constexpr (VW == 8) {
+        const uint4 u = *reinterpret_cast<const uint4*>(row + e0);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+          v[k * 8 + 2 * i] = f.x;
+          v[k * 8 + 2 * i + 1] = f.y;
+        }
+      } else {
+        const uint2 u = *reinterpret_cast<const uint2*>(row + e0);
+        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+        const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+        v[k * 4 + 0] = f0.x;
+        v[k * 4 + 1] = f0.y;
+        v[k * 4 + 2] = f1.x;
+        v[k * 4 + 3] = f1.y;
+      }
+    }
+    float sq = 0.f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) sq = fmaf(v[i], v[i], sq);
+    const float r = 1.0f / sqrtf(warp_sum(sq) * inv_c + eps);
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) v[i] *= r;
+  };
+  auto token = [&](int t) {
+    int tok = tokens[(size_t)b * T_ + t];
+    if (tok < 0 || tok >= V) {
+      if (lane == 0) atomicOr(status, kStatusData);
+      tok = min(max(tok, 0), V - 1);
+    }
+    return tok;
+  };
+  float prev[EPL];
+  if (smear && t0 > 0) {
+    // its out-of-range flag is raised by the warp that owns that position
+    int tp = tokens[(size_t)b * T_ + t0 - 1];
+    load_norm(min(max(tp, 0), V - 1), prev);
+  }
+  const float scale = *lam0p + *mu0p;
+  for (int t = t0; t < t1; ++t) {
+    float cur[EPL];
+    load_norm(token(t), cur);
+    float g = 0.f;
+    if (smear && t > 0) {
+      float d = 0.f;
+#pragma unroll
+      for (int k = 0; k < NCH; ++k)
+#pragma unroll
+        for (int i = 0; i < VW; ++i) {
+          const int c = (k * 32 + lane) * VW + i;
+          if (c < gc) d = fmaf(smear_gate[c], cur[k * VW + i], d);
+        }
+      g = sigmoidf_(warp_sum(d));
+    }
+    const size_t m = (size_t)b * T_ + t;
+    float sq = 0.f;
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+      const int e0 = (k * 32 + lane) * VW;
+      float o[VW];
+#pragma unroll
+      for (int i = 0; i < VW; ++i) {
+        o[i] = (smear && t > 0) ? fmaf(g, prev[k * VW + i], cur[k * VW + i]) : cur[k * VW + i];
+        prev[k * VW + i] = cur[k * VW + i];
+      }
+#pragma unroll
+      for (int i = 0; i < VW; i += 4) {
+        *reinterpret_cast<float4*>(x0 + m * C + e0 + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+        const float4 xv = make_float4(scale * o[i], scale * o[i + 1], scale * o[i + 2], scale * o[i + 3]);
+        *reinterpret_cast<float4*>(x + m * C + e0 + i) = xv;
+        sq = fmaf(xv.x, xv.x, fmaf(xv.y, xv.y, fmaf(xv.z, xv.z, fmaf(xv.w, xv.w, sq))));
+        if (xb != nullptr) {
+          const __nv_bfloat162 b0 = __floats2bfloat162_rn(xv.x, xv.y), b1 = __floats2bfloat162_rn(xv.z, xv.w);
+          *reinterpret_cast<uint2*>(xb + m * C + e0 + i) =
+              make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
+        }
+      }
+    }
+    if (xb != nullptr) {
+      // the first block's norm input: sum of squares in slot 0, other slots 0
+      sq = warp_sum(sq);
+      for (int j = lane; j < ss_parts; j += 32) ss[m * ss_parts + j] = j == 0 ? sq : 0.f;
+    }
+  }
+}
+
 // xn = RMSNorm(x) (act dtype), one warp per row; optionally the value-embedding
 // gate g[m, h] = gate_scale * sigmoid(xn[:gc] . W_gate[h]) from the fp32
 // normalised values.
@@ -264,6 +383,96 @@ __global__ void k_rope_qknorm_copy(const T* q, const T* k, T* qo, T* ko, int T_,
   rope_norm_head<T>(src, dst, cos_t + (size_t)t * (D / 2), sin_t + (size_t)t * (D / 2), alpha, eps, lane);
 }
 
+// The same for bf16 q/k with 16-byte accesses: eight lanes per head vector,
+// lane i holding elements [8 i, 8 i + 8) of each half (so the pairs (j, j + 64)
+// it rotates are its own), the sum of squares reduced over the eight lanes.
+// A warp covers four head vectors.
+__global__ void __launch_bounds__(256) k_rope_qknorm_copy_bf16(
+    const bf16* __restrict__ q, const bf16* __restrict__ k, bf16* __restrict__ qo, bf16* __restrict__ ko, int T_,
+    int H, int Hkv, const float* __restrict__ cos_t, const float* __restrict__ sin_t, float alpha, float eps,
+    int M) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int slots = H + Hkv;
+  const long long hv = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * 4 + (lane >> 3);
+  const bool valid = hv < (long long)M * slots;
+  const int m = valid ? (int)(hv / slots) : 0;
+  const int s = valid ? (int)(hv % slots) : 0;
+  const int t = m % T_;
+  const int i8 = (lane & 7) * 8;
+  const bf16* src = s < H ? q + ((size_t)m * H + s) * 128 : k + ((size_t)m * Hkv + (s - H)) * 128;
+  bf16* dst = s < H ? qo + ((size_t)m * H + s) * 128 : ko + ((size_t)m * Hkv + (s - H)) * 128;
+  float a[8], bb[8], cs[8], sn[8];
+  if (valid) {
+    const uint4 ua = *reinterpret_cast<const uint4*>(src + i8);
+    const uint4 ub = *reinterpret_cast<const uint4*>(src + 64 + i8);
+    const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w}, wb[4] = {ub.x, ub.y, ub.z, ub.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wa[i]));
+      const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wb[i]));
+      a[2 * i] = fa.x;
+      a[2 * i + 1] = fa.y;
+      bb[2 * i] = fb.x;
+      bb[2 * i + 1] = fb.y;
+    }
+    const float4* c4 = reinterpret_cast<const float4*>(cos_t + (size_t)t * 64 + i8);
+    const float4* s4 = reinterpret_cast<const float4*>(sin_t + (size_t)t * 64 + i8);
+    const float4 c0 = c4[0], c1 = c4[1], s0 = s4[0], s1 = s4[1];
+    const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      cs[i] = cv[i];
+      sn[i] = sv[i];
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = bb[i] = cs[i] = sn[i] = 0.f;
+  }
+  float y1[8], y2[8], ssq = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    y1[i] = a[i] * cs[i] + bb[i] * sn[i];
+    y2[i] = -a[i] * sn[i] + bb[i] * cs[i];
+    ssq = fmaf(y1[i], y1[i], fmaf(y2[i], y2[i], ssq));
+  }
+  ssq += __shfl_xor_sync(0xffffffffu, ssq, 1);
+  ssq += __shfl_xor_sync(0xffffffffu, ssq, 2);
+  ssq += __shfl_xor_sync(0xffffffffu, ssq, 4);
+  const float r = alpha / sqrtf(ssq / 128.0f + eps);
+  if (valid) {
+    uint32_t w1[4], w2[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 p1 = __floats2bfloat162_rn(y1[2 * i] * r, y1[2 * i + 1] * r);
+      const __nv_bfloat162 p2 = __floats2bfloat162_rn(y2[2 * i] * r, y2[2 * i + 1] * r);
+      w1[i] = *reinterpret_cast<const uint32_t*>(&p1);
+      w2[i] = *reinterpret_cast<const uint32_t*>(&p2);
+    }
+    *reinterpret_cast<uint4*>(dst + i8) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+    *reinterpret_cast<uint4*>(dst + 64 + i8) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+  }
+}
+
+// out = bf16(g * in) over n elements (n % 8 == 0), 16-byte accesses.
+__global__ void k_scale_bf16(const bf16* __restrict__ in, bf16* __restrict__ out, long long n8, float g) {
+  pdl_launch_dependents();
+  pdl_wait();
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (long long)gridDim.x * blockDim.x) {
+    const uint4 u = reinterpret_cast<const uint4*>(in)[i];
+    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+      const __nv_bfloat162 b = __floats2bfloat162_rn(g * f.x, g * f.y);
+      w[j] = *reinterpret_cast<const uint32_t*>(&b);
+    }
+    reinterpret_cast<uint4*>(out)[i] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
 // Per-token CE from materialised softcapped logits (fp32 path): one CTA per row.
 __global__ void k_ce_rows(const float* logits, int ldl, const int32_t* targets, int V, float* loss,
                           int* status) {
@@ -298,7 +507,7 @@ __global__ void k_ce_rows(const float* logits, int ldl, const int32_t* targets, 
 // Merge per-(row, tile) partial sums sum_n exp(zhat_n - offset) into the
 // row's log-sum-exp and subtract the target's zhat.  One warp per row.
 __global__ void k_ce_combine(const float* ce_sum, const float* ce_tgt, int n_tiles, float offset,
-                             const int32_t* targets, int M, int V, float* loss, int* status) {
+                             const int32_t* targets, int M, int V, float* loss, float* lse, int* status) {
   pdl_launch_dependents();
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -310,12 +519,61 @@ __global__ void k_ce_combine(const float* ce_sum, const float* ce_tgt, int n_til
   s = warp_sum(s);
   if (lane == 0) {
     const int y = targets[m];
+    const float row_lse = offset + logf(s);
     float l = 0.f;
     if (y != -1) {
       if (y < 0 || y >= V) atomicOr(status, kStatusData);
-      l = (offset + logf(s)) - ce_tgt[m];
+      l = row_lse - ce_tgt[m];
     }
     loss[m] = l;
+    if (lse != nullptr) lse[m] = row_lse;
+  }
+}
+
+// 1 / (number of targets != -1), 0 when there is none.  One CTA.
+__global__ void k_inv_count(const int32_t* targets, int n, float* inv_count) {
+  pdl_launch_dependents();
+  pdl_wait();
+  __shared__ int part[32];
+  int c = 0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) c += targets[i] != -1;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int total = 0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) total += part[i];
+    *inv_count = total > 0 ? 1.0f / (float)total : 0.f;
+  }
+}
+
+// RMSNorm backward ("The Mathematics of Karpathy's nanochat", §RMS
+// Normalization: xn = x r, r = (mean(x^2) + eps)^(-1/2)): with g = r dL/dxn,
+// dL/dx = r dL/dxn - x r^3 (x . dL/dxn) / C = g - x r^2 (x . g) / C.  One warp
+// per row, 16-byte accesses (C % 4 == 0).
+__global__ void k_rmsnorm_bwd(const float* __restrict__ x, const float* __restrict__ g, float* __restrict__ dx,
+                              int M, int C, float eps) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (m >= M) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)m * C);
+  const float4* gr = reinterpret_cast<const float4*>(g + (size_t)m * C);
+  float ss = 0.f, xg = 0.f;
+  for (int i = lane; i < C / 4; i += 32) {
+    const float4 a = xr[i], b = gr[i];
+    ss = fmaf(a.x, a.x, fmaf(a.y, a.y, fmaf(a.z, a.z, fmaf(a.w, a.w, ss))));
+    xg = fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, xg))));
+  }
+  ss = warp_sum(ss);
+  xg = warp_sum(xg);
+  const float k = xg / (ss + eps * (float)C);  // r^2 (x . g) / C
+  float4* dr = reinterpret_cast<float4*>(dx + (size_t)m * C);
+  for (int i = lane; i < C / 4; i += 32) {
+    const float4 a = xr[i], b = gr[i];
+    dr[i] = make_float4(b.x - k * a.x, b.y - k * a.y, b.z - k * a.z, b.w - k * a.w);
   }
 }
 
@@ -356,6 +614,24 @@ void launch_embed(const void* wte, const int32_t* tokens, const float* smear_gat
                   cudaStream_t st) {
   LaunchScope scope_(KK_EMBED, st);
   const int M = B * T;
+  if (act_bf16 && C % 128 == 0 && C <= 2048) {
+    constexpr int kRun = 4;
+    const int warps = B * ((T + kRun - 1) / kRun);
+    const dim3 grid((warps + 3) / 4), block(128);
+    const bf16* w = (const bf16*)wte;
+    switch (C / 32) {
+#define NC_EMBED_CASE(E)                                                                                      \
+  case E:                                                                                                     \
+    launch_pdl(k_embed_vec<E>, grid, block, 0, st, 1, w, tokens, smear_gate, smear, gate_channels, lam0, mu0, \
+               eps, B, T, C, V, kRun, x, x0, xb, ss, ss_parts, status);                                       \
+    return;
+      NC_EMBED_CASE(4) NC_EMBED_CASE(8) NC_EMBED_CASE(12) NC_EMBED_CASE(16) NC_EMBED_CASE(20) NC_EMBED_CASE(24)
+      NC_EMBED_CASE(28) NC_EMBED_CASE(32) NC_EMBED_CASE(36) NC_EMBED_CASE(40) NC_EMBED_CASE(44) NC_EMBED_CASE(48)
+      NC_EMBED_CASE(52) NC_EMBED_CASE(56) NC_EMBED_CASE(60) NC_EMBED_CASE(64)
+#undef NC_EMBED_CASE
+      default: break;
+    }
+  }
   const size_t sh = (size_t)(2 * C + 32) * sizeof(float);
   if (act_bf16)
     launch_pdl(k_embed<bf16>, dim3(M), dim3(256), sh, st, 1, (const bf16*)wte, tokens, smear_gate, smear,
@@ -413,6 +689,12 @@ void launch_rope_qknorm_copy(const void* q, const void* k, void* qo, void* ko, i
   const int M = B * T;
   const long long warps = (long long)M * (H + Hkv);
   const int wpb = 8;
+  if (act_bf16 && D == 128) {
+    const long long vwarps = (warps + 3) / 4;  // four head vectors per warp
+    launch_pdl(k_rope_qknorm_copy_bf16, dim3((unsigned)((vwarps + wpb - 1) / wpb)), dim3(wpb * 32), 0, st, 1,
+               (const bf16*)q, (const bf16*)k, (bf16*)qo, (bf16*)ko, T, H, Hkv, cos_t, sin_t, alpha, eps, M);
+    return;
+  }
   const unsigned grid = (unsigned)((warps + wpb - 1) / wpb);
   if (act_bf16)
     launch_pdl(k_rope_qknorm_copy<bf16>, dim3(grid), dim3(wpb * 32), 0, st, 1, (const bf16*)q, (const bf16*)k,
@@ -429,11 +711,31 @@ void launch_ce_rows(const float* logits, int ldl, const int32_t* targets, int M,
 }
 
 void launch_ce_combine(const float* ce_sum, const float* ce_tgt, int n_tiles, float offset,
-                       const int32_t* targets, int M, int V, float* loss, int* status, cudaStream_t st) {
+                       const int32_t* targets, int M, int V, float* loss, float* lse, int* status, cudaStream_t st) {
   LaunchScope scope_(KK_CE_COMBINE, st);
   const int wpb = 8;
   launch_pdl(k_ce_combine, dim3((M + wpb - 1) / wpb), dim3(wpb * 32), 0, st, 1, ce_sum, ce_tgt, n_tiles, offset,
-             targets, M, V, loss, status);
+             targets, M, V, loss, lse, status);
+}
+
+void launch_scale_bf16(const bf16* in, bf16* out, long long n, float g, int num_sms, cudaStream_t st) {
+  LaunchScope scope_(KK_ROPE_QKNORM, st);
+  const long long n8 = n / 8;
+  long long blocks = (n8 + 255) / 256;
+  if (blocks > 8LL * num_sms) blocks = 8LL * num_sms;
+  if (blocks < 1) blocks = 1;
+  launch_pdl(k_scale_bf16, dim3((unsigned)blocks), dim3(256), 0, st, 1, in, out, n8, g);
+}
+
+void launch_inv_count(const int32_t* targets, int n, float* inv_count, cudaStream_t st) {
+  LaunchScope scope_(KK_HEAD_BWD_ROWS, st);
+  launch_pdl(k_inv_count, dim3(1), dim3(1024), 0, st, 1, targets, n, inv_count);
+}
+
+void launch_rmsnorm_bwd(const float* x, const float* g, float* dx, int M, int C, float eps, cudaStream_t st) {
+  LaunchScope scope_(KK_HEAD_BWD_ROWS, st);
+  const int wpb = 8;
+  launch_pdl(k_rmsnorm_bwd, dim3((M + wpb - 1) / wpb), dim3(wpb * 32), 0, st, 1, x, g, dx, M, C, eps);
 }
 
 void launch_loss_mean(const float* loss, const int32_t* targets, int n, float* out, cudaStream_t st) {

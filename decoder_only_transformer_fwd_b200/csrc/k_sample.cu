@@ -515,11 +515,8 @@ template <typename TW, int NB>
 void launch_last_logits_nb(const float* x, int ldx, int T, int b0, const TW* W, int V, int C, float cap, float eps,
                            float* out, int ldo, int num_sms, int* status, cudaStream_t st) {
   const LastGeom g = last_geom(C, (int)sizeof(TW), NB);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_last_logits<TW, NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
-    attr = true;
-  }
+  // a failure here leaves the launch to fail, which the entry point reports
+  if (!smem_optin(k_last_logits<TW, NB>, 220 * 1024)) return;
   launch_pdl(k_last_logits<TW, NB>, dim3(num_sms), dim3(kLastThreads), g.smem, st, 1, x, ldx, T, b0, W, V, C, cap,
              eps, out, ldo, g.stages, status);
 }
@@ -563,11 +560,7 @@ static bool sample_in_smem(int V) { return (size_t)V * 4 <= kSampleSmemMax; }
 void launch_sample(const float* logits, int B, int V, int ldl, float temperature, int top_k,
                    const float* uniforms, int32_t* out, int* status, cudaStream_t st) {
   LaunchScope scope_(KK_SAMPLE, st);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k_sample, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(kSampleSmemMax + kCand * 4));
-    attr = true;
-  }
+  if (!smem_optin(k_sample, (int)(kSampleSmemMax + kCand * 4))) return;
   const bool sm = sample_in_smem(V);
   launch_pdl(k_sample, dim3(B), dim3(kSampleThreads), (size_t)kCand * 4 + (sm ? (size_t)V * 4 : 0), st, 1, logits, V,
              ldl, temperature,

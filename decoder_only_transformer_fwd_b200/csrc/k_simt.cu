@@ -193,11 +193,11 @@ void launch_attn_simt(const void* q, const void* k, const void* v, int ldq, int 
   const size_t sh = (size_t)(2 * kAD * 65 + kAK * kAD + kAK * 65) * sizeof(float);
   dim3 grid((T + kAQ - 1) / kAQ, H, B);
   if (act_bf16) {
-    cudaFuncSetAttribute(k_attn_simt<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
+    if (!smem_optin(k_attn_simt<bf16>, (int)sh)) return;
     k_attn_simt<bf16><<<grid, 256, sh, st>>>((const bf16*)q, (const bf16*)k, (const bf16*)v, ldq, ldk,
                                              ldv, (bf16*)o, ldo, T, H, Hkv, window, scale);
   } else {
-    cudaFuncSetAttribute(k_attn_simt<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh);
+    if (!smem_optin(k_attn_simt<float>, (int)sh)) return;
     k_attn_simt<float><<<grid, 256, sh, st>>>((const float*)q, (const float*)k, (const float*)v, ldq,
                                               ldk, ldv, (float*)o, ldo, T, H, Hkv, window, scale);
   }

@@ -12,7 +12,10 @@
 #include <cmath>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "nc_internal.cuh"
 
@@ -56,6 +59,53 @@ void launch_end(int kind, cudaStream_t st) {
 
 static void set_err(const char* where, cudaError_t e) {
   snprintf(t_err, sizeof(t_err), "%s: %s", where, cudaGetErrorString(e));
+}
+
+void record_error(const char* where, cudaError_t e) { set_err(where, e); }
+
+void reset_launch_count() { t_launches = 0; }
+
+int check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_err(what, e);
+    return NC_ERR_CUDA;
+  }
+  return NC_OK;
+}
+
+namespace {
+std::atomic<unsigned long long> g_flag_wait_ns{kWaitLimitNs};
+std::atomic<unsigned> g_flag_skew{0};
+}  // namespace
+
+void flag_wait_test(unsigned long long* limit_ns, unsigned* skew) {
+  *limit_ns = g_flag_wait_ns.load();
+  *skew = g_flag_skew.load();
+}
+
+namespace {
+std::mutex g_optin_mu;
+std::set<std::pair<const void*, int>> g_optin_done;  // (kernel, device) pairs already raised
+}  // namespace
+
+bool smem_optin(const void* kernel, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    set_err("cudaGetDevice", e);
+    return false;
+  }
+  std::lock_guard<std::mutex> lk(g_optin_mu);
+  const std::pair<const void*, int> key(kernel, dev);
+  if (g_optin_done.count(key)) return true;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) {
+    set_err("cudaFuncSetAttribute", e);
+    return false;
+  }
+  g_optin_done.insert(key);
+  return true;
 }
 
 namespace {
@@ -110,7 +160,7 @@ size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 constexpr int kStreamKPairs = 96;
 
 struct Layout {
-  size_t x, x0, xbo, xn, qkv, o, h, gate, ss, rcos, rsin, rfreq, ce_sum, ce_tgt, logits, tok, tgt, loss;
+  size_t x, x0, xbo, xn, qkv, o, h, gate, ss, rcos, rsin, rfreq, ce_sum, ce_tgt, lse, logits, tok, tgt, loss;
   size_t skws, skflags;
   size_t total;
   int ce_tiles;
@@ -158,6 +208,7 @@ Layout layout(const nc_config& c, int max_tokens) {
   L.ce_tiles = 2 * ((c.vocab_padded + 127) / 128);  // per (row, 128-or-256-column tile, half)
   L.ce_sum = take(M * L.ce_tiles * 4);
   L.ce_tgt = take(M * 4);
+  L.lse = take(M * 4);
   const bool simt_head = c.dtype == NC_FP32 || c.gemm_impl != 0;
   L.logits = take(simt_head ? M * (size_t)c.vocab * 4 : 0);
   // stream-K partial sums of the tcgen05 pair GEMM: one 128 x 256 fp32 tile
@@ -192,15 +243,6 @@ EpiParams epi(int mode) {
   memset(&e, 0, sizeof(e));
   e.mode = mode;
   return e;
-}
-
-int check_launch(const char* what) {
-  const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    set_err(what, e);
-    return NC_ERR_CUDA;
-  }
-  return NC_OK;
 }
 
 }  // namespace
@@ -460,7 +502,8 @@ int forward_impl(const nc_params* p, const int32_t* tokens, const int32_t* targe
     e.ce_tgt = at<float>(ws, Lw.ce_tgt);
     e.ce_tiles = tiles;
     if (!gemm(c, d, xn, C, p->lm_head, C, M, c.vocab_padded, C, e, st)) return NC_ERR_CUDA;
-    launch_ce_combine(e.ce_sum, e.ce_tgt, tiles, c.softcap, targets, M, V, out_loss, d.status, st);
+    launch_ce_combine(e.ce_sum, e.ce_tgt, tiles, c.softcap, targets, M, V, out_loss, at<float>(ws, Lw.lse), d.status,
+                      st);
   } else {
     launch_rmsnorm(x, xn, M, C, c.eps, bf, nullptr, 0, 0, 0.f, nullptr, st);
     float* logits = out_logits ? out_logits : at<float>(ws, Lw.logits);
@@ -543,6 +586,74 @@ int nc_forward_host(const nc_params* p, const int32_t* h_tokens, const int32_t* 
   return NC_OK;
 }
 
+size_t nc_head_backward_workspace_bytes(const nc_config* cfg, int max_tokens) {
+  if (cfg == nullptr || max_tokens <= 0 || !config_ok(*cfg)) return 0;
+  const size_t M = (size_t)max_tokens;
+  return align256(M * (size_t)cfg->vocab_padded * 2) + align256(M * (size_t)cfg->n_embd * 4) + 256;
+}
+
+int nc_head_backward(const nc_params* p, const int32_t* targets, int B, int T, float* out_dx, float* out_dw,
+                     void* bwd_workspace, size_t bwd_workspace_bytes, void* stream) {
+  t_launches = 0;
+  if (p == nullptr || targets == nullptr || out_dx == nullptr || out_dw == nullptr) return NC_ERR_ARG;
+  const nc_config& c = p->cfg;
+  if (!config_ok(c)) return NC_ERR_SHAPE;
+  if (c.dtype != NC_BF16 || c.gemm_impl != 0 || c.vocab_padded % 128 != 0) return NC_ERR_SHAPE;
+  if (B <= 0 || T <= 0 || T > c.max_T || (long long)B * T > (long long)p->max_tokens) return NC_ERR_SHAPE;
+  if (!aligned16(targets) || !aligned16(out_dx) || !aligned16(out_dw) || !aligned16(p->lm_head) ||
+      !aligned16(bwd_workspace) || !aligned16(p->workspace))
+    return NC_ERR_ALIGN;
+  const Layout Lw = layout(c, p->max_tokens);
+  if (p->workspace == nullptr || p->workspace_bytes < Lw.total) return NC_ERR_WORKSPACE;
+  const size_t need = nc_head_backward_workspace_bytes(&c, p->max_tokens);
+  if (bwd_workspace == nullptr || bwd_workspace_bytes < need) return NC_ERR_WORKSPACE;
+  DevInfo d;
+  if (!dev_info(&d)) return NC_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int M = B * T, C = c.n_embd, V = c.vocab, Vp = c.vocab_padded;
+  void* ws = p->workspace;
+  char* bw = static_cast<char*>(bwd_workspace);
+  bf16* dz = reinterpret_cast<bf16*>(bw);                                  // [M, Vp] bf16, rows scaled by 1/rms
+  float* g = reinterpret_cast<float*>(bw + align256((size_t)p->max_tokens * Vp * 2));  // [M, C]
+  float* inv_count = reinterpret_cast<float*>(bw + align256((size_t)p->max_tokens * Vp * 2) +
+                                              align256((size_t)p->max_tokens * C * 4));
+  const bf16* xb = at<bf16>(ws, Lw.xn);        // bf16(x) of the final residual, the head's A operand
+  const float* x = at<float>(ws, Lw.x);        // the final residual (after backout), fp32
+  const float* ss = at<float>(ws, Lw.ss);      // its row sums of squares, per column group
+  const int ss_parts = C / (gemm_tc_bn(C) / 2);
+  launch_inv_count(targets, M, inv_count, st);
+  // dz' = (1/rms) dL/dz: the head GEMM recomputed, the CE gradient in its epilogue
+  EpiParams e = epi(EPI_DZ);
+  e.ss_in = ss;
+  e.ss_in_parts = ss_parts;
+  e.inv_c = 1.0f / (float)C;
+  e.eps = c.eps;
+  e.cap = c.softcap;
+  e.vocab = V;
+  e.targets = targets;
+  e.lse = at<float>(ws, Lw.lse);
+  e.inv_count = inv_count;
+  e.out = dz;
+  e.ldo = Vp;
+  if (!launch_gemm_tc_layout(xb, C, 0, static_cast<const bf16*>(p->lm_head), C, 0, M, Vp, C, e, d.status, d.num_sms,
+                             st))
+    return NC_ERR_CUDA;
+  // g = dz' W_U = (1/rms) dL/dxn; then dx = g - x r^2 (x . g) / C
+  e = epi(EPI_F32);
+  e.out = g;
+  e.ldo = C;
+  if (!launch_gemm_tc_layout(dz, Vp, 0, static_cast<const bf16*>(p->lm_head), C, 1, M, C, Vp, e, d.status, d.num_sms,
+                             st))
+    return NC_ERR_CUDA;
+  launch_rmsnorm_bwd(x, g, out_dx, M, C, c.eps, st);
+  // dW_U = dz'^T bf16(x) = dL/dz^T xn
+  e = epi(EPI_F32);
+  e.out = out_dw;
+  e.ldo = C;
+  if (!launch_gemm_tc_layout(dz, Vp, 1, xb, C, 1, V, C, M, e, d.status, d.num_sms, st)) return NC_ERR_CUDA;
+  return check_launch("nc_head_backward");
+}
+
 int nc_loss_mean(const float* loss, const int32_t* targets, int n, float* out_mean, void* stream) {
   if (loss == nullptr || targets == nullptr || out_mean == nullptr || n < 0) return NC_ERR_ARG;
   launch_loss_mean(loss, targets, n, out_mean, static_cast<cudaStream_t>(stream));
@@ -601,6 +712,39 @@ int nc_attention(const void* q, const void* k, const void* v, void* out, int B, 
   return check_launch("nc_attention");
 }
 
+size_t nc_routing_attention_workspace_bytes(int B, int T, int H, int D) {
+  if (B <= 0 || T <= 0 || H <= 0 || D <= 0) return 0;
+  return align256((size_t)B * T * H * D * 2);
+}
+
+int nc_routing_attention(const void* q2, const void* k2, const void* v2, const void* q1, const void* k1, void* out,
+                         int B, int T, int H, int Hkv, int D, int window, float gate_logit, float softmax_scale,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  t_launches = 0;
+  if (!q2 || !k2 || !v2 || !q1 || !k1 || !out) return NC_ERR_ARG;
+  if (!(softmax_scale > 0.f) || !std::isfinite(gate_logit)) return NC_ERR_ARG;
+  if (B <= 0 || T <= 0 || H <= 0 || Hkv <= 0 || D != 128 || H % Hkv != 0) return NC_ERR_SHAPE;
+  if (!aligned16(q2) || !aligned16(k2) || !aligned16(v2) || !aligned16(q1) || !aligned16(k1) || !aligned16(out) ||
+      !aligned16(workspace))
+    return NC_ERR_ALIGN;
+  if (workspace == nullptr || workspace_bytes < nc_routing_attention_workspace_bytes(B, T, H, D))
+    return NC_ERR_WORKSPACE;
+  DevInfo d;
+  if (!dev_info(&d)) return NC_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // g = softplus(gate_logit), evaluated without overflow
+  const double a = gate_logit;
+  const float g = (float)(a > 0 ? a + log1p(exp(-a)) : log1p(exp(a)));
+  bf16* q1s = static_cast<bf16*>(workspace);
+  launch_scale_bf16(static_cast<const bf16*>(q1), q1s, (long long)B * T * H * D, g, d.num_sms, st);
+  const int w = (window <= 0 || window >= T) ? T : window;
+  if (!launch_attn_route_tc(static_cast<const bf16*>(q2), static_cast<const bf16*>(k2), static_cast<const bf16*>(v2),
+                            q1s, static_cast<const bf16*>(k1), static_cast<bf16*>(out), B, T, H, Hkv, w,
+                            softmax_scale, d.status, d.num_sms, st))
+    return check_launch("nc_routing_attention") == NC_OK ? NC_ERR_CUDA : NC_ERR_CUDA;
+  return check_launch("nc_routing_attention");
+}
+
 int nc_get_status(void* stream, int* out_bits) {
   DevInfo d;
   if (!dev_info(&d)) return NC_ERR_CUDA;
@@ -638,6 +782,13 @@ const char* nc_last_error(void) { return t_err; }
 
 int nc_last_launch_count(void) { return t_launches; }
 
+int nc_set_flag_wait_test(int skew, double wait_limit_ms) {
+  if (skew < 0 || !(wait_limit_ms > 0.0) || wait_limit_ms > 1000.0) return NC_ERR_ARG;
+  g_flag_wait_ns.store((unsigned long long)(wait_limit_ms * 1e6));
+  g_flag_skew.store((unsigned)skew);
+  return NC_OK;
+}
+
 int nc_set_launch_timing(void** events, int* kinds, int capacity, unsigned kind_mask) {
   if (events != nullptr && (kinds == nullptr || capacity <= 0)) return NC_ERR_ARG;
   t_timing = Timing();
@@ -654,7 +805,7 @@ const char* nc_kernel_name(int kind) {
   static const char* names[KK_COUNT] = {
       "embed_norm_smear", "rmsnorm", "rope_table", "rope_qknorm", "gemm_tcgen05", "gemm_cuda_core",
       "attention_tcgen05", "attention_cuda_core", "ce_combine", "ce_rows", "loss_mean", "last_logits",
-      "sample"};
+      "sample", "gemm_tcgen05_bwd", "head_bwd_rows"};
   return (kind >= 0 && kind < KK_COUNT) ? names[kind] : "unknown";
 }
 

@@ -54,7 +54,9 @@ enum EpiMode : int {
   EPI_BLOCK_END = 3, // x += acc; capture x_bo; then re-inject for the next block or apply backout
   EPI_SOFTCAP = 4,   // logits[m, n] = cap tanh(acc / cap)    (fp32; CUDA-core path)
   EPI_CE = 5,        // softcap + per-(row, tile) log-sum-exp partials (+ optional logits)
-  EPI_QKV = 6        // q, k heads: RoPE + QK-norm; v heads: + gate * VE[tok]; bf16 out (tcgen05 path)
+  EPI_QKV = 6,       // q, k heads: RoPE + QK-norm; v heads: + gate * VE[tok]; bf16 out (tcgen05 path)
+  EPI_DZ = 7,        // head backward: d loss / d z of the softcapped CE, times 1/rms of the row, bf16 out
+  EPI_F32 = 8        // out[m, n] = acc (fp32)
 };
 
 struct EpiParams {
@@ -104,6 +106,12 @@ struct EpiParams {
   const float* ss_in;
   int ss_in_parts;
   float inv_c;        // 1 / C
+  // EPI_DZ (A = bf16(x), rows scaled by 1 / rms through ss_in as for EPI_CE;
+  // targets, vocab and cap as for EPI_CE): with zhat = cap tanh(z / cap),
+  //   out[m, n] = bf16( rscale_m * inv_count * (exp(zhat - lse[m]) - [n == y_m]) * (1 - (zhat / cap)^2) )
+  // for rows with a valid target and n < vocab, 0 elsewhere
+  const float* lse;        // [M] log-sum-exp of the row's softcapped logits
+  const float* inv_count;  // device scalar: 1 / (number of valid targets), 0 if none
   // value-embedding gate inside the QKV epilogue (when gate == NULL):
   // g = gate_scale * sigmoid(rstd * x[m, :gate_c] . gate_w[h, :gate_c])
   const float* gate_w;
@@ -131,7 +139,15 @@ void launch_rope_qknorm_copy(const void* q, const void* k, void* qo, void* ko, i
 void launch_ce_rows(const float* logits, int ldl, const int32_t* targets, int M, int V, float* loss,
                     int* status, cudaStream_t st);
 void launch_ce_combine(const float* ce_sum, const float* ce_tgt, int n_tiles, float offset,
-                       const int32_t* targets, int M, int V, float* loss, int* status, cudaStream_t st);
+                       const int32_t* targets, int M, int V, float* loss, float* lse, int* status,
+                       cudaStream_t st);
+// head backward helpers: 1 / (number of targets != -1) into *inv_count, and
+// the RMSNorm backward dx = g - x r^2 (x . g) / C with r = 1 / rms(x) per row
+// (g = r * dL/dxn, fp32 [M, C])
+void launch_inv_count(const int32_t* targets, int n, float* inv_count, cudaStream_t st);
+// out = bf16(g * in), n a multiple of 8 elements, 16-byte aligned buffers
+void launch_scale_bf16(const bf16* in, bf16* out, long long n, float g, int num_sms, cudaStream_t st);
+void launch_rmsnorm_bwd(const float* x, const float* g, float* dx, int M, int C, float eps, cudaStream_t st);
 void launch_loss_mean(const float* loss, const int32_t* targets, int n, float* out, cudaStream_t st);
 // generation: softcapped logits of the last position of each of B rows
 // (x: the final fp32 residual [B T, ldx]; W: lm_head [V_padded, C], bf16 or
@@ -165,15 +181,50 @@ struct StreamK {
 bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int N, int K,
                     const EpiParams& ep, int* status, int num_sms, cudaStream_t st, bool pair,
                     const StreamK* sk = nullptr);
+// tcgen05 GEMM with operands in either layout, single-CTA kernel (bf16):
+// C[M, N] = A[M, K] B[N, K]^T where A is stored row-major [M, lda] when
+// a_mn == 0 (K contiguous) or as its transpose [K, lda] when a_mn == 1 (M
+// contiguous), likewise B ([N, ldb] or [K, ldb]).  K need not be a multiple
+// of 64 (out-of-range k reads zeros).  Used by the head backward.
+bool launch_gemm_tc_layout(const bf16* A, int lda, int a_mn, const bf16* Bm, int ldb, int b_mn, int M, int N,
+                           int K, const EpiParams& ep, int* status, int num_sms, cudaStream_t st);
 // tcgen05 attention (bf16 only)
+// pass-2 routing attention: logits scale (q2 . k2 + q1s . k1) with q1s = g q1
+// already scaled; all inputs [B, T, heads, 128] contiguous, o [B, T, H, 128]
+bool launch_attn_route_tc(const bf16* q2, const bf16* k2, const bf16* v2, const bf16* q1s, const bf16* k1, bf16* o,
+                          int B, int T, int H, int Hkv, int window, float scale, int* status, int num_sms,
+                          cudaStream_t st);
 bool launch_attn_tc(const bf16* q, const bf16* k, const bf16* v, int ldq, int ldk, int ldv, bf16* o,
                     int ldo, int B, int T, int H, int Hkv, int window, float scale, int* status,
                     int num_sms, cudaStream_t st);
 
+// Raise `kernel`'s dynamic shared-memory limit to `bytes` on the current
+// device.  The attribute belongs to the device's context, so it is set once
+// per (kernel, device): a process that drives several devices sets it on
+// each.  Returns false, with the CUDA error recorded for nc_last_error(),
+// when the device cannot be queried or the attribute cannot be set.
+bool smem_optin(const void* kernel, int bytes);
+template <typename... KArgs>
+bool smem_optin(void (*kernel)(KArgs...), int bytes) {
+  return smem_optin(reinterpret_cast<const void*>(kernel), bytes);
+}
+// Settings of nc_set_flag_wait_test(): the limit (ns) of the split-K
+// partial-sum flag wait and the generation offset that wait expects (0 in
+// normal operation; non-zero makes the flags it waits for never arrive).
+void flag_wait_test(unsigned long long* limit_ns, unsigned* skew);
+// Record a CUDA error for nc_last_error() (this host thread).
+void record_error(const char* where, cudaError_t e);
+// Start a new launch count for nc_last_launch_count() (this host thread).
+void reset_launch_count();
+// NC_OK, or NC_ERR_CUDA with the error recorded, after the launches of an
+// entry point (cudaGetLastError).
+int check_launch(const char* what);
+
 // Kernel kinds, for the launch counter and the optional per-launch timing.
 enum KernelKind : int {
   KK_EMBED = 0, KK_RMSNORM, KK_ROPE_TABLE, KK_ROPE_QKNORM, KK_GEMM_TC, KK_GEMM_SIMT, KK_ATTN_TC,
-  KK_ATTN_SIMT, KK_CE_COMBINE, KK_CE_ROWS, KK_LOSS_MEAN, KK_LAST_LOGITS, KK_SAMPLE, KK_COUNT
+  KK_ATTN_SIMT, KK_CE_COMBINE, KK_CE_ROWS, KK_LOSS_MEAN, KK_LAST_LOGITS, KK_SAMPLE, KK_GEMM_TC_BWD,
+  KK_HEAD_BWD_ROWS, KK_COUNT
 };
 // Every launcher holds one of these around its kernel launch: it counts the
 // launch (per host thread) and, when the caller enabled timing for this kind,

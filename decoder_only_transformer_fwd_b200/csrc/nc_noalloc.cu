@@ -24,12 +24,18 @@ std::mutex g_scratch_mu;
 bool scratch_on_current_device(unsigned char** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    record_error("nc_attention_noalloc: cudaGetDevice", e != cudaSuccess ? e : cudaErrorInvalidDevice);
+    return false;
+  }
   std::lock_guard<std::mutex> lk(g_scratch_mu);
   if (!g_scratch_ready[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr) return false;
+    if (e != cudaSuccess || p == nullptr) {
+      record_error("nc_attention_noalloc: cudaGetSymbolAddress", e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+      return false;
+    }
     g_scratch_ptr[dev] = static_cast<unsigned char*>(p);
     g_scratch_ready[dev] = true;
   }
@@ -53,6 +59,7 @@ extern "C" size_t nc_attention_noalloc_max_bytes(void) { return kScratchBytes; }
 extern "C" int nc_attention_noalloc(const void* q, const void* k, const void* v, void* out, int B, int T, int H,
                                     int Hkv, int D, int window, float alpha, float softmax_scale,
                                     float rope_base, float eps, int dtype, void* stream) {
+  reset_launch_count();
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return NC_ERR_ARG;
   if (dtype != NC_BF16 && dtype != NC_FP32) return NC_ERR_ARG;
   if (!(softmax_scale > 0.f) || !(eps >= 0.f)) return NC_ERR_ARG;
@@ -72,9 +79,12 @@ extern "C" int nc_attention_noalloc(const void* q, const void* k, const void* v,
   int* status = nullptr;
   if (!status_word(&status)) return NC_ERR_CUDA;
   int sms = 0, dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) {
+    record_error("nc_attention_noalloc: device query", e);
     return NC_ERR_CUDA;
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* rc = reinterpret_cast<float*>(base);
   float* rs = reinterpret_cast<float*>(base + tab);
@@ -87,10 +97,12 @@ extern "C" int nc_attention_noalloc(const void* q, const void* k, const void* v,
   launch_rope_qknorm_copy(q, k, qo, ko, B, T, H, Hkv, D, rc, rs, alpha, eps, bf, st);
   if (bf) {
     if (!launch_attn_tc((const bf16*)qo, (const bf16*)ko, (const bf16*)v, H * D, Hkv * D, Hkv * D, (bf16*)out,
-                        H * D, B, T, H, Hkv, w, softmax_scale, status, sms, st))
+                        H * D, B, T, H, Hkv, w, softmax_scale, status, sms, st)) {
+      check_launch("nc_attention_noalloc");
       return NC_ERR_CUDA;
+    }
   } else {
     launch_attn_simt(qo, ko, v, H * D, Hkv * D, Hkv * D, out, H * D, B, T, H, Hkv, w, softmax_scale, bf, st);
   }
-  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+  return check_launch("nc_attention_noalloc");
 }

@@ -82,11 +82,18 @@ _SIGS = {
                                        C.c_int, C.c_int, C.c_int, C.c_int, C.c_float, C.c_float, C.c_float,
                                        C.c_float, C.c_int, C.c_void_p]),
     "nc_attention_noalloc_max_bytes": (C.c_size_t, []),
+    "nc_set_flag_wait_test": (C.c_int, [C.c_int, C.c_double]),
+    "nc_routing_attention_workspace_bytes": (C.c_size_t, [C.c_int] * 4),
+    "nc_routing_attention": (C.c_int, [C.c_void_p] * 6 + [C.c_int] * 6 + [C.c_float, C.c_float, C.c_void_p,
+                                                                         C.c_size_t, C.c_void_p]),
+    "nc_head_backward_workspace_bytes": (C.c_size_t, [C.POINTER(nc_config), C.c_int]),
+    "nc_head_backward": (C.c_int, [C.POINTER(nc_params), C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p,
+                                   C.c_void_p, C.c_size_t, C.c_void_p]),
 }
 
 KERNEL_KINDS = ["embed_norm_smear", "rmsnorm", "rope_table", "rope_qknorm", "gemm_tcgen05",
                 "gemm_cuda_core", "attention_tcgen05", "attention_cuda_core", "ce_combine", "ce_rows",
-                "loss_mean", "last_logits", "sample"]
+                "loss_mean", "last_logits", "sample", "gemm_tcgen05_bwd", "head_bwd_rows"]
 
 
 class LaunchTimer:
@@ -218,6 +225,19 @@ def nc_forward_host(params: nc_params, tokens: np.ndarray, targets: np.ndarray, 
                                  _stream(stream)), "nc_forward_host")
 
 
+def nc_head_backward_workspace_bytes(cfg: nc_config, max_tokens: int) -> int:
+    return int(lib().nc_head_backward_workspace_bytes(C.byref(cfg), max_tokens))
+
+
+def nc_head_backward(params: nc_params, targets, out_dx, out_dw, workspace, stream=None):
+    """dL/dx [B*T, C] and dL/dW_U [V, C] (fp32 device tensors) of the mean CE,
+    right after nc_forward on the same params and targets [B, T]."""
+    B, T = targets.shape
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().nc_head_backward(C.byref(params), _ptr(targets), B, T, _ptr(out_dx), _ptr(out_dw), _ptr(workspace),
+                                  nbytes, _stream(stream)), "nc_head_backward")
+
+
 def nc_loss_mean(loss, targets, out_mean, stream=None):
     _check(lib().nc_loss_mean(_ptr(loss), _ptr(targets), loss.numel(), _ptr(out_mean),
                               _stream(stream)), "nc_loss_mean")
@@ -242,6 +262,22 @@ def nc_attention(q, k, v, out, window: int, rope_qknorm: int = 1, alpha: float =
                               nbytes, _stream(stream)), "nc_attention")
 
 
+def nc_routing_attention(q2, k2, v2, q1, k1, out, window: int, gate_logit: float,
+                         softmax_scale: float | None = None, workspace=None, stream=None):
+    """Pass-2 routing attention (bf16 device tensors [B, T, heads, 128])."""
+    import torch
+    B, T, H, D = q2.shape
+    Hkv = k2.shape[2]
+    scale = D ** -0.5 if softmax_scale is None else softmax_scale
+    if workspace is None:
+        workspace = torch.empty(int(lib().nc_routing_attention_workspace_bytes(B, T, H, D)), dtype=torch.uint8,
+                                device=q2.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().nc_routing_attention(_ptr(q2), _ptr(k2), _ptr(v2), _ptr(q1), _ptr(k1), _ptr(out), B, T, H, Hkv, D,
+                                      window, gate_logit, scale, _ptr(workspace), nbytes, _stream(stream)),
+           "nc_routing_attention")
+
+
 def nc_get_status(stream=None) -> tuple[int, int]:
     bits = C.c_int(0)
     rc = lib().nc_get_status(_stream(stream), C.byref(bits))
@@ -250,6 +286,10 @@ def nc_get_status(stream=None) -> tuple[int, int]:
 
 def nc_last_launch_count() -> int:
     return int(lib().nc_last_launch_count())
+
+
+def nc_set_flag_wait_test(skew: int, wait_limit_ms: float):
+    _check(lib().nc_set_flag_wait_test(int(skew), float(wait_limit_ms)), "nc_set_flag_wait_test")
 
 
 # --------------------------------------------------------------------------

@@ -182,6 +182,35 @@ int nc_generate_next(const nc_params* p, const int32_t* tokens, int B, int T, fl
                      int top_k, const float* uniforms, int32_t* out_next, float* out_logits,
                      void* stream);
 
+/* Bytes of the extra workspace nc_head_backward() needs for up to
+ * max_tokens tokens: the per-token gradient of the logits in bf16
+ * ([max_tokens, V_pad], 64 MiB per 1024 tokens at V = 32768) and one fp32
+ * [max_tokens, C] buffer.  Host function; 0 on invalid config. */
+size_t nc_head_backward_workspace_bytes(const nc_config* cfg, int max_tokens);
+
+/* Backward pass of the head: the gradients of the mean cross-entropy
+ * L = (1/|T|) sum_{t in T} (logsumexp(zhat_t) - zhat_t[y_t]), T = {t : y_t != -1},
+ * with respect to the final residual stream and to the unembedding matrix
+ * ("The Mathematics of Karpathy's nanochat", §Cross-Entropy Loss, §Logit
+ * Softcap with d zhat/d z = 1 - tanh^2(z/15), §RMS Normalization; the chain
+ * rule through these steps in reverse order):
+ *   out_dx [B*T, C] fp32: dL/dx, x the final residual after backout (the
+ *     input of the final RMSNorm);
+ *   out_dw [V, C] fp32: dL/dW_U (rows V..V_pad-1 are not written).
+ * It consumes what the forward pass left in p->workspace (bf16(x), the row
+ * sums of squares of x, x itself and the per-row log-sum-exp), so it must
+ * follow nc_forward(p, tokens, targets, B, T, ...) on the same stream with the
+ * same p, B, T and targets, with no other call using that workspace in
+ * between.  The logits are recomputed (one more head GEMM) and their gradient
+ * is held in bf16 in bwd_workspace (>= nc_head_backward_workspace_bytes).
+ * Then dL/dxn = dL/dz W_U and dL/dW_U = dL/dz^T xn run as tensor-core GEMMs
+ * (xn in bf16 as the forward's head consumed it), and the RMSNorm backward
+ * gives dL/dx.  With no valid target both gradients are 0.  bf16 mode with
+ * tensor-core GEMMs only (NC_ERR_SHAPE otherwise); requirements and status
+ * codes as nc_forward, NC_ERR_WORKSPACE for a missing or short bwd_workspace. */
+int nc_head_backward(const nc_params* p, const int32_t* targets, int B, int T, float* out_dx, float* out_dw,
+                     void* bwd_workspace, size_t bwd_workspace_bytes, void* stream);
+
 /* Mean of loss[i] over i with targets[i] != -1 ([Math] §Cross-Entropy Loss),
  * written to *out_mean (device fp32); NaN when no target is valid.  n >= 0. */
 int nc_loss_mean(const float* loss, const int32_t* targets, int n, float* out_mean, void* stream);
@@ -233,6 +262,27 @@ int nc_attention_noalloc(const void* q, const void* k, const void* v, void* out,
 /* Size in bytes of nc_attention_noalloc's fixed scratch array. */
 size_t nc_attention_noalloc_max_bytes(void);
 
+/* Pass-2 attention of the looped ("routing") variant ("looped-nanochat-d24"
+ * model card, What is the routing loop?): every pass-2 layer adds a causal
+ * attention-logit prior from a pass-1 layer,
+ *   logits_ij = softmax_scale * (q2_i . k2_j + g q1_i . k1_j),  g = softplus(gate_logit),
+ * over the base model's visible keys (j <= i, i - j < window; window <= 0 or
+ * >= T means plain causal), then o_i = sum_j softmax_j(logits_ij) v2_j.
+ *   q2, q1 [B, T, H, D] and k2, k1, v2 [B, T, H_kv, D], bf16, contiguous: q and
+ *     k are the features as they enter the attention (after RoPE and QK-norm
+ *     of their pass); query head h reads k/v head h / (H / H_kv);
+ *   out [B, T, H, D] bf16.
+ * As on the card, the prior never forms a T x T matrix: it is one QK^T over
+ * the augmented width [q2 | g q1] . [k2 | k1] on the tensor cores.  g q1 is
+ * written (bf16) to `workspace` (>= nc_routing_attention_workspace_bytes).
+ * bf16 only; D == 128, H % H_kv == 0, softmax_scale > 0, finite gate_logit,
+ * 16-byte aligned pointers (NC_ERR_SHAPE / NC_ERR_ARG / NC_ERR_ALIGN /
+ * NC_ERR_WORKSPACE otherwise). */
+size_t nc_routing_attention_workspace_bytes(int B, int T, int H, int D);
+int nc_routing_attention(const void* q2, const void* k2, const void* v2, const void* q1, const void* k1, void* out,
+                         int B, int T, int H, int Hkv, int D, int window, float gate_logit, float softmax_scale,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
 /* Synchronise `stream`, read the device status word (an OR of
  * 1 << NC_ERR_DATA and 1 << NC_ERR_TIMEOUT bits set by kernels since the last
  * read), clear it, and return NC_OK, NC_ERR_DATA or NC_ERR_TIMEOUT (timeout
@@ -248,6 +298,19 @@ const char* nc_last_error(void);
 /* Number of kernel launches issued by the last nc_forward() / nc_attention()
  * on this thread. */
 int nc_last_launch_count(void);
+
+/* Test hook for the device-side timeout path (process-wide; not for normal
+ * use).  With gemm_pair == 2 the MLP down-projection's partial last wave of
+ * tiles is split over CTA pairs, and the pair that finishes a tile waits for
+ * its contributors' flags (a generation number per launch).  With skew != 0
+ * that wait expects generation + skew, which never arrives: after
+ * wait_limit_ms the kernel records NC_ERR_TIMEOUT in the status word, skips
+ * the wait and completes (its output is then not the model's).  wait_limit_ms
+ * bounds that wait in every case (default 1000; nc_set_flag_wait_test(0,
+ * 1000) restores normal operation).  Waits on in-flight copies and MMAs keep
+ * their own one-second limit.  NC_ERR_ARG for skew < 0 or a limit outside
+ * (0, 1000] ms.  There is no counterpart on the pages. */
+int nc_set_flag_wait_test(int skew, double wait_limit_ms);
 
 /* Optional per-launch device timing for profiling.  `events` is an array of
  * 2 * capacity cudaEvent_t created by the caller (passed as void*), `kinds`

@@ -226,3 +226,37 @@ def test_flop_accounting_matches_pages():
     # brute force of the closed form
     for T, wd in [(7, 3), (10, 10), (5, 9)]:
         assert abs(flops.mean_visible_keys(T, wd) - sum(min(i + 1, wd) for i in range(T)) / T) < 1e-12
+
+
+def test_flag_wait_test_hook_argument_checks():
+    lib = nc.lib()
+    assert lib.nc_set_flag_wait_test(-1, 10.0) == nc.STATUS_CODES["NC_ERR_ARG"]
+    assert lib.nc_set_flag_wait_test(0, 0.0) == nc.STATUS_CODES["NC_ERR_ARG"]
+    assert lib.nc_set_flag_wait_test(0, 1000.5) == nc.STATUS_CODES["NC_ERR_ARG"]
+    assert lib.nc_set_flag_wait_test(0, 1000.0) == 0   # normal operation
+
+
+def test_head_backward_rejects_bad_arguments_without_launching():
+    lib = nc.lib()
+    buf = (C.c_byte * 4096)()
+    a16 = C.c_void_p((C.addressof(buf) + 15) & ~15)
+    ARG, SHAPE, WS = (nc.STATUS_CODES[k] for k in ("NC_ERR_ARG", "NC_ERR_SHAPE", "NC_ERR_WORKSPACE"))
+    cfg = nc.nc_init_config(4, 256, "bf16", "SSSL", 128)
+    p = nc.nc_params()
+    assert lib.nc_params_init(C.byref(p), C.byref(cfg)) == 0
+    call = lambda **kw: lib.nc_head_backward(C.byref(p), kw.get("y", a16), kw.get("B", 1), kw.get("T", 8),
+                                             kw.get("dx", a16), kw.get("dw", a16), kw.get("ws", a16),
+                                             kw.get("wsb", 16), None)
+    assert call(y=None) == ARG and call(dx=None) == ARG and call(dw=None) == ARG
+    assert call() == SHAPE                      # max_tokens == 0
+    p.max_tokens = 8
+    assert call(T=300) == SHAPE and call(B=0) == SHAPE
+    assert call() == WS                         # no forward workspace
+    need = lib.nc_head_backward_workspace_bytes(C.byref(cfg), 8)
+    assert need >= 8 * cfg.vocab_padded * 2 + 8 * cfg.n_embd * 4
+    p.cfg.gemm_impl = 1                         # tensor-core path only
+    assert call() == SHAPE
+    cfg32 = nc.nc_init_config(4, 256, "fp32", "SSSL", 128)
+    assert lib.nc_params_init(C.byref(p), C.byref(cfg32)) == 0
+    p.max_tokens = 8
+    assert call() == SHAPE                      # bf16 mode only

@@ -1,74 +1,53 @@
-"""Evidence for the bf16-mode loss tolerance.
+"""Evidence for how the bf16-mode tolerances are applied.
 
-The bf16 path rounds to bf16 exactly at the GEMM operands and stored
-activations: the normalised block inputs, q and k after RoPE + QK-norm and v
-after the value-embedding mix (all three applied to the fp32 accumulator of
-the QKV GEMM), the attention output, the ReLU^2 output and the head input; everything else (the residual stream,
-accumulation, softmax, softcap, log-sum-exp) stays in fp32 or better.  This
-test applies those roundings to the oracle's own fp64 steps and measures the
-per-token loss error they cause: its rms sets the bound the GPU parity tests
-use (rms <= 6e-3), and it is large enough that a bound on the maximum of 1e-2
-over thousands of tokens (about 3.5 sigma) could not hold for any bf16
-implementation.  Rounding is the only difference between the two runs here.
+bf16_emulation.py applies the bf16 roundings of the tensor-core path (GEMM A
+operands, q/k/v, the softmax weights entering P V, the attention output, the
+ReLU^2 output) to the oracle's own fp64 steps; rounding is the only
+difference between the two runs.  These tests pin what that rounding alone
+does on the seeded random-init workloads:
+  * the per-token loss error is about 4e-3 rms, unbiased;
+  * its tails pass the stated per-value tolerances: the logit error exceeds
+    3e-2 on seeded cases (on about one logit in ten million), and the loss
+    error exceeds 1e-2 on one to three percent of the tokens of every case.
+So no implementation that rounds at these points can hold 1e-2 and 3e-2 as
+maxima; bf16_parity.py holds the GPU to the emulation's error on the same
+inputs instead.
 """
 import numpy as np
+import pytest
 
+import bf16_emulation as E
 from decoder_only_transformer_fwd_b200 import synth
 from oracle import nanochat_fwd as O
 
-F64 = np.float64
 
-
-def _rb(a):
-    return synth.round_bf16(np.asarray(a, np.float32)).astype(F64)
-
-
-def _forward_rounded(cfg, p, tok, y):
-    T = tok.shape[0]
-    H, D, eps = cfg["n_head"], cfg["head_dim"], cfg["eps"]
-    x = O.embed(cfg, p, tok)
-    x0 = x.copy()
-    x_bo = None
-    pos = np.arange(T)
-    for l in range(cfg["n_layer"]):
-        lp = p["layers"][l]
-        x = p["resid_lambdas"][l] * x + p["x0_lambdas"][l] * x0
-        a = O.rmsnorm(x, eps)
-        qkv = _rb(a) @ np.asarray(lp["w_qkv"], F64).T
-        q = qkv[:, :H * D].reshape(T, H, D)
-        k = qkv[:, H * D:2 * H * D].reshape(T, H, D)
-        v = qkv[:, 2 * H * D:].reshape(T, H, D)
-        if lp["ve"] is not None:
-            g = O.ve_gate(a[:, :12], lp["ve_gate"])
-            v = v + g[:, :, None] * np.asarray(lp["ve"], F64)[tok].reshape(T, H, D)
-        v = _rb(v)
-        qh = _rb(O.qk_norm(O.rope(q, pos), cfg["qk_alpha"], eps))
-        kh = _rb(O.qk_norm(O.rope(k, pos), cfg["qk_alpha"], eps))
-        o = _rb(O.attention(qh, kh, v, cfg["windows"][l], cfg["softmax_scale"]))
-        x = x + o.reshape(T, H * D) @ np.asarray(lp["w_o"], F64).T
-        h = _rb(O.relu2(_rb(O.rmsnorm(x, eps)) @ np.asarray(lp["w_fc1"], F64).T))
-        x = x + h @ np.asarray(lp["w_fc2"], F64).T
-        if l == cfg["backout_layer"]:
-            x_bo = x.copy()
-    x = x - float(p["backout_lambda"]) * x_bo
-    z = _rb(O.rmsnorm(x, eps)) @ np.asarray(p["lm_head"][: cfg["vocab"]], F64).T
-    return O.cross_entropy_per_token(O.softcap(z), y)
+def _case(depth, B, T, short, seed, max_T):
+    cfg = O.make_config(depth, max_T, short)
+    p = synth.params(seed, n_layer=depth, n_embd=cfg["n_embd"], n_head=cfg["n_head"],
+                     n_kv_head=cfg["n_kv_head"], head_dim=128, vocab=32768, vocab_padded=32768,
+                     ve_layers=cfg["ve_layers"], bf16=True)
+    return cfg, p, synth.tokens(seed, B, T, 32768), synth.targets(seed, B, T, 32768)
 
 
 def test_bf16_operand_rounding_sets_the_loss_error():
-    depth, T = 4, 512
-    cfg = O.make_config(depth, T, T // 2)
-    p = synth.params(20261, n_layer=depth, n_embd=cfg["n_embd"], n_head=cfg["n_head"],
-                     n_kv_head=cfg["n_kv_head"], head_dim=128, vocab=32768, vocab_padded=32768,
-                     ve_layers=cfg["ve_layers"], bf16=True)
-    tok = synth.tokens(20261, 1, T, 32768)
-    y = synth.targets(20261, 1, T, 32768)
+    cfg, p, tok, y = _case(4, 1, 512, 256, 20261, 512)
     exact, _ = O.forward(cfg, p, tok, y)
-    rounded = _forward_rounded(cfg, p, tok[0].astype(np.int64), y[0])
-    err = rounded - exact[0]
+    rounded, _ = E.forward(cfg, p, tok, y)
+    err = rounded[0] - exact[0]
     rms = float(np.sqrt(np.mean(err ** 2)))
-    # sigma of the bf16 per-token loss error: well above what a 1e-2 bound on
-    # the max over >= 2048 tokens tolerates (1e-2 / 3.5), inside the 6e-3 bound
-    assert 1e-2 / 3.5 < rms < 6e-3, rms
+    assert 3e-3 < rms < 6e-3, rms
     assert abs(err.mean()) < 1e-3
-    assert np.max(np.abs(err)) < 3e-2
+
+
+@pytest.mark.parametrize("seed", [5004, 5005])
+def test_rounding_alone_exceeds_the_stated_logit_tolerance(seed):
+    """d4, three rows of 200 tokens, short window 64 (the ragged-shape GPU case)."""
+    cfg, p, tok, y = _case(4, 3, 200, 64, seed, 256)
+    ex_l, ex_z = O.forward(cfg, p, tok, y, want_logits=True)
+    em_l, em_z = E.forward(cfg, p, tok, y, want_logits=True)
+    dz = np.abs(em_z - ex_z)
+    assert dz.max() > 3.4e-2
+    assert 0 < np.mean(dz > 3e-2) < 1e-6       # a handful of the 19.7M logits
+    dl = np.abs(em_l - ex_l)
+    assert dl.max() > 1.3e-2
+    assert 0.01 < np.mean(dl > 1e-2) < 0.05     # a few percent of the tokens
