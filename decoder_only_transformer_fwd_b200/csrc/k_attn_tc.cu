@@ -456,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float2 e = ffma2(make_float2(x[32 * qd + 2 * i], x[32 * qd + 2 * i + 1]), c2, mc2);
-            const float2 p = (POLY > 0 && i % POLY == POLY - 1) ? exp2_poly(e) : make_float2(ex2(e.x), ex2(e.y));
+            const float2 p = (POLY > 0 && i % (POLY > 0 ? POLY : 1) == POLY - 1) ? exp2_poly(e) : make_float2(ex2(e.x), ex2(e.y));
             sm[i & 3] = fadd2(sm[i & 3], p);
             pk[i] = pack_bf16(p.x, p.y);
           }
@@ -521,7 +521,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         put(8, o2);
         put(12, o3);
       }
-      if (lane == 0) ptx::mbar_arrive(bar(B_OE + g));
     }
     if (!ok) *abort_flag = 1;
   }

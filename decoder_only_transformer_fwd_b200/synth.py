@@ -95,6 +95,13 @@ def sampling_logits(seed: int, B: int, V: int, cap: float = 15.0, ties: int = 0)
     return z
 
 
+def binade_logits(seed: int, B: int, V: int, lo: float = 1.0) -> np.ndarray:
+    """float32 logits uniform in [lo, 2 lo): every entry shares one sign and
+    exponent, i.e. one binade."""
+    g = _gen(seed, _ID_LOGITS)
+    return (lo * (1.0 + g.random(size=(B, V)))).astype(np.float32)
+
+
 def params(seed: int, *, n_layer: int, n_embd: int, n_head: int, n_kv_head: int,
            head_dim: int, vocab: int, vocab_padded: int, ve_layers, gate_channels: int = 12,
            bf16: bool = True, layers=None) -> dict:

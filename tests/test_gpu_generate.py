@@ -99,6 +99,20 @@ def test_sampling_matches_oracle(V, tau, k, ties):
     assert exact >= B // 2 or V == 1
 
 
+@pytest.mark.parametrize("V,k,lo", [(32768, 50, 1.0), (32768, 16384, 1.0), (32768, 16384, 0.5), (50000, 7, 4.0)])
+def test_top_k_when_one_binade_holds_the_row(V, k, lo):
+    """All logits in one binade put every key in the top digit's bin, far more
+    than the 4096 candidates the select compacts: the lower digits are then
+    counted over the whole row."""
+    B = 8
+    z = synth.binade_logits(3100 + k, B, V, lo)
+    u = synth.uniforms(3100 + k, B)
+    got, rc = _sample(z, 1.0, k, u)
+    assert rc == 0
+    exact = _check_draws(z, 1.0, k, u, got)
+    assert exact >= B // 2
+
+
 def test_top_k_ties_are_all_kept():
     # every row: 5th-largest value repeated 6 times; k = 5 keeps all of them,
     # and a u grid walks through every kept token
