@@ -547,12 +547,28 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
 }
 
 
+// Producers of the fused norm's input (EPI_RESID / EPI_BLOCK_END) store each
+// row's sum of squares per 32-column chunk: slot n / 32 of the row's
+// ss_parts = N / 32 slots (lane (q, 0) holds the sums of rows 4 i + q); ssr
+// is cleared for the next chunk.
+__device__ __forceinline__ void store_chunk_ss(const EpiParams& ep, const TcArgs& a, int row0, int n, int lane,
+                                               float (&ssr)[8]) {
+  if (ep.ss_out != nullptr && (lane & 7) == 0) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int mr = row0 + 4 * i + (lane >> 3);
+      if (mr < a.M) ep.ss_out[(size_t)mr * ep.ss_parts + (n >> 5)] = ssr[i];
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ssr[i] = 0.f;
+}
+
 template <int BN, int MODE>
 __device__ __forceinline__ RowPre epilogue_pre(const EpiParams& ep, const TcArgs& a, int mb, int nb, int g,
-                                               int half, int lane) {
-  constexpr int HALF = BN / 2;
+                                               int c_lo, int lane) {
   const int m = mb * kBM + g * 32 + lane;
-  const int n_lo = nb * BN + half * HALF;
+  const int n_lo = nb * BN + c_lo;
   RowPre p{1.f, 0.f, -1, 0, 0.f};
   if (m >= a.M) return p;
   if constexpr (MODE == EPI_QKV || MODE == EPI_RELU2 || MODE == EPI_CE || MODE == EPI_DZ) {
@@ -599,25 +615,24 @@ __device__ __forceinline__ RowPre epilogue_pre(const EpiParams& ep, const TcArgs
 // tile (mb, nb) will read: called one tile ahead, so the reads hit L2.
 template <int BN, int MODE>
 __device__ __forceinline__ void epilogue_prefetch(const EpiParams& ep, const TcArgs& a, int mb, int nb, int g,
-                                                  int half, int lane) {
-  constexpr int HALF = BN / 2;
+                                                  int c_lo, int c_cnt, int lane) {
   const int m = mb * kBM + g * 32 + lane;
-  const int n_lo = nb * BN + half * HALF;
+  const int n_lo = nb * BN + c_lo;
   if (m >= a.M) return;
   if constexpr (MODE == EPI_RESID || MODE == EPI_BLOCK_END) {
-    // this thread's row of the warp's column half of x (and x0 / x_bo)
-    const int nc = min(HALF, a.N - n_lo);
+    // this thread's row of the warp's columns of x (and x0 / x_bo)
+    const int nc = min(c_cnt, a.N - n_lo);
     if (nc > 0) {
       const char* xr = reinterpret_cast<const char*>(ep.x + (size_t)m * ep.ldx + n_lo);
 #pragma unroll
-      for (int o = 0; o < HALF * 4; o += 128)
+      for (int o = 0; o < (BN / 2) * 4; o += 128)
         if (o < nc * 4) ptx::prefetch_l2(xr + o);
       if (MODE == EPI_BLOCK_END) {
         const float* z = ep.end_kind == 1 ? ep.x0 : ((ep.end_kind == 2 && !ep.capture_bo) ? ep.xbo : nullptr);
         if (z != nullptr) {
           const char* zr = reinterpret_cast<const char*>(z + (size_t)m * ep.ldx + n_lo);
 #pragma unroll
-          for (int o = 0; o < HALF * 4; o += 128)
+          for (int o = 0; o < (BN / 2) * 4; o += 128)
             if (o < nc * 4) ptx::prefetch_l2(zr + o);
         }
       }
@@ -630,10 +645,9 @@ __device__ __forceinline__ void epilogue_prefetch(const EpiParams& ep, const TcA
 // lines of the output region are in place when the first accumulator is ready.
 template <int BN, int MODE>
 __device__ __forceinline__ void epilogue_touch_outputs(const EpiParams& ep, const TcArgs& a, int mb, int nb, int g,
-                                                       int half, int lane) {
-  constexpr int HALF = BN / 2;
+                                                       int c_lo, int lane) {
   const int m = mb * kBM + g * 32 + lane;
-  const int n_lo = nb * BN + half * HALF;
+  const int n_lo = nb * BN + c_lo;
   if (m >= a.M || n_lo >= a.N) return;
   if constexpr (MODE == EPI_STORE || MODE == EPI_RELU2 || MODE == EPI_QKV) {
     ptx::prefetch_l2(reinterpret_cast<const bf16*>(ep.out) + (size_t)m * ep.ldo + n_lo);
@@ -643,15 +657,14 @@ __device__ __forceinline__ void epilogue_touch_outputs(const EpiParams& ep, cons
 }
 
 // Epilogue work of one warp on one tile: rows g*32 .. g*32+31 of the tile
-// (its TMEM lane quarter) and the columns [c_lo, c_lo + BN/2) of its half.
+// (its TMEM lane quarter) and the columns [c_lo, c_lo + c_cnt) (a multiple
+// of 32; the two warps of a lane quarter split the tile's columns).
 template <int BN, int MODE>
 __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs& a, uint32_t taddr, int mb,
-                                              int nb, int g, int half, int lane, float* stage,
+                                              int nb, int g, int c_lo, int c_cnt, int lane, float* stage,
                                               const RowPre& pre) {
-  constexpr int HALF = BN / 2;
   const int row = g * 32 + lane;
   const int m = mb * kBM + row;
-  const int c_lo = half * HALF;
   const int n_lo = nb * BN + c_lo;
   const float rscale = pre.rscale;  // fused RMSNorm of the A operand: 1 / rms of this thread's row
   if constexpr (MODE == EPI_QKV) {
@@ -666,7 +679,7 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs&
     const float c2 = -2.0f * ep.cap;
     float sum = 0.f, tgt = 0.f;
 #pragma unroll 1
-    for (int c = 0; c < HALF; c += 32) {
+    for (int c = 0; c < c_cnt; c += 32) {
       uint32_t r[32];
       ptx::tmem_ld32(taddr + (uint32_t)(c_lo + c), r);
       ptx::tmem_ld_wait();
@@ -694,20 +707,20 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs&
       }
     }
     if (m < a.M) {
-      ep.ce_sum[(size_t)m * ep.ce_tiles + nb * 2 + half] = sum;
-      if (y >= n_lo && y < n_lo + HALF) ep.ce_tgt[m] = tgt;
+      ep.ce_sum[(size_t)m * ep.ce_tiles + nb * 2 + (2 * c_lo) / BN] = sum;
+      if (y >= n_lo && y < n_lo + c_cnt) ep.ce_tgt[m] = tgt;
     }
   } else if constexpr (MODE == EPI_DZ || MODE == EPI_F32) {
     const float ginv = MODE == EPI_DZ ? *ep.inv_count : 0.f;
     uint32_t r[32];
     ptx::tmem_ld32(taddr + (uint32_t)c_lo, r);
 #pragma unroll 1
-    for (int c = 0; c < HALF; c += 32) {
+    for (int c = 0; c < c_cnt; c += 32) {
       ptx::tmem_ld_wait();
       uint32_t rc[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) rc[i] = r[i];
-      if (c + 32 < HALF) ptx::tmem_ld32(taddr + (uint32_t)(c_lo + c + 32), r);
+      if (c + 32 < c_cnt) ptx::tmem_ld32(taddr + (uint32_t)(c_lo + c + 32), r);
       epi_bwd_chunk<MODE>(ep, a, stage, mb * kBM + g * 32, n_lo + c, rc, lane, pre, ginv);
     }
   } else if constexpr (MODE == EPI_RESID) {
@@ -718,29 +731,22 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs&
     ptx::tmem_ld32(taddr + (uint32_t)c_lo, r);
     resid_load(ep, a, row0, n_lo, lane, xv);
 #pragma unroll 1
-    for (int c = 0; c < HALF; c += 32) {
+    for (int c = 0; c < c_cnt; c += 32) {
       ptx::tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = __uint_as_float(r[i]);
       __syncwarp();
       float4 xn[8];
-      if (c + 32 < HALF) {
+      if (c + 32 < c_cnt) {
         ptx::tmem_ld32(taddr + (uint32_t)(c_lo + c + 32), r);
         resid_load(ep, a, row0, n_lo + c + 32, lane, xn);
       }
       resid_apply(ep, a, stage, row0, n_lo + c, lane, xv, ssr);
       __syncwarp();
-      if (c + 32 < HALF) {
+      store_chunk_ss(ep, a, row0, n_lo + c, lane, ssr);
+      if (c + 32 < c_cnt) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) xv[i] = xn[i];
-      }
-    }
-    // lane (q, 0) holds the sums of rows 4 i + q
-    if (ep.ss_out != nullptr && (lane & 7) == 0) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int mr = row0 + 4 * i + (lane >> 3);
-        if (mr < a.M) ep.ss_out[(size_t)mr * ep.ss_parts + n_lo / HALF] = ssr[i];
       }
     }
   } else {
@@ -749,28 +755,20 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs&
     uint32_t r[32];
     ptx::tmem_ld32(taddr + (uint32_t)c_lo, r);
 #pragma unroll 1
-    for (int c = 0; c < HALF; c += 32) {
+    for (int c = 0; c < c_cnt; c += 32) {
       ptx::tmem_ld_wait();
       uint32_t rc[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) rc[i] = r[i];
-      if (c + 32 < HALF) ptx::tmem_ld32(taddr + (uint32_t)(c_lo + c + 32), r);
+      if (c + 32 < c_cnt) ptx::tmem_ld32(taddr + (uint32_t)(c_lo + c + 32), r);
       if constexpr (MODE == EPI_BLOCK_END) {
         epi_resid_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, rc, lane, ssr);
+        store_chunk_ss(ep, a, mb * kBM + g * 32, n_lo + c, lane, ssr);
       } else {
         epi_store_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, rc, lane, MODE == EPI_RELU2, rscale);
       }
     }
-    if constexpr (MODE == EPI_BLOCK_END) {
-      // lane (q, 0) holds the sums of rows 4 i + q
-      if (ep.ss_out != nullptr && (lane & 7) == 0) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int mr = mb * kBM + g * 32 + 4 * i + (lane >> 3);
-          if (mr < a.M) ep.ss_out[(size_t)mr * ep.ss_parts + n_lo / HALF] = ssr[i];
-        }
-      }
-    }
+
   }
 }
 
@@ -921,25 +919,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int ew = warp - 2;
     const int g = warp & 3;
     const int half = ew >> 2;
+    const int c_lo = half * (BN / 2), c_cnt = BN / 2;
     float* stage = epi_stage + ew * Cf::STAGE_FLOATS;
     int acc = 0;
     uint32_t aph = 0;
     if (blockIdx.x < a.num_tiles) {
-      epilogue_prefetch<BN, MODE>(ep, a, blockIdx.x % a.tiles_m, blockIdx.x / a.tiles_m, g, half, lane);
-      epilogue_touch_outputs<BN, MODE>(ep, a, blockIdx.x % a.tiles_m, blockIdx.x / a.tiles_m, g, half, lane);
+      epilogue_prefetch<BN, MODE>(ep, a, blockIdx.x % a.tiles_m, blockIdx.x / a.tiles_m, g, c_lo, c_cnt, lane);
+      epilogue_touch_outputs<BN, MODE>(ep, a, blockIdx.x % a.tiles_m, blockIdx.x / a.tiles_m, g, c_lo, lane);
     }
     for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
       const int mb = tile % a.tiles_m, nb = tile / a.tiles_m;
-      const RowPre pre = epilogue_pre<BN, MODE>(ep, a, mb, nb, g, half, lane);
+      const RowPre pre = epilogue_pre<BN, MODE>(ep, a, mb, nb, g, c_lo, lane);
       const int nxt = tile + gridDim.x;
-      if (nxt < a.num_tiles) epilogue_prefetch<BN, MODE>(ep, a, nxt % a.tiles_m, nxt / a.tiles_m, g, half, lane);
+      if (nxt < a.num_tiles)
+        epilogue_prefetch<BN, MODE>(ep, a, nxt % a.tiles_m, nxt / a.tiles_m, g, c_lo, c_cnt, lane);
       if (*abort_flag || !ptx::mbar_wait(tfull(acc), aph, a.status)) {
         *abort_flag = 1;
         break;
       }
       ptx::tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(g * 32) << 16) + (uint32_t)(acc * BN);
-      epilogue_tile<BN, MODE>(ep, a, taddr, mb, nb, g, half, lane, stage, pre);
+      epilogue_tile<BN, MODE>(ep, a, taddr, mb, nb, g, c_lo, c_cnt, lane, stage, pre);
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(tempty(acc));
@@ -974,24 +974,29 @@ constexpr int kPairWarpTma = 8, kPairWarpMma = 9;
 constexpr int kPairRegsLow = 88, kPairRegsHigh = 208;
 static_assert(2 * 128 * kPairRegsHigh + 128 * kPairRegsLow <= kPairThreads * 168, "register split");
 
+// BN_ = 256: 256 x 256 pair tiles.  BN_ = 96: 256 x 96 pair tiles for N =
+// 1536 (the output and down projections): 16 x 32 = 512 tiles at M = 8192 are
+// 6.92 waves over 74 CTA pairs, where 256 x 256 tiles are 2.59 waves run as 3.
+template <int BN_>
 struct PairCfg {
-  static constexpr int BN = 256;
-  static constexpr int STAGES = 6;
+  static constexpr int BN = BN_;
+  static constexpr int STAGES = BN == 256 ? 6 : 8;
   static constexpr int A_BYTES = kBM * kBK * 2;       // 16 KB: this CTA's 128 rows of A
-  static constexpr int B_BYTES = (BN / 2) * kBK * 2;  // 16 KB: this CTA's 128 rows of B
+  static constexpr int B_BYTES = (BN / 2) * kBK * 2;  // this CTA's BN/2 rows of B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int TMEM_COLS = 2 * BN;
+  static_assert(STAGE_BYTES % 1024 == 0, "stages stay aligned to the 128-byte swizzle atom");
+  static constexpr int TMEM_COLS = BN == 256 ? 512 : 256;  // two accumulators, rounded to a power of 2
   static constexpr int NBARS = 2 * STAGES + 5;
   static constexpr int STAGE_FLOATS = 32 * 33;
   static constexpr int EPI_BYTES = kEpiWarps * STAGE_FLOATS * 4;
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256 + EPI_BYTES;
 };
 
-template <int MODE>
+template <int MODE, int BN_ = 256>
 __global__ void __launch_bounds__(kPairThreads, 1)
     k_gemm_tc2(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const TcArgs a, const EpiParams ep) {
-  using Cf = PairCfg;
+  using Cf = PairCfg<BN_>;
   constexpr int BN = Cf::BN;
   constexpr int S = Cf::STAGES;
   pdl_launch_dependents();
@@ -1132,31 +1137,47 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const int ew = warp;
     const int g = warp & 3;  // TMEM lane quarter
     const int half = ew >> 2;
+    // the two warps of a lane quarter split the tile's columns: halves of
+    // BN / 2, or for BN = 96 the 32-column chunks {0, 1} and {2}, the two
+    // shares swapping from one job to the next
+    auto cols = [&](int j, int& c_lo, int& c_cnt) {
+      if (BN == 96) {
+        const bool big = (j & 1) == half;
+        c_lo = big ? 0 : 64;
+        c_cnt = big ? 64 : 32;
+      } else {
+        c_lo = half * (BN / 2);
+        c_cnt = BN / 2;
+      }
+    };
     float* stage = epi_stage + ew * Cf::STAGE_FLOATS;
     int acc = 0;
     uint32_t aph = 0;
     if (sched.njobs > 0) {
       int pt, kb_lo, kb_hi, kind;
       job_at(sched, 0, pt, kb_lo, kb_hi, kind);
-      int mbp, nb;
+      int mbp, nb, c_lo, c_cnt;
       pair_tile(a, pt, tiles_mp, mbp, nb);
-      epilogue_prefetch<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, half, lane);
-      epilogue_touch_outputs<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, half, lane);
+      cols(0, c_lo, c_cnt);
+      epilogue_prefetch<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, c_lo, c_cnt, lane);
+      epilogue_touch_outputs<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, c_lo, lane);
     }
     for (int j = 0; j < sched.njobs; ++j) {
       int pt, kb_lo, kb_hi, kind;
       job_at(sched, j, pt, kb_lo, kb_hi, kind);
       const bool head = kind == 1;  // k-blocks of a tile another pair finishes: write a partial
       const bool tail = kind == 2;  // finishes a tile: add the earlier pairs' partials
-      int mbp, nb;
+      int mbp, nb, c_lo, c_cnt;
       pair_tile(a, pt, tiles_mp, mbp, nb);
-      const RowPre pre = epilogue_pre<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, half, lane);
+      cols(j, c_lo, c_cnt);
+      const RowPre pre = epilogue_pre<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, c_lo, lane);
       if (j + 1 < sched.njobs) {
-        int ptn, kln, khn, kn;
+        int ptn, kln, khn, kn, cln, ccn;
         job_at(sched, j + 1, ptn, kln, khn, kn);
         int mbn, nbn;
         pair_tile(a, ptn, tiles_mp, mbn, nbn);
-        epilogue_prefetch<BN, MODE>(ep, a, mbn * 2 + (int)rank, nbn, g, half, lane);
+        cols(j + 1, cln, ccn);
+        epilogue_prefetch<BN, MODE>(ep, a, mbn * 2 + (int)rank, nbn, g, cln, ccn, lane);
       }
       if (*abort_flag || !ptx::mbar_wait_cluster(tfull(acc), aph, a.status)) {
         *abort_flag = 1;
@@ -1218,7 +1239,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             ptx::tmem_st_wait();
           }
         }
-        epilogue_tile<BN, MODE>(ep, a, taddr, mbp * 2 + (int)rank, nb, g, half, lane, stage, pre);
+        epilogue_tile<BN, MODE>(ep, a, taddr, mbp * 2 + (int)rank, nb, g, c_lo, c_cnt, lane, stage, pre);
       }
       ptx::tc_fence_before();
       __syncwarp();
@@ -1269,16 +1290,23 @@ bool launch_layout_mode(const CUtensorMap& ta, const CUtensorMap& tb, const TcAr
                     ep) == cudaSuccess;
 }
 
-template <int MODE>
+template <int MODE, int BN = 256>
 bool launch_pair_mode(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep,
                       int nclusters, cudaStream_t st) {
-  if (!smem_optin(k_gemm_tc2<MODE>, PairCfg::SMEM)) return false;
-  return launch_pdl(k_gemm_tc2<MODE>, dim3(2 * nclusters), dim3(kPairThreads), PairCfg::SMEM, st, 2, ta, tb, a,
-                    ep) == cudaSuccess;
+  if (!smem_optin(k_gemm_tc2<MODE, BN>, PairCfg<BN>::SMEM)) return false;
+  return launch_pdl(k_gemm_tc2<MODE, BN>, dim3(2 * nclusters), dim3(kPairThreads), PairCfg<BN>::SMEM, st, 2, ta, tb,
+                    a, ep) == cudaSuccess;
 }
 
 bool launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep, int nclusters,
-                 cudaStream_t st) {
+                 cudaStream_t st, int bn) {
+  if (bn == 96) {
+    switch (ep.mode) {
+      case EPI_RESID: return launch_pair_mode<EPI_RESID, 96>(ta, tb, a, ep, nclusters, st);
+      case EPI_BLOCK_END: return launch_pair_mode<EPI_BLOCK_END, 96>(ta, tb, a, ep, nclusters, st);
+      default: return false;
+    }
+  }
   switch (ep.mode) {
     case EPI_STORE: return launch_pair_mode<EPI_STORE>(ta, tb, a, ep, nclusters, st);
     case EPI_RELU2: return launch_pair_mode<EPI_RELU2>(ta, tb, a, ep, nclusters, st);
@@ -1367,16 +1395,20 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
                     const StreamK* sk) {
   const int BN = gemm_tc_bn(N);
   if (pair && BN == 256 && num_sms >= 2) {
-    // CTA pairs: each CTA loads 128 rows of A and 128 rows of B per k-slice
+    // CTA pairs: each CTA loads 128 rows of A and BN_p / 2 rows of B per k-slice.
+    // The residual-update GEMMs take 256 x 96 tiles when N allows (a finer
+    // wave quantisation at N = 1536), unless the split-tail schedule is asked for.
+    const bool narrow = (ep.mode == EPI_RESID || ep.mode == EPI_BLOCK_END) && N % 96 == 0 && sk == nullptr;
+    const int bnp = narrow ? 96 : 256;
     CUtensorMap ta, tb;
     if (!make_tmap_2d(&ta, A, M, K, lda, kBM, kBK)) return false;
-    if (!make_tmap_2d(&tb, Bm, N, K, ldb, BN / 2, kBK)) return false;
+    if (!make_tmap_2d(&tb, Bm, N, K, ldb, bnp / 2, kBK)) return false;
     TcArgs a;
     a.M = M;
     a.N = N;
     a.K = K;
     a.tiles_m = (M + kBM - 1) / kBM;
-    a.tiles_n = N / BN;
+    a.tiles_n = N / bnp;
     a.num_tiles = a.tiles_m * a.tiles_n;
     a.n_fastest = ep.mode != EPI_CE;
     a.status = status;
@@ -1393,7 +1425,7 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
     a.sk_wait_ns = kWaitLimitNs;
     // (and when the partial wave is at least a quarter full, so that a tile is
     // cut among a few pairs only)
-    if (sk != nullptr && sk->ws != nullptr && ncl <= sk->max_pairs && ep.mode == EPI_BLOCK_END && nk >= 1 &&
+    if (!narrow && sk != nullptr && sk->ws != nullptr && ncl <= sk->max_pairs && ep.mode == EPI_BLOCK_END && nk >= 1 &&
         num_pt >= ncl && num_pt % ncl != 0 && 4 * (num_pt % ncl) >= ncl) {
       a.streamk = 1;
       a.sk_ws = sk->ws;
@@ -1404,7 +1436,7 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
       a.sk_expect = sk->gen + skew;
     }
     LaunchScope scope_(KK_GEMM_TC, st);
-    return launch_pair(ta, tb, a, ep, ncl, st);
+    return launch_pair(ta, tb, a, ep, ncl, st, bnp);
   }
   CUtensorMap ta, tb;
   if (!make_tmap_2d(&ta, A, M, K, lda, kBM, kBK)) return false;

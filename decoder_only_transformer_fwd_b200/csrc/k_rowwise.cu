@@ -94,20 +94,20 @@ __global__ void k_embed(const T* __restrict__ wte, const int32_t* __restrict__ t
 }
 
 // bf16 tables, C = 32 * EPL: one warp walks a run of `run` consecutive
-// positions of one row.  Lane l holds elements [(k * 32 + l) * VW, + VW) of
-// every row for k < EPL / VW, so each load and store is a 16- or 8-byte vector
-// and consecutive lanes touch consecutive bytes.  The normalised embedding of
-// the position before the run is loaded once and then carried in registers
-// from one position to the next (it is what smear mixes in).  Same outputs as
-// k_embed: x0, x = (lam0 + mu0) x0, bf16(x) and its sum of squares.
+// positions of one row.  Lane l holds elements [4 (k * 32 + l), + 4) of every
+// row for k < EPL / 4, so each warp-wide access is contiguous: 256 bytes of a
+// bf16 row, 512 bytes of an fp32 row.  The next position's embedding row is
+// requested before the current one is normalised and stored, so a warp keeps
+// two rows of loads in flight; the normalised embedding of the previous
+// position is carried in registers (it is what smear mixes in).  Same
+// outputs as k_embed: x0, x = (lam0 + mu0) x0, bf16(x) and its sum of squares.
 template <int EPL>
-__global__ void __launch_bounds__(128) k_embed_vec(
+__global__ void __launch_bounds__(64) k_embed_vec(
     const bf16* __restrict__ wte, const int32_t* __restrict__ tokens, const float* __restrict__ smear_gate,
     int smear, int gc, const float* __restrict__ lam0p, const float* __restrict__ mu0p, float eps, int B, int T_,
     int C, int V, int run, float* __restrict__ x, float* __restrict__ x0, bf16* __restrict__ xb,
     float* __restrict__ ss, int ss_parts, int* status) {
-  constexpr int VW = (EPL % 8 == 0) ? 8 : 4;  // elements per vector access
-  constexpr int NCH = EPL / VW;
+  constexpr int NCH = EPL / 4;
   pdl_launch_dependents();
   pdl_wait();
   const int lane = threadIdx.x & 31;
@@ -118,34 +118,24 @@ __global__ void __launch_bounds__(128) k_embed_vec(
   const int t0 = (wid % runs_per_row) * run;
   const int t1 = min(T_, t0 + run);
   const float inv_c = 1.0f / (float)C;
-  // the normalised embedding row of token `tok` into v
-  auto load_norm = [&](int tok, float (&v)[EPL]) {
-    const bf16* row = wte + (size_t)tok * C;
+  auto load_raw = [&](int tok, uint2 (&u)[NCH]) {
+    const uint2* row = reinterpret_cast<const uint2*>(wte + (size_t)tok * C);
 #pragma unroll
-    for (int k = 0; k < NCH; ++k) {
-      const int e0 = (k * 32 + lane) * VW;
-      if constexpr (VW == 8) {
-        const uint4 u = *reinterpret_cast<const uint4*>(row + e0);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-          v[k * 8 + 2 * i] = f.x;
-          v[k * 8 + 2 * i + 1] = f.y;
-        }
-      } else {
-        const uint2 u = *reinterpret_cast<const uint2*>(row + e0);
-        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-        const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-        v[k * 4 + 0] = f0.x;
-        v[k * 4 + 1] = f0.y;
-        v[k * 4 + 2] = f1.x;
-        v[k * 4 + 3] = f1.y;
-      }
-    }
+    for (int k = 0; k < NCH; ++k) u[k] = row[k * 32 + lane];
+  };
+  // raw row -> normalised fp32 values
+  auto normalise = [&](const uint2 (&u)[NCH], float (&v)[EPL]) {
     float sq = 0.f;
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) sq = fmaf(v[i], v[i], sq);
+    for (int k = 0; k < NCH; ++k) {
+      const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[k].x));
+      const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[k].y));
+      v[4 * k] = f0.x;
+      v[4 * k + 1] = f0.y;
+      v[4 * k + 2] = f1.x;
+      v[4 * k + 3] = f1.y;
+      sq = fmaf(f0.x, f0.x, fmaf(f0.y, f0.y, fmaf(f1.x, f1.x, fmaf(f1.y, f1.y, sq))));
+    }
     const float r = 1.0f / sqrtf(warp_sum(sq) * inv_c + eps);
 #pragma unroll
     for (int i = 0; i < EPL; ++i) v[i] *= r;
@@ -159,24 +149,28 @@ __global__ void __launch_bounds__(128) k_embed_vec(
     return tok;
   };
   float prev[EPL];
+  uint2 raw[NCH], nxt[NCH];
   if (smear && t0 > 0) {
     // its out-of-range flag is raised by the warp that owns that position
-    int tp = tokens[(size_t)b * T_ + t0 - 1];
-    load_norm(min(max(tp, 0), V - 1), prev);
+    const int tp = tokens[(size_t)b * T_ + t0 - 1];
+    load_raw(min(max(tp, 0), V - 1), raw);
+    normalise(raw, prev);
   }
+  load_raw(token(t0), raw);
   const float scale = *lam0p + *mu0p;
   for (int t = t0; t < t1; ++t) {
+    if (t + 1 < t1) load_raw(token(t + 1), nxt);  // in flight while this position is processed
     float cur[EPL];
-    load_norm(token(t), cur);
+    normalise(raw, cur);
     float g = 0.f;
     if (smear && t > 0) {
       float d = 0.f;
 #pragma unroll
       for (int k = 0; k < NCH; ++k)
 #pragma unroll
-        for (int i = 0; i < VW; ++i) {
-          const int c = (k * 32 + lane) * VW + i;
-          if (c < gc) d = fmaf(smear_gate[c], cur[k * VW + i], d);
+        for (int i = 0; i < 4; ++i) {
+          const int c = (k * 32 + lane) * 4 + i;
+          if (c < gc) d = fmaf(smear_gate[c], cur[4 * k + i], d);
         }
       g = sigmoidf_(warp_sum(d));
     }
@@ -184,24 +178,21 @@ __global__ void __launch_bounds__(128) k_embed_vec(
     float sq = 0.f;
 #pragma unroll
     for (int k = 0; k < NCH; ++k) {
-      const int e0 = (k * 32 + lane) * VW;
-      float o[VW];
+      const int e0 = (k * 32 + lane) * 4;
+      float o[4];
 #pragma unroll
-      for (int i = 0; i < VW; ++i) {
-        o[i] = (smear && t > 0) ? fmaf(g, prev[k * VW + i], cur[k * VW + i]) : cur[k * VW + i];
-        prev[k * VW + i] = cur[k * VW + i];
+      for (int i = 0; i < 4; ++i) {
+        o[i] = (smear && t > 0) ? fmaf(g, prev[4 * k + i], cur[4 * k + i]) : cur[4 * k + i];
+        prev[4 * k + i] = cur[4 * k + i];
       }
-#pragma unroll
-      for (int i = 0; i < VW; i += 4) {
-        *reinterpret_cast<float4*>(x0 + m * C + e0 + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
-        const float4 xv = make_float4(scale * o[i], scale * o[i + 1], scale * o[i + 2], scale * o[i + 3]);
-        *reinterpret_cast<float4*>(x + m * C + e0 + i) = xv;
-        sq = fmaf(xv.x, xv.x, fmaf(xv.y, xv.y, fmaf(xv.z, xv.z, fmaf(xv.w, xv.w, sq))));
-        if (xb != nullptr) {
-          const __nv_bfloat162 b0 = __floats2bfloat162_rn(xv.x, xv.y), b1 = __floats2bfloat162_rn(xv.z, xv.w);
-          *reinterpret_cast<uint2*>(xb + m * C + e0 + i) =
-              make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
-        }
+      *reinterpret_cast<float4*>(x0 + m * C + e0) = make_float4(o[0], o[1], o[2], o[3]);
+      const float4 xv = make_float4(scale * o[0], scale * o[1], scale * o[2], scale * o[3]);
+      *reinterpret_cast<float4*>(x + m * C + e0) = xv;
+      sq = fmaf(xv.x, xv.x, fmaf(xv.y, xv.y, fmaf(xv.z, xv.z, fmaf(xv.w, xv.w, sq))));
+      if (xb != nullptr) {
+        const __nv_bfloat162 b0 = __floats2bfloat162_rn(xv.x, xv.y), b1 = __floats2bfloat162_rn(xv.z, xv.w);
+        *reinterpret_cast<uint2*>(xb + m * C + e0) =
+            make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
       }
     }
     if (xb != nullptr) {
@@ -209,6 +200,8 @@ __global__ void __launch_bounds__(128) k_embed_vec(
       sq = warp_sum(sq);
       for (int j = lane; j < ss_parts; j += 32) ss[m * ss_parts + j] = j == 0 ? sq : 0.f;
     }
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) raw[k] = nxt[k];
   }
 }
 
@@ -515,7 +508,16 @@ __global__ void k_ce_combine(const float* ce_sum, const float* ce_tgt, int n_til
   if (m >= M) return;
   const float* ps = ce_sum + (size_t)m * n_tiles;
   float s = 0.f;
-  for (int i = lane; i < n_tiles; i += 32) s += ps[i];
+  if ((n_tiles & 3) == 0) {
+    // 16-byte loads: a row of 2 V_pad / 128 partial sums is 2 KB at V = 32768
+    const float4* p4 = reinterpret_cast<const float4*>(ps);
+    for (int i = lane; i < n_tiles / 4; i += 32) {
+      const float4 v = p4[i];
+      s += (v.x + v.y) + (v.z + v.w);
+    }
+  } else {
+    for (int i = lane; i < n_tiles; i += 32) s += ps[i];
+  }
   s = warp_sum(s);
   if (lane == 0) {
     const int y = targets[m];
@@ -615,9 +617,9 @@ void launch_embed(const void* wte, const int32_t* tokens, const float* smear_gat
   LaunchScope scope_(KK_EMBED, st);
   const int M = B * T;
   if (act_bf16 && C % 128 == 0 && C <= 2048) {
-    constexpr int kRun = 4;
+    constexpr int kRun = 8;
     const int warps = B * ((T + kRun - 1) / kRun);
-    const dim3 grid((warps + 3) / 4), block(128);
+    const dim3 grid((warps + 1) / 2), block(64);
     const bf16* w = (const bf16*)wte;
     switch (C / 32) {
 #define NC_EMBED_CASE(E)                                                                                      \
