@@ -127,28 +127,6 @@ using ptx::ex2;
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
-// 2^e on the FMA and integer pipes, for a share of the exponentials, so that
-// the special-function unit (16 results per clock per SM, the same rate at
-// which the tensor core consumes them at D = 128) is not the bound.  Range
-// reduction e = n + f with n = rint(e), f in [-0.5, 0.5]: adding 1.5 * 2^23
-// leaves n in the low mantissa bits of t; 2^f by a cubic fitted to minimise
-// the relative error on [-0.5, 0.5] (max 7.5e-5, far below the bf16 step
-// 2^-8 that p is rounded to); n is added to the exponent field.  e is
-// clamped at -125 so that the result stays a normal number (2^-125 for masked
-// entries, which no output can see next to the row's maximum term 2^0..2^8).
-__device__ __forceinline__ float2 exp2_poly(float2 e) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  e.x = fmaxf(e.x, -125.0f);
-  e.y = fmaxf(e.y, -125.0f);
-  const float2 t = __fadd2_rn(e, make_float2(kShift, kShift));
-  const float2 n = __fadd2_rn(t, make_float2(-kShift, -kShift));
-  const float2 f = __ffma2_rn(n, make_float2(-1.0f, -1.0f), e);
-  float2 q = __ffma2_rn(make_float2(0.05517132f, 0.05517132f), f, make_float2(0.24261054f, 0.24261054f));
-  q = __ffma2_rn(q, f, make_float2(0.69326099f, 0.69326099f));
-  q = __ffma2_rn(q, f, make_float2(0.99992811f, 0.99992811f));
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
-}
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -166,7 +144,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 // [k2 | k1] (the card's own construction).  Q2 and the pre-scaled Q1 fill the
 // two Q buffers (so an item is one query tile), and each key tile takes three
 // ring slots: K2, K1, V.
-template <int POLY, bool ROUTE>
+template <int OPT, bool ROUTE>
 __global__ void __launch_bounds__(kThreads, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ1,
@@ -411,56 +389,102 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*abort_flag || !ptx::mbar_wait(bar(B_S + g), cnt & 1, a.status)) { ok = false; break; }
         ptx::tc_fence_after();
         float x[128];
-        {
-          // four TMEM loads in flight behind one wait
-          uint32_t u0[32], u1[32], u2[32], u3[32];
-          ptx::tmem_ld32(tS, u0);
-          ptx::tmem_ld32(tS + 32, u1);
-          ptx::tmem_ld32(tS + 64, u2);
-          ptx::tmem_ld32(tS + 96, u3);
-          ptx::tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            x[i] = __uint_as_float(u0[i]);
-            x[32 + i] = __uint_as_float(u1[i]);
-            x[64 + i] = __uint_as_float(u2[i]);
-            x[96 + i] = __uint_as_float(u3[i]);
-          }
-        }
         // visible keys of this row in this tile: columns [clo, chi]
         const int clo = qi - a.window + 1 - k0;
         const int chi = qi - k0;
-        if (!(clo <= 0 && chi >= kK - 1)) {
-#pragma unroll
-          for (int i = 0; i < 128; ++i) x[i] = (i >= clo && i <= chi) ? x[i] : -INFINITY;
-        }
-        // row max: eight chains of three-input max
-        float mx[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(x[2 * k], x[2 * k + 1]);
-#pragma unroll
-        for (int i = 16; i < 128; i += 16)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], x[i + 2 * k], x[i + 2 * k + 1]);
-        const float tmax = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-        // lazy max (raw score units): move it only when it grows by more than 2^8 after scaling
-        const bool rescale = (tmax - m_run) * c > kRescaleThreshold;
-        const float m_new = rescale ? tmax : m_run;
-        const float mc = (m_new == -INFINITY) ? 0.f : m_new * c;
-        // p = 2^(s c - m c) on pairs, packed to bf16 over S's first 64 columns
+        const bool full_tile = clo <= 0 && chi >= kK - 1;
         float2 sm[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        const float2 c2 = make_float2(c, c), mc2 = make_float2(-mc, -mc);
-#pragma unroll
-        for (int qd = 0; qd < 4; ++qd) {
+        const float2 c2 = make_float2(c, c);
+        // p = 2^(s c - m c) for quarter qd (32 keys), packed to bf16 over S's columns [16 qd, 16 qd + 16)
+        auto exp_quarter = [&](int qd, float mcq) {
+          const float2 mc2 = make_float2(-mcq, -mcq);
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float2 e = ffma2(make_float2(x[32 * qd + 2 * i], x[32 * qd + 2 * i + 1]), c2, mc2);
-            const float2 p = (POLY > 0 && i % (POLY > 0 ? POLY : 1) == POLY - 1) ? exp2_poly(e) : make_float2(ex2(e.x), ex2(e.y));
+            const float2 p = make_float2(ex2(e.x), ex2(e.y));
             sm[i & 3] = fadd2(sm[i & 3], p);
             pk[i] = pack_bf16(p.x, p.y);
           }
           ptx::tmem_st16(tS + (uint32_t)(16 * qd), pk);
+        };
+        float mx[8];
+        bool rescale;
+        float mc, m_new;
+        if (OPT && t != t_lo && __all_sync(0xffffffffu, m_run != -INFINITY)) {
+          // Every row of the warp has a finite running max: the exponentials
+          // use it straight away, quarter by quarter, while the next quarter's
+          // scores come from tensor memory; the tile's max is gathered along
+          // the way.  P overwrites only scores already read.  In the rare case
+          // that a row's max grew past the threshold, the warp recomputes the
+          // tile's p from the scores kept in registers.
+          const float mc_old = m_run * c;
+          uint32_t u[32];
+          ptx::tmem_ld32(tS, u);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int col = 32 * qd + i;
+              x[col] = (full_tile || (col >= clo && col <= chi)) ? __uint_as_float(u[i]) : -INFINITY;
+            }
+            if (qd < 3) ptx::tmem_ld32(tS + (uint32_t)(32 * (qd + 1)), u);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const float a0 = fmaxf(x[32 * qd + 4 * k], x[32 * qd + 4 * k + 1]);
+              const float a1 = max3(a0, x[32 * qd + 4 * k + 2], x[32 * qd + 4 * k + 3]);
+              mx[k] = qd == 0 ? a1 : fmaxf(mx[k], a1);
+            }
+            exp_quarter(qd, mc_old);
+            if (qd < 3) ptx::tmem_ld_wait();
+          }
+          const float tmax = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+          rescale = (tmax - m_run) * c > kRescaleThreshold;
+          m_new = rescale ? tmax : m_run;
+          mc = rescale ? tmax * c : mc_old;
+          if (__any_sync(0xffffffffu, rescale)) {
+            ptx::tmem_st_wait();
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sm[k] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd) exp_quarter(qd, mc);
+          }
+        } else {
+          // four TMEM loads in flight behind one wait; the row max first
+          {
+            uint32_t u0[32], u1[32], u2[32], u3[32];
+            ptx::tmem_ld32(tS, u0);
+            ptx::tmem_ld32(tS + 32, u1);
+            ptx::tmem_ld32(tS + 64, u2);
+            ptx::tmem_ld32(tS + 96, u3);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              x[i] = __uint_as_float(u0[i]);
+              x[32 + i] = __uint_as_float(u1[i]);
+              x[64 + i] = __uint_as_float(u2[i]);
+              x[96 + i] = __uint_as_float(u3[i]);
+            }
+          }
+          if (!full_tile) {
+#pragma unroll
+            for (int i = 0; i < 128; ++i) x[i] = (i >= clo && i <= chi) ? x[i] : -INFINITY;
+          }
+          // row max: eight chains of three-input max
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = fmaxf(x[2 * k], x[2 * k + 1]);
+#pragma unroll
+          for (int i = 16; i < 128; i += 16)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], x[i + 2 * k], x[i + 2 * k + 1]);
+          const float tmax = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+          // lazy max (raw score units): move it only when it grows by more than 2^8 after scaling
+          rescale = (tmax - m_run) * c > kRescaleThreshold;
+          m_new = rescale ? tmax : m_run;
+          mc = (m_new == -INFINITY) ? 0.f : m_new * c;
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd) exp_quarter(qd, mc);
         }
         const float alpha = rescale ? ex2(m_run * c - mc) : 1.f;  // 0 when m_run == -inf
         if (rescale) {
@@ -559,12 +583,9 @@ bool launch_attn_common(const bf16* q, const bf16* k, const bf16* v, const bf16*
   a.scale_log2 = scale * 1.4426950408889634f;
   a.o = o;
   a.status = status;
-  static const int poly = getenv("NC_ATTN_POLY") ? atoi(getenv("NC_ATTN_POLY")) : 0;
+  static const int opt = getenv("NC_ATTN_OPT") ? atoi(getenv("NC_ATTN_OPT")) : 1;
   void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, AttnArgs) =
-      route ? k_attn_tc<0, true>
-            : (poly == 2 ? k_attn_tc<2, false>
-                         : poly == 3 ? k_attn_tc<3, false>
-                                     : poly == 4 ? k_attn_tc<4, false> : poly == 8 ? k_attn_tc<8, false> : k_attn_tc<0, false>);
+      route ? (opt ? k_attn_tc<1, true> : k_attn_tc<0, true>) : (opt ? k_attn_tc<1, false> : k_attn_tc<0, false>);
   if (!smem_optin(kern, SMEM_BYTES)) return false;
   LaunchScope scope_(KK_ATTN_TC, st);
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;

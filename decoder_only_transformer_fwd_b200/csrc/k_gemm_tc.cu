@@ -974,9 +974,8 @@ constexpr int kPairWarpTma = 8, kPairWarpMma = 9;
 constexpr int kPairRegsLow = 88, kPairRegsHigh = 208;
 static_assert(2 * 128 * kPairRegsHigh + 128 * kPairRegsLow <= kPairThreads * 168, "register split");
 
-// BN_ = 256: 256 x 256 pair tiles.  BN_ = 96: 256 x 96 pair tiles for N =
-// 1536 (the output and down projections): 16 x 32 = 512 tiles at M = 8192 are
-// 6.92 waves over 74 CTA pairs, where 256 x 256 tiles are 2.59 waves run as 3.
+// BN_: the pair tile's width (256; the epilogue also handles 96, whose
+// 32-column chunks the two warps of a lane quarter share unevenly).
 template <int BN_>
 struct PairCfg {
   static constexpr int BN = BN_;
@@ -1300,13 +1299,7 @@ bool launch_pair_mode(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs
 
 bool launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, const EpiParams& ep, int nclusters,
                  cudaStream_t st, int bn) {
-  if (bn == 96) {
-    switch (ep.mode) {
-      case EPI_RESID: return launch_pair_mode<EPI_RESID, 96>(ta, tb, a, ep, nclusters, st);
-      case EPI_BLOCK_END: return launch_pair_mode<EPI_BLOCK_END, 96>(ta, tb, a, ep, nclusters, st);
-      default: return false;
-    }
-  }
+  if (bn != 256) return false;
   switch (ep.mode) {
     case EPI_STORE: return launch_pair_mode<EPI_STORE>(ta, tb, a, ep, nclusters, st);
     case EPI_RELU2: return launch_pair_mode<EPI_RELU2>(ta, tb, a, ep, nclusters, st);
@@ -1395,11 +1388,12 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
                     const StreamK* sk) {
   const int BN = gemm_tc_bn(N);
   if (pair && BN == 256 && num_sms >= 2) {
-    // CTA pairs: each CTA loads 128 rows of A and BN_p / 2 rows of B per k-slice.
-    // The residual-update GEMMs take 256 x 96 tiles when N allows (a finer
-    // wave quantisation at N = 1536), unless the split-tail schedule is asked for.
-    const bool narrow = (ep.mode == EPI_RESID || ep.mode == EPI_BLOCK_END) && N % 96 == 0 && sk == nullptr;
-    const int bnp = narrow ? 96 : 256;
+    // CTA pairs: each CTA loads 128 rows of A and 128 rows of B per k-slice.
+    // (256 x 96 tiles would quantise N = 1536 into 6.92 waves instead of 2.59
+    // run as 3, but each CTA then streams 22 KB of operands per 1.6 MFLOP of
+    // MMA, more than L2 delivers to 148 SMs at once: measured 13.9 ms per d24
+    // step against 12.3 ms with 256 x 256 tiles.)
+    const int bnp = 256;
     CUtensorMap ta, tb;
     if (!make_tmap_2d(&ta, A, M, K, lda, kBM, kBK)) return false;
     if (!make_tmap_2d(&tb, Bm, N, K, ldb, bnp / 2, kBK)) return false;
@@ -1425,7 +1419,7 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
     a.sk_wait_ns = kWaitLimitNs;
     // (and when the partial wave is at least a quarter full, so that a tile is
     // cut among a few pairs only)
-    if (!narrow && sk != nullptr && sk->ws != nullptr && ncl <= sk->max_pairs && ep.mode == EPI_BLOCK_END && nk >= 1 &&
+    if (sk != nullptr && sk->ws != nullptr && ncl <= sk->max_pairs && ep.mode == EPI_BLOCK_END && nk >= 1 &&
         num_pt >= ncl && num_pt % ncl != 0 && 4 * (num_pt % ncl) >= ncl) {
       a.streamk = 1;
       a.sk_ws = sk->ws;
