@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   enum {
-    B_QF = 0, B_QE = 1, B_SLF = 2, B_SLE = B_SLF + SLOTS, B_S = B_SLE + SLOTS, B_P = B_S + 2, B_O = B_P + 2,
+    B_QF = 0, B_QE = 2, B_SLF = 4, B_SLE = B_SLF + SLOTS, B_S = B_SLE + SLOTS, B_P = B_S + 2, B_O = B_P + 2,
     B_OE = B_O + 2, B_DONE = B_OE + 2, NB = B_DONE + 1
   };
   static_assert(NB * 8 + 8 <= 256, "barrier area");
@@ -166,8 +166,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(bar(B_QF), 1);
-    ptx::mbar_init(bar(B_QE), 1);
+    for (int g = 0; g < 2; ++g) {
+      ptx::mbar_init(bar(B_QF + g), 1);
+      ptx::mbar_init(bar(B_QE + g), 1);
+    }
     for (int s = 0; s < SLOTS; ++s) {
       ptx::mbar_init(bar(B_SLF + s), 1);
       ptx::mbar_init(bar(B_SLE + s), 1);
@@ -207,8 +209,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kWarpTma) {
     if (ptx::elect_one()) {
       // ---------------- TMA producer ----------------
-      uint32_t issued = 0, par = 0, qpar = 0;
-      bool qissued = false, ok = true;
+      uint32_t issued = 0, par = 0;
+      int qn[2] = {0, 0}, qpar[2] = {0, 0};  // Q loads issued per buffer group, parity of the last
+      bool ok = true;
       int sc = 0, it = 0;
       for (int item = item_of(0); ok && item < a.n_items; ++it, item = item_of(it)) {
         const Item w = decode_item<ROUTE>(a, item);
@@ -233,30 +236,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         // the item's first K/V tiles do not need the Q buffers: start them first
         if (!load_kv(w.lo)) { ok = false; break; }
-        // the previous item's QK MMAs have finished reading the Q buffers
-        if (*abort_flag || !ptx::mbar_wait(bar(B_QE), (it & 1) ^ 1, a.status)) { ok = false; break; }
-        ptx::mbar_arrive_expect_tx(bar(B_QF), (ROUTE || w.has_b ? 2 : 1) * TILE_BYTES);
-        if (ROUTE) {
-          // Q2 into the first buffer, the pre-scaled Q1 into the second
-          for (int g = 0; g < 2; ++g) {
-            const void* tq = g == 0 ? (const void*)&tmQ : (const void*)&tmQ1;
-            ptx::tma_load_2d(sQ(g), tq, bar(B_QF), qcol, row_base + w.q0);
-            ptx::tma_load_2d(sQ(g) + BOX_BYTES, tq, bar(B_QF), qcol + 64, row_base + w.q0);
+        // each group's Q buffer is reloaded once that group's QK MMAs of its
+        // previous item have finished reading it (ROUTE: group 0 owns both
+        // buffers, Q2 in the first and the pre-scaled Q1 in the second)
+        for (int g = 0; g < (ROUTE ? 1 : (w.has_b ? 2 : 1)); ++g) {
+          if (*abort_flag || !ptx::mbar_wait(bar(B_QE + g), (qn[g] & 1) ^ 1, a.status)) { ok = false; break; }
+          ptx::mbar_arrive_expect_tx(bar(B_QF + g), (ROUTE ? 2 : 1) * TILE_BYTES);
+          for (int h = 0; h < (ROUTE ? 2 : 1); ++h) {
+            const int buf = ROUTE ? h : g;
+            const void* tq = (ROUTE && h == 1) ? (const void*)&tmQ1 : (const void*)&tmQ;
+            const int qrow = row_base + w.q0 + (ROUTE ? 0 : g * kQ);
+            ptx::tma_load_2d(sQ(buf), tq, bar(B_QF + g), qcol, qrow);
+            ptx::tma_load_2d(sQ(buf) + BOX_BYTES, tq, bar(B_QF + g), qcol + 64, qrow);
           }
-        } else {
-          for (int g = 0; g < (w.has_b ? 2 : 1); ++g) {
-            ptx::tma_load_2d(sQ(g), &tmQ, bar(B_QF), qcol, row_base + w.q0 + g * kQ);
-            ptx::tma_load_2d(sQ(g) + BOX_BYTES, &tmQ, bar(B_QF), qcol + 64, row_base + w.q0 + g * kQ);
-          }
+          qpar[g] = qn[g] & 1;
+          ++qn[g];
         }
-        qissued = true;
-        qpar = it & 1;
+        if (!ok) break;
         for (int t = w.lo + 1; ok && t <= w.hi; ++t)
           if (!load_kv(t)) ok = false;
       }
       if (!ok) *abort_flag = 1;
       // every copy this thread issued has landed before the CTA may exit
-      if (qissued) ptx::mbar_wait(bar(B_QF), qpar, a.status);
+      for (int g = 0; g < 2; ++g)
+        if (qn[g] > 0) ptx::mbar_wait(bar(B_QF + g), qpar[g], a.status);
       for (int s = 0; s < SLOTS; ++s)
         if (issued & (1u << s)) ptx::mbar_wait(bar(B_SLF + s), (par >> s) & 1, a.status);
     }
@@ -265,9 +268,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------- MMA issuer ----------------
       constexpr uint32_t idesc_qk = ptx::idesc_bf16(kQ, kK, 0, 0);
       constexpr uint32_t idesc_pv = ptx::idesc_bf16(kQ, kD, 0, 1);  // V is MN-major
-      auto slot_wait = [&](int sc) -> bool {
-        return !*abort_flag && ptx::mbar_wait(bar(B_SLF + sc % SLOTS), (uint32_t)(sc / SLOTS) & 1u, a.status);
-      };
       // shared-memory descriptors are built once; the k-steps add constants
       // to their start-address field (16-byte units): K-major steps of 16
       // elements are 32 B within a 64-column box and BOX_BYTES between the
@@ -298,65 +298,129 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::mma_bf16_ts(tO, tP + (uint32_t)(kk * 8), dv + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
                            (!first || kk > 0) ? 1u : 0u);
       };
-      bool ok = true;
-      int sc = 0, it = 0;
-      int pc0 = 0, pc1 = 0, ic0 = 0, ic1 = 0;  // P phases consumed, items finished, per group
-      for (int item = item_of(0); ok && item < a.n_items; ++it, item = item_of(it)) {
-        const Item w = decode_item<ROUTE>(a, item);
-        if (*abort_flag || !ptx::mbar_wait(bar(B_QF), it & 1, a.status)) { ok = false; break; }
-        ptx::tc_fence_after();
-        // K_lo feeds the first S of every group that sees key tile lo
-        if (!slot_wait(sc) || (ROUTE && !slot_wait(sc + 1))) { ok = false; break; }
-        ptx::tc_fence_after();
+      // The two groups advance independently through this CTA's items: group
+      // 0 (tile A) finishes an item one key tile before group 1 (tile B) and
+      // starts the next item's QK while group 1 still works on its last tile.
+      // Each group is a cursor (item, key tile, state); the thread serves
+      // whichever group's next step has its inputs ready (non-blocking
+      // tests), so neither group's wait holds up the other.  A ring slot is
+      // released (tcgen05.commit on its "empty" barrier) after the last of
+      // the groups that use its tile has issued the MMA reading it.
+      struct Cursor {
+        int k, base, t, state;  // state: 0 first QK of an item pending, 1 waiting for P(t), 2 done
+        int pc, ic, qc;         // P phases consumed, items finished, Q phases consumed
+        Item w;
+        int lo, hi;             // this group's key tiles in the item
+      };
+      int uses[SLOTS];
 #pragma unroll
-        for (int g = 0; g < 2; ++g)
-          if (active(w, g, w.lo)) {
-            qk(g, sc);
-            ptx::mma_commit(bar(B_S + g));
-          }
-        if (w.lo == w.hi) ptx::mma_commit(bar(B_QE));
-        ptx::mma_commit(bar(B_SLE + sc % SLOTS));
-        if (ROUTE) ptx::mma_commit(bar(B_SLE + (sc + 1) % SLOTS));
-        for (int t = w.lo; ok && t <= w.hi; ++t) {
-          const int scV = sc + PER_TILE * (t - w.lo) + PER_TILE - 1, scK1 = scV + 1;
-          const bool more = t < w.hi;
-          if (!slot_wait(scV) || (more && !slot_wait(scK1)) || (ROUTE && more && !slot_wait(scK1 + 1))) {
-            ok = false;
-            break;
-          }
-          ptx::tc_fence_after();
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            const bool act = active(w, g, t);
-            const bool next = more && active(w, g, t + 1);
-            if (act) {
-              // group g has written P_g(t)
-              int& pc = g == 0 ? pc0 : pc1;
-              if (*abort_flag || !ptx::mbar_wait(bar(B_P + g), pc & 1, a.status)) { ok = false; break; }
-              ++pc;
-              const bool first = t == (g == 0 ? w.lo0 : w.lo1);
-              // the output of this group's previous item has been read out of O_g
-              const int ic = g == 0 ? ic0 : ic1;
-              if (first && !ptx::mbar_wait(bar(B_OE + g), (ic & 1) ^ 1, a.status)) { ok = false; break; }
-              ptx::tc_fence_after();
-              pv(g, scV, first);
-            }
-            if (next) {
-              qk(g, scK1);
-              ptx::mma_commit(bar(B_S + g));
-            } else if (act) {
-              ptx::mma_commit(bar(B_O + g));  // g's last tile of this item: O_g is final
-            }
-          }
-          if (!ok) break;
-          if (t + 1 == w.hi) ptx::mma_commit(bar(B_QE));  // the item's last QKs are issued
-          ptx::mma_commit(bar(B_SLE + scV % SLOTS));
-          if (more) ptx::mma_commit(bar(B_SLE + scK1 % SLOTS));
-          if (ROUTE && more) ptx::mma_commit(bar(B_SLE + (scK1 + 1) % SLOTS));
+      for (int s = 0; s < SLOTS; ++s) uses[s] = 0;
+      // tile t's users in item w: group 0 when t is one of its tiles, group 1 likewise
+      auto users = [&](const Item& w, int t) { return (int)active(w, 0, t) + (int)active(w, 1, t); };
+      // one use of global ring slot sc (holding a tile of item w at key tile t)
+      auto use_slot = [&](int sc, const Item& w, int t) {
+        const int s = sc % SLOTS;
+        if (uses[s] == 0) uses[s] = users(w, t);
+        if (--uses[s] == 0) ptx::mma_commit(bar(B_SLE + s));
+      };
+      auto slot_ready = [&](int sc) { return ptx::mbar_test(bar(B_SLF + sc % SLOTS), (uint32_t)(sc / SLOTS) & 1u); };
+      // move group g's cursor to the next item in which it has a tile (or done)
+      auto advance = [&](Cursor& c, int g, bool first_call) {
+        if (!first_call) {
+          c.base += PER_TILE * (c.w.hi - c.w.lo + 1);
+          ++c.k;
         }
-        ++ic0;
-        if (w.has_b) ++ic1;
-        sc += PER_TILE * (w.hi - w.lo + 1);
+        while (true) {
+          const int item = item_of(c.k);
+          if (item >= a.n_items) {
+            c.state = 2;
+            return;
+          }
+          c.w = decode_item<ROUTE>(a, item);
+          if (g == 0 || c.w.has_b) break;
+          c.base += PER_TILE * (c.w.hi - c.w.lo + 1);
+          ++c.k;
+        }
+        c.lo = g == 0 ? c.w.lo0 : c.w.lo1;
+        c.hi = g == 0 ? c.w.hi0 : c.w.hi1;
+        c.state = 0;
+      };
+      Cursor cur[2];
+      for (int g = 0; g < 2; ++g) {
+        cur[g].k = 0;
+        cur[g].base = 0;
+        cur[g].t = 0;
+        cur[g].pc = cur[g].ic = cur[g].qc = 0;
+        if (ROUTE && g == 1) {
+          cur[g].state = 2;
+        } else {
+          advance(cur[g], g, true);
+        }
+      }
+      auto k_slot = [&](const Cursor& c, int t) { return c.base + PER_TILE * (t - c.w.lo); };
+      bool ok = true;
+      uint64_t idle_since = 0;
+      while (ok && (cur[0].state != 2 || cur[1].state != 2)) {
+        bool progressed = false;
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          Cursor& c = cur[g];
+          if (c.state == 0) {
+            // the item's first S_g = Q_g K_lo^T: Q_g loaded, K_lo (ROUTE: and K1_lo) in the ring
+            const int sk = k_slot(c, c.lo);
+            if (!ptx::mbar_test(bar(B_QF + g), c.qc & 1) || !slot_ready(sk) || (ROUTE && !slot_ready(sk + 1)))
+              continue;
+            ++c.qc;
+            ptx::tc_fence_after();
+            qk(g, sk);
+            ptx::mma_commit(bar(B_S + g));
+            if (c.lo == c.hi) ptx::mma_commit(bar(B_QE + g));
+            use_slot(sk, c.w, c.lo);
+            if (ROUTE) use_slot(sk + 1, c.w, c.lo);
+            c.t = c.lo;
+            c.state = 1;
+            progressed = true;
+          } else if (c.state == 1) {
+            // P_g(t) written: O_g += P_g V_t, then the next S_g = Q_g K_{t+1}^T
+            const bool first = c.t == c.lo, more = c.t < c.hi;
+            const int sv = k_slot(c, c.t) + PER_TILE - 1, sk = k_slot(c, c.t + 1);
+            if (!ptx::mbar_test(bar(B_P + g), c.pc & 1)) continue;
+            // O_g is free once the group's previous output has been read out
+            if (first && !ptx::mbar_test(bar(B_OE + g), (c.ic & 1) ^ 1)) continue;
+            if (!slot_ready(sv) || (more && (!slot_ready(sk) || (ROUTE && !slot_ready(sk + 1))))) continue;
+            ++c.pc;
+            ptx::tc_fence_after();
+            pv(g, sv, first);
+            use_slot(sv, c.w, c.t);
+            if (more) {
+              qk(g, sk);
+              ptx::mma_commit(bar(B_S + g));
+              if (c.t + 1 == c.hi) ptx::mma_commit(bar(B_QE + g));  // g's last QK of the item
+              use_slot(sk, c.w, c.t + 1);
+              if (ROUTE) use_slot(sk + 1, c.w, c.t + 1);
+              ++c.t;
+            } else {
+              ptx::mma_commit(bar(B_O + g));  // g's last tile of this item: O_g is final
+              ++c.ic;
+              advance(c, g, false);
+            }
+            progressed = true;
+          }
+        }
+        if (progressed) {
+          idle_since = 0;
+        } else if (*abort_flag) {
+          ok = false;
+        } else {
+          // bounded: give up after kWaitLimitNs without any step ready
+          const uint64_t now = ptx::globaltimer();
+          if (idle_since == 0) {
+            idle_since = now;
+          } else if (now - idle_since > kWaitLimitNs) {
+            atomicOr(a.status, kStatusTimeout);
+            ok = false;
+          }
+        }
       }
       if (!ok) *abort_flag = 1;
       ptx::mma_commit(bar(B_DONE));
