@@ -34,8 +34,6 @@
 // are counted over the CTA's whole sequence.  Every wait is bounded; on a
 // timeout the CTA records NC_ERR_TIMEOUT and returns after its copies and
 // MMAs have landed.
-#include <stdlib.h>
-
 #include "nc_internal.cuh"
 #include "ptx.cuh"
 
@@ -61,9 +59,10 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kThreads = 384;
 constexpr int kWarpTma = 8, kWarpMma = 9;
 // registers: launched at 168 per thread (65536 / 384, rounded down to 8);
-// the TMA/MMA warpgroup drops to 104 and the two softmax warpgroups rise to
-// 200: 2 * 128 * 200 + 128 * 104 = 64512 = 384 * 168
-constexpr int kRegsLow = 104, kRegsHigh = 200;
+// the TMA/MMA warpgroup drops to 136 and the two softmax warpgroups rise to
+// 184: 2 * 128 * 184 + 128 * 136 = 64512 = 384 * 168 (the split at which the
+// compiler spills least: 104 / 200 spilled in the MMA issuer)
+constexpr int kRegsLow = 136, kRegsHigh = 184;
 static_assert(2 * 128 * kRegsHigh + 128 * kRegsLow <= kThreads * 168, "register split");
 
 struct AttnArgs {
@@ -144,7 +143,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 // [k2 | k1] (the card's own construction).  Q2 and the pre-scaled Q1 fill the
 // two Q buffers (so an item is one query tile), and each key tile takes three
 // ring slots: K2, K1, V.
-template <int OPT, bool ROUTE>
+template <bool ROUTE>
 __global__ void __launch_bounds__(kThreads, 1)
     k_attn_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQ1,
@@ -298,129 +297,93 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::mma_bf16_ts(tO, tP + (uint32_t)(kk * 8), dv + (uint64_t)(kk * (2048 >> 4)), idesc_pv,
                            (!first || kk > 0) ? 1u : 0u);
       };
-      // The two groups advance independently through this CTA's items: group
-      // 0 (tile A) finishes an item one key tile before group 1 (tile B) and
-      // starts the next item's QK while group 1 still works on its last tile.
-      // Each group is a cursor (item, key tile, state); the thread serves
-      // whichever group's next step has its inputs ready (non-blocking
-      // tests), so neither group's wait holds up the other.  A ring slot is
-      // released (tcgen05.commit on its "empty" barrier) after the last of
-      // the groups that use its tile has issued the MMA reading it.
-      struct Cursor {
-        int k, base, t, state;  // state: 0 first QK of an item pending, 1 waiting for P(t), 2 done
-        int pc, ic, qc;         // P phases consumed, items finished, Q phases consumed
-        Item w;
-        int lo, hi;             // this group's key tiles in the item
+      auto slot_wait = [&](int sc) -> bool {
+        return !*abort_flag && ptx::mbar_wait(bar(B_SLF + sc % SLOTS), (uint32_t)(sc / SLOTS) & 1u, a.status);
       };
-      int uses[SLOTS];
-#pragma unroll
-      for (int s = 0; s < SLOTS; ++s) uses[s] = 0;
-      // tile t's users in item w: group 0 when t is one of its tiles, group 1 likewise
-      auto users = [&](const Item& w, int t) { return (int)active(w, 0, t) + (int)active(w, 1, t); };
-      // one use of global ring slot sc (holding a tile of item w at key tile t)
-      auto use_slot = [&](int sc, const Item& w, int t) {
-        const int s = sc % SLOTS;
-        if (uses[s] == 0) uses[s] = users(w, t);
-        if (--uses[s] == 0) ptx::mma_commit(bar(B_SLE + s));
+      // group g's Q buffer holds the current item's tile (QF_g phase qc[g])
+      int qc[2] = {0, 0};
+      auto q_wait = [&](int g) -> bool {
+        const bool r = !*abort_flag && ptx::mbar_wait(bar(B_QF + g), qc[g] & 1, a.status);
+        ++qc[g];
+        return r;
       };
-      auto slot_ready = [&](int sc) { return ptx::mbar_test(bar(B_SLF + sc % SLOTS), (uint32_t)(sc / SLOTS) & 1u); };
-      // move group g's cursor to the next item in which it has a tile (or done)
-      auto advance = [&](Cursor& c, int g, bool first_call) {
-        if (!first_call) {
-          c.base += PER_TILE * (c.w.hi - c.w.lo + 1);
-          ++c.k;
-        }
-        while (true) {
-          const int item = item_of(c.k);
-          if (item >= a.n_items) {
-            c.state = 2;
-            return;
-          }
-          c.w = decode_item<ROUTE>(a, item);
-          if (g == 0 || c.w.has_b) break;
-          c.base += PER_TILE * (c.w.hi - c.w.lo + 1);
-          ++c.k;
-        }
-        c.lo = g == 0 ? c.w.lo0 : c.w.lo1;
-        c.hi = g == 0 ? c.w.hi0 : c.w.hi1;
-        c.state = 0;
-      };
-      Cursor cur[2];
-      for (int g = 0; g < 2; ++g) {
-        cur[g].k = 0;
-        cur[g].base = 0;
-        cur[g].t = 0;
-        cur[g].pc = cur[g].ic = cur[g].qc = 0;
-        if (ROUTE && g == 1) {
-          cur[g].state = 2;
-        } else {
-          advance(cur[g], g, true);
-        }
-      }
-      auto k_slot = [&](const Cursor& c, int t) { return c.base + PER_TILE * (t - c.w.lo); };
       bool ok = true;
-      uint64_t idle_since = 0;
-      while (ok && (cur[0].state != 2 || cur[1].state != 2)) {
-        bool progressed = false;
+      int sc = 0, it = 0;
+      int pc0 = 0, pc1 = 0, ic0 = 0, ic1 = 0;  // P phases consumed, items finished, per group
+      bool a_started = false;  // tile A's first QK of this item was issued during the previous item
+      for (int item = item_of(0); ok && item < a.n_items; ++it, item = item_of(it)) {
+        const Item w = decode_item<ROUTE>(a, item);
+        // K_lo feeds the first S of every group that sees key tile lo
+        if (!slot_wait(sc) || (ROUTE && !slot_wait(sc + 1))) { ok = false; break; }
 #pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          Cursor& c = cur[g];
-          if (c.state == 0) {
-            // the item's first S_g = Q_g K_lo^T: Q_g loaded, K_lo (ROUTE: and K1_lo) in the ring
-            const int sk = k_slot(c, c.lo);
-            if (!ptx::mbar_test(bar(B_QF + g), c.qc & 1) || !slot_ready(sk) || (ROUTE && !slot_ready(sk + 1)))
-              continue;
-            ++c.qc;
+        for (int g = 0; g < 2; ++g)
+          if (active(w, g, w.lo) && !(g == 0 && a_started)) {
+            if (!q_wait(g)) { ok = false; break; }
             ptx::tc_fence_after();
-            qk(g, sk);
+            qk(g, sc);
             ptx::mma_commit(bar(B_S + g));
-            if (c.lo == c.hi) ptx::mma_commit(bar(B_QE + g));
-            use_slot(sk, c.w, c.lo);
-            if (ROUTE) use_slot(sk + 1, c.w, c.lo);
-            c.t = c.lo;
-            c.state = 1;
-            progressed = true;
-          } else if (c.state == 1) {
-            // P_g(t) written: O_g += P_g V_t, then the next S_g = Q_g K_{t+1}^T
-            const bool first = c.t == c.lo, more = c.t < c.hi;
-            const int sv = k_slot(c, c.t) + PER_TILE - 1, sk = k_slot(c, c.t + 1);
-            if (!ptx::mbar_test(bar(B_P + g), c.pc & 1)) continue;
-            // O_g is free once the group's previous output has been read out
-            if (first && !ptx::mbar_test(bar(B_OE + g), (c.ic & 1) ^ 1)) continue;
-            if (!slot_ready(sv) || (more && (!slot_ready(sk) || (ROUTE && !slot_ready(sk + 1))))) continue;
-            ++c.pc;
-            ptx::tc_fence_after();
-            pv(g, sv, first);
-            use_slot(sv, c.w, c.t);
-            if (more) {
-              qk(g, sk);
-              ptx::mma_commit(bar(B_S + g));
-              if (c.t + 1 == c.hi) ptx::mma_commit(bar(B_QE + g));  // g's last QK of the item
-              use_slot(sk, c.w, c.t + 1);
-              if (ROUTE) use_slot(sk + 1, c.w, c.t + 1);
-              ++c.t;
-            } else {
-              ptx::mma_commit(bar(B_O + g));  // g's last tile of this item: O_g is final
-              ++c.ic;
-              advance(c, g, false);
-            }
-            progressed = true;
+            if (w.lo == (g == 0 ? w.hi0 : w.hi1)) ptx::mma_commit(bar(B_QE + g));  // g's only tile
           }
-        }
-        if (progressed) {
-          idle_since = 0;
-        } else if (*abort_flag) {
-          ok = false;
-        } else {
-          // bounded: give up after kWaitLimitNs without any step ready
-          const uint64_t now = ptx::globaltimer();
-          if (idle_since == 0) {
-            idle_since = now;
-          } else if (now - idle_since > kWaitLimitNs) {
-            atomicOr(a.status, kStatusTimeout);
+        if (!ok) break;
+        a_started = false;
+        ptx::mma_commit(bar(B_SLE + sc % SLOTS));
+        if (ROUTE) ptx::mma_commit(bar(B_SLE + (sc + 1) % SLOTS));
+        for (int t = w.lo; ok && t <= w.hi; ++t) {
+          const int scV = sc + PER_TILE * (t - w.lo) + PER_TILE - 1, scK1 = scV + 1;
+          const bool more = t < w.hi;
+          if (!slot_wait(scV) || (more && !slot_wait(scK1)) || (ROUTE && more && !slot_wait(scK1 + 1))) {
             ok = false;
+            break;
           }
+          ptx::tc_fence_after();
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            const bool act = active(w, g, t);
+            const bool next = more && active(w, g, t + 1);
+            if (act) {
+              // group g has written P_g(t)
+              int& pc = g == 0 ? pc0 : pc1;
+              if (*abort_flag || !ptx::mbar_wait(bar(B_P + g), pc & 1, a.status)) { ok = false; break; }
+              ++pc;
+              const bool first = t == (g == 0 ? w.lo0 : w.lo1);
+              // the output of this group's previous item has been read out of O_g
+              const int ic = g == 0 ? ic0 : ic1;
+              if (first && !ptx::mbar_wait(bar(B_OE + g), (ic & 1) ^ 1, a.status)) { ok = false; break; }
+              ptx::tc_fence_after();
+              pv(g, scV, first);
+            }
+            if (next) {
+              // tile B's first key tile may follow the item's first (its Q was not needed before)
+              if (!act && !q_wait(g)) { ok = false; break; }
+              ptx::tc_fence_after();
+              qk(g, scK1);
+              ptx::mma_commit(bar(B_S + g));
+              if (t + 1 == (g == 0 ? w.hi0 : w.hi1)) ptx::mma_commit(bar(B_QE + g));  // g's last QK of the item
+            } else if (act) {
+              ptx::mma_commit(bar(B_O + g));  // g's last tile of this item: O_g is final
+              const int nitem = item_of(it + 1);
+              if (g == 0 && nitem < a.n_items) {
+                // tile A is done with this item: start its next item's first S
+                // now, while tile B still works on its last key tiles
+                const Item wn = decode_item<ROUTE>(a, nitem);
+                const int scn = sc + PER_TILE * (w.hi - w.lo + 1);
+                if (!q_wait(0) || !slot_wait(scn) || (ROUTE && !slot_wait(scn + 1))) { ok = false; break; }
+                ptx::tc_fence_after();
+                qk(0, scn);
+                ptx::mma_commit(bar(B_S + 0));
+                if (wn.lo0 == wn.hi0) ptx::mma_commit(bar(B_QE + 0));
+                a_started = true;
+              }
+            }
+          }
+          if (!ok) break;
+          ptx::mma_commit(bar(B_SLE + scV % SLOTS));
+          if (more) ptx::mma_commit(bar(B_SLE + scK1 % SLOTS));
+          if (ROUTE && more) ptx::mma_commit(bar(B_SLE + (scK1 + 1) % SLOTS));
         }
+        ++ic0;
+        if (w.has_b) ++ic1;
+        sc += PER_TILE * (w.hi - w.lo + 1);
       }
       if (!ok) *abort_flag = 1;
       ptx::mma_commit(bar(B_DONE));
@@ -475,81 +438,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         float mx[8];
         bool rescale;
         float mc, m_new;
-        if (OPT && t != t_lo && __all_sync(0xffffffffu, m_run != -INFINITY)) {
-          // Every row of the warp has a finite running max: the exponentials
-          // use it straight away, quarter by quarter, while the next quarter's
-          // scores come from tensor memory; the tile's max is gathered along
-          // the way.  P overwrites only scores already read.  In the rare case
-          // that a row's max grew past the threshold, the warp recomputes the
-          // tile's p from the scores kept in registers.
-          const float mc_old = m_run * c;
-          uint32_t u[32];
-          ptx::tmem_ld32(tS, u);
+        // four TMEM loads in flight behind one wait; the row max first
+        {
+          uint32_t u0[32], u1[32], u2[32], u3[32];
+          ptx::tmem_ld32(tS, u0);
+          ptx::tmem_ld32(tS + 32, u1);
+          ptx::tmem_ld32(tS + 64, u2);
+          ptx::tmem_ld32(tS + 96, u3);
           ptx::tmem_ld_wait();
 #pragma unroll
-          for (int qd = 0; qd < 4; ++qd) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int col = 32 * qd + i;
-              x[col] = (full_tile || (col >= clo && col <= chi)) ? __uint_as_float(u[i]) : -INFINITY;
-            }
-            if (qd < 3) ptx::tmem_ld32(tS + (uint32_t)(32 * (qd + 1)), u);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const float a0 = fmaxf(x[32 * qd + 4 * k], x[32 * qd + 4 * k + 1]);
-              const float a1 = max3(a0, x[32 * qd + 4 * k + 2], x[32 * qd + 4 * k + 3]);
-              mx[k] = qd == 0 ? a1 : fmaxf(mx[k], a1);
-            }
-            exp_quarter(qd, mc_old);
-            if (qd < 3) ptx::tmem_ld_wait();
+          for (int i = 0; i < 32; ++i) {
+            x[i] = __uint_as_float(u0[i]);
+            x[32 + i] = __uint_as_float(u1[i]);
+            x[64 + i] = __uint_as_float(u2[i]);
+            x[96 + i] = __uint_as_float(u3[i]);
           }
-          const float tmax = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-          rescale = (tmax - m_run) * c > kRescaleThreshold;
-          m_new = rescale ? tmax : m_run;
-          mc = rescale ? tmax * c : mc_old;
-          if (__any_sync(0xffffffffu, rescale)) {
-            ptx::tmem_st_wait();
-#pragma unroll
-            for (int k = 0; k < 4; ++k) sm[k] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int qd = 0; qd < 4; ++qd) exp_quarter(qd, mc);
-          }
-        } else {
-          // four TMEM loads in flight behind one wait; the row max first
-          {
-            uint32_t u0[32], u1[32], u2[32], u3[32];
-            ptx::tmem_ld32(tS, u0);
-            ptx::tmem_ld32(tS + 32, u1);
-            ptx::tmem_ld32(tS + 64, u2);
-            ptx::tmem_ld32(tS + 96, u3);
-            ptx::tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              x[i] = __uint_as_float(u0[i]);
-              x[32 + i] = __uint_as_float(u1[i]);
-              x[64 + i] = __uint_as_float(u2[i]);
-              x[96 + i] = __uint_as_float(u3[i]);
-            }
-          }
-          if (!full_tile) {
-#pragma unroll
-            for (int i = 0; i < 128; ++i) x[i] = (i >= clo && i <= chi) ? x[i] : -INFINITY;
-          }
-          // row max: eight chains of three-input max
-#pragma unroll
-          for (int k = 0; k < 8; ++k) mx[k] = fmaxf(x[2 * k], x[2 * k + 1]);
-#pragma unroll
-          for (int i = 16; i < 128; i += 16)
-#pragma unroll
-            for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], x[i + 2 * k], x[i + 2 * k + 1]);
-          const float tmax = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-          // lazy max (raw score units): move it only when it grows by more than 2^8 after scaling
-          rescale = (tmax - m_run) * c > kRescaleThreshold;
-          m_new = rescale ? tmax : m_run;
-          mc = (m_new == -INFINITY) ? 0.f : m_new * c;
-#pragma unroll
-          for (int qd = 0; qd < 4; ++qd) exp_quarter(qd, mc);
         }
+        if (!full_tile) {
+#pragma unroll
+          for (int i = 0; i < 128; ++i) x[i] = (i >= clo && i <= chi) ? x[i] : -INFINITY;
+        }
+        // row max: eight chains of three-input max
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(x[2 * k], x[2 * k + 1]);
+#pragma unroll
+        for (int i = 16; i < 128; i += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], x[i + 2 * k], x[i + 2 * k + 1]);
+        const float tmax = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+        // lazy max (raw score units): move it only when it grows by more than 2^8 after scaling
+        rescale = (tmax - m_run) * c > kRescaleThreshold;
+        m_new = rescale ? tmax : m_run;
+        mc = (m_new == -INFINITY) ? 0.f : m_new * c;
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) exp_quarter(qd, mc);
         const float alpha = rescale ? ex2(m_run * c - mc) : 1.f;  // 0 when m_run == -inf
         if (rescale) {
           l_run *= alpha;
@@ -584,30 +506,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++icnt;
       ptx::tc_fence_after();
       const float inv = l_run > 0.f ? 1.0f / l_run : 0.f;
-      // read all of O_g, release it to the next item's P V, then store
-      uint32_t o0[32], o1[32], o2[32], o3[32];
-      ptx::tmem_ld32(tO, o0);
-      ptx::tmem_ld32(tO + 32, o1);
-      ptx::tmem_ld32(tO + 64, o2);
-      ptx::tmem_ld32(tO + 96, o3);
-      ptx::tmem_ld_wait();
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(B_OE + g));
-      if (qi < a.T) {
-        uint4* d4 = reinterpret_cast<uint4*>(a.o + (size_t)(w.b * a.T + qi) * a.ldo + w.h * kD);
-        auto put = [&](int q0, const uint32_t (&u)[32]) {
+      // O_g is read one 32-column chunk at a time and stored; it is released
+      // to the next item's P V as soon as its last chunk is in registers
+      uint4* d4 = reinterpret_cast<uint4*>(a.o + (size_t)(w.b * a.T + qi) * a.ldo + w.h * kD);
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t u[32];
+        ptx::tmem_ld32(tO + (uint32_t)(cc * 32), u);
+        ptx::tmem_ld_wait();
+        if (cc == 3) {
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(bar(B_OE + g));
+        }
+        if (qi < a.T) {
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            d4[q0 + q] = make_uint4(pack_bf16(__uint_as_float(u[8 * q + 0]) * inv, __uint_as_float(u[8 * q + 1]) * inv),
-                                    pack_bf16(__uint_as_float(u[8 * q + 2]) * inv, __uint_as_float(u[8 * q + 3]) * inv),
-                                    pack_bf16(__uint_as_float(u[8 * q + 4]) * inv, __uint_as_float(u[8 * q + 5]) * inv),
-                                    pack_bf16(__uint_as_float(u[8 * q + 6]) * inv, __uint_as_float(u[8 * q + 7]) * inv));
-        };
-        put(0, o0);
-        put(4, o1);
-        put(8, o2);
-        put(12, o3);
+            d4[4 * cc + q] = make_uint4(pack_bf16(__uint_as_float(u[8 * q + 0]) * inv, __uint_as_float(u[8 * q + 1]) * inv),
+                                        pack_bf16(__uint_as_float(u[8 * q + 2]) * inv, __uint_as_float(u[8 * q + 3]) * inv),
+                                        pack_bf16(__uint_as_float(u[8 * q + 4]) * inv, __uint_as_float(u[8 * q + 5]) * inv),
+                                        pack_bf16(__uint_as_float(u[8 * q + 6]) * inv, __uint_as_float(u[8 * q + 7]) * inv));
+        }
       }
     }
     if (!ok) *abort_flag = 1;
@@ -647,9 +566,8 @@ bool launch_attn_common(const bf16* q, const bf16* k, const bf16* v, const bf16*
   a.scale_log2 = scale * 1.4426950408889634f;
   a.o = o;
   a.status = status;
-  static const int opt = getenv("NC_ATTN_OPT") ? atoi(getenv("NC_ATTN_OPT")) : 1;
   void (*kern)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, AttnArgs) =
-      route ? (opt ? k_attn_tc<1, true> : k_attn_tc<0, true>) : (opt ? k_attn_tc<1, false> : k_attn_tc<0, false>);
+      route ? k_attn_tc<true> : k_attn_tc<false>;
   if (!smem_optin(kern, SMEM_BYTES)) return false;
   LaunchScope scope_(KK_ATTN_TC, st);
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;

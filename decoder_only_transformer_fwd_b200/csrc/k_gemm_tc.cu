@@ -548,20 +548,18 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
 
 
 // Producers of the fused norm's input (EPI_RESID / EPI_BLOCK_END) store each
-// row's sum of squares per 32-column chunk: slot n / 32 of the row's
-// ss_parts = N / 32 slots (lane (q, 0) holds the sums of rows 4 i + q); ssr
-// is cleared for the next chunk.
-__device__ __forceinline__ void store_chunk_ss(const EpiParams& ep, const TcArgs& a, int row0, int n, int lane,
-                                               float (&ssr)[8]) {
+// row's sum of squares over the warp's c_cnt columns [n_lo, n_lo + c_cnt) in
+// slot n_lo / c_cnt of the row's ss_parts = N / c_cnt slots (lane (q, 0)
+// holds the sums of rows 4 i + q).
+__device__ __forceinline__ void store_row_ss(const EpiParams& ep, const TcArgs& a, int row0, int n_lo, int c_cnt,
+                                             int lane, const float (&ssr)[8]) {
   if (ep.ss_out != nullptr && (lane & 7) == 0) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int mr = row0 + 4 * i + (lane >> 3);
-      if (mr < a.M) ep.ss_out[(size_t)mr * ep.ss_parts + (n >> 5)] = ssr[i];
+      if (mr < a.M) ep.ss_out[(size_t)mr * ep.ss_parts + n_lo / c_cnt] = ssr[i];
     }
   }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) ssr[i] = 0.f;
 }
 
 template <int BN, int MODE>
@@ -743,12 +741,12 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs&
       }
       resid_apply(ep, a, stage, row0, n_lo + c, lane, xv, ssr);
       __syncwarp();
-      store_chunk_ss(ep, a, row0, n_lo + c, lane, ssr);
       if (c + 32 < c_cnt) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) xv[i] = xn[i];
       }
     }
+    store_row_ss(ep, a, row0, n_lo, c_cnt, lane, ssr);
   } else {
     float ssr[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     // chunk c + 1's TMEM columns are requested before chunk c is processed
@@ -763,11 +761,11 @@ __device__ __forceinline__ void epilogue_tile(const EpiParams& ep, const TcArgs&
       if (c + 32 < c_cnt) ptx::tmem_ld32(taddr + (uint32_t)(c_lo + c + 32), r);
       if constexpr (MODE == EPI_BLOCK_END) {
         epi_resid_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, rc, lane, ssr);
-        store_chunk_ss(ep, a, mb * kBM + g * 32, n_lo + c, lane, ssr);
       } else {
         epi_store_chunk(ep, a, stage, mb * kBM + g * 32, n_lo + c, rc, lane, MODE == EPI_RELU2, rscale);
       }
     }
+    if constexpr (MODE == EPI_BLOCK_END) store_row_ss(ep, a, mb * kBM + g * 32, n_lo, c_cnt, lane, ssr);
 
   }
 }
@@ -974,8 +972,7 @@ constexpr int kPairWarpTma = 8, kPairWarpMma = 9;
 constexpr int kPairRegsLow = 88, kPairRegsHigh = 208;
 static_assert(2 * 128 * kPairRegsHigh + 128 * kPairRegsLow <= kPairThreads * 168, "register split");
 
-// BN_: the pair tile's width (256; the epilogue also handles 96, whose
-// 32-column chunks the two warps of a lane quarter share unevenly).
+// BN_: the pair tile's width.
 template <int BN_>
 struct PairCfg {
   static constexpr int BN = BN_;
@@ -1136,18 +1133,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const int ew = warp;
     const int g = warp & 3;  // TMEM lane quarter
     const int half = ew >> 2;
-    // the two warps of a lane quarter split the tile's columns: halves of
-    // BN / 2, or for BN = 96 the 32-column chunks {0, 1} and {2}, the two
-    // shares swapping from one job to the next
-    auto cols = [&](int j, int& c_lo, int& c_cnt) {
-      if (BN == 96) {
-        const bool big = (j & 1) == half;
-        c_lo = big ? 0 : 64;
-        c_cnt = big ? 64 : 32;
-      } else {
-        c_lo = half * (BN / 2);
-        c_cnt = BN / 2;
-      }
+    // the two warps of a lane quarter take the two column halves of the tile
+    auto cols = [&](int, int& c_lo, int& c_cnt) {
+      c_lo = half * (BN / 2);
+      c_cnt = BN / 2;
     };
     float* stage = epi_stage + ew * Cf::STAGE_FLOATS;
     int acc = 0;

@@ -201,7 +201,7 @@ Layout layout(const nc_config& c, int max_tokens) {
   L.o = take(M * c.n_head * D * esz);
   L.h = take(M * (size_t)c.mlp_hidden * esz);
   L.gate = take(M * c.n_kv_head * 4);
-  L.ss = take(M * (C / 32) * 4);  // per-row sums of squares of the residual, one slot per 32 columns
+  L.ss = take(M * (C / 64) * 4);  // per-row sums of squares of the residual, per column group
   L.rcos = take((size_t)c.max_T * D / 2 * 4);
   L.rsin = take((size_t)c.max_T * D / 2 * 4);
   L.rfreq = take(D * 4);
@@ -390,7 +390,7 @@ int forward_impl(const nc_params* p, const int32_t* tokens, const int32_t* targe
   while ((1 << tbits) < T) ++tbits;
   launch_rope_table(rcos, rsin, T, D, c.rope_base, st, rfreq, tbits);
   float* ss = at<float>(ws, Lw.ss);
-  const int ss_parts = C / 32;  // per-row sums of squares, one slot per 32-column chunk
+  const int ss_parts = C / (gemm_tc_bn(C) / 2);  // per-row sums of squares, one slot per epilogue warp's columns
   bf16* xb = tc ? static_cast<bf16*>(xn) : nullptr;
   launch_embed(p->wte, tokens, p->smear_gate, c.smear && c.gate_channels > 0, c.gate_channels,
                p->resid_lambdas, p->x0_lambdas, c.eps, B, T, C, V, bf, x, x0, xb, tc ? ss : nullptr,
@@ -620,7 +620,7 @@ int nc_head_backward(const nc_params* p, const int32_t* targets, int B, int T, f
   const bf16* xb = at<bf16>(ws, Lw.xn);        // bf16(x) of the final residual, the head's A operand
   const float* x = at<float>(ws, Lw.x);        // the final residual (after backout), fp32
   const float* ss = at<float>(ws, Lw.ss);      // its row sums of squares, per column group
-  const int ss_parts = C / 32;  // per-row sums of squares, one slot per 32-column chunk
+  const int ss_parts = C / (gemm_tc_bn(C) / 2);  // per-row sums of squares, one slot per epilogue warp's columns
   launch_inv_count(targets, M, inv_count, st);
   // dz' = (1/rms) dL/dz: the head GEMM recomputed, the CE gradient in its epilogue
   EpiParams e = epi(EPI_DZ);
