@@ -59,11 +59,14 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kThreads = 384;
 constexpr int kWarpTma = 8, kWarpMma = 9;
 // registers: launched at 168 per thread (65536 / 384, rounded down to 8);
-// the TMA/MMA warpgroup drops to 136 and the two softmax warpgroups rise to
-// 184: 2 * 128 * 184 + 128 * 136 = 64512 = 384 * 168 (the split at which the
-// compiler spills least: 104 / 200 spilled in the MMA issuer)
-constexpr int kRegsLow = 136, kRegsHigh = 184;
-static_assert(2 * 128 * kRegsHigh + 128 * kRegsLow <= kThreads * 168, "register split");
+// the TMA/MMA warpgroup drops to kRegsLow and the two softmax warpgroups rise
+// to kRegsHigh, 2 * 128 * kRegsHigh + 128 * kRegsLow <= 64512 = 384 * 168.
+// The splits are those at which the compiler spills nothing (base attention:
+// 120 / 192) or least (routing, with its second Q operand: 144 / 176).
+template <bool ROUTE> constexpr int kRegsLow = ROUTE ? 144 : 120;
+template <bool ROUTE> constexpr int kRegsHigh = ROUTE ? 176 : 192;
+static_assert(2 * 128 * kRegsHigh<false> + 128 * kRegsLow<false> <= kThreads * 168, "register split");
+static_assert(2 * 128 * kRegsHigh<true> + 128 * kRegsLow<true> <= kThreads * 168, "register split");
 
 struct AttnArgs {
   int B, T, H, Hkv, window;
@@ -204,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto sSlot = [&](int s) { return ptx::smem_u32(smem + OFF_SLOT + s * TILE_BYTES); };
 
   if (warp >= 8) {
-    ptx::setmaxnreg_dec<kRegsLow>();
+    ptx::setmaxnreg_dec<kRegsLow<ROUTE>>();
     if (warp == kWarpTma) {
     if (ptx::elect_one()) {
       // ---------------- TMA producer ----------------
@@ -391,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     }
   } else {
-    ptx::setmaxnreg_inc<kRegsHigh>();
+    ptx::setmaxnreg_inc<kRegsHigh<ROUTE>>();
     // ---------------- softmax + epilogue: group 0 = warps 0..3, group 1 = warps 4..7 ----------------
     const int g = warp >> 2;
     const int gq = warp & 3;
@@ -454,24 +457,63 @@ __global__ void __launch_bounds__(kThreads, 1)
             x[96 + i] = __uint_as_float(u3[i]);
           }
         }
-        if (!full_tile) {
+        // A warp whose 32 rows see every key of the tile takes the plain path.
+        // Otherwise masking is decided per 32-key quarter for the whole warp
+        // (its rows' visible ranges are consecutive): a quarter that every row
+        // sees needs no select, one that no row sees gets P = 0 without its
+        // exponentials, and only the quarters between take per-key selects.
+        const bool warp_full = __all_sync(0xffffffffu, full_tile);
+        unsigned vis = 0xFu;  // bit qd: some row sees quarter qd
+        if (warp_full) {
+          // row max: eight chains of three-input max
 #pragma unroll
-          for (int i = 0; i < 128; ++i) x[i] = (i >= clo && i <= chi) ? x[i] : -INFINITY;
+          for (int k = 0; k < 8; ++k) mx[k] = fmaxf(x[2 * k], x[2 * k + 1]);
+#pragma unroll
+          for (int i = 16; i < 128; i += 16)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], x[i + 2 * k], x[i + 2 * k + 1]);
+        } else {
+          const int lo_min = __reduce_min_sync(0xffffffffu, clo), lo_max = __reduce_max_sync(0xffffffffu, clo);
+          const int hi_min = __reduce_min_sync(0xffffffffu, chi), hi_max = __reduce_max_sync(0xffffffffu, chi);
+          vis = 0u;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd) {
+            const int b0 = 32 * qd, b1 = 32 * qd + 31;
+            if (b1 < lo_min || b0 > hi_max) continue;  // no row sees this quarter
+            vis |= 1u << qd;
+            if (!(b0 >= lo_max && b1 <= hi_min)) {     // some row sees only part of it
+#pragma unroll
+              for (int i = 32 * qd; i < 32 * qd + 32; ++i) x[i] = (i >= clo && i <= chi) ? x[i] : -INFINITY;
+            }
+#pragma unroll
+            for (int i = 32 * qd; i < 32 * qd + 32; i += 16)
+#pragma unroll
+              for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], x[i + 2 * k], x[i + 2 * k + 1]);
+          }
         }
-        // row max: eight chains of three-input max
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(x[2 * k], x[2 * k + 1]);
-#pragma unroll
-        for (int i = 16; i < 128; i += 16)
-#pragma unroll
-          for (int k = 0; k < 8; ++k) mx[k] = max3(mx[k], x[i + 2 * k], x[i + 2 * k + 1]);
         const float tmax = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
         // lazy max (raw score units): move it only when it grows by more than 2^8 after scaling
         rescale = (tmax - m_run) * c > kRescaleThreshold;
         m_new = rescale ? tmax : m_run;
         mc = (m_new == -INFINITY) ? 0.f : m_new * c;
+        if (warp_full) {
 #pragma unroll
-        for (int qd = 0; qd < 4; ++qd) exp_quarter(qd, mc);
+          for (int qd = 0; qd < 4; ++qd) exp_quarter(qd, mc);
+        } else {
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd) {
+            if (vis & (1u << qd)) {
+              exp_quarter(qd, mc);
+            } else {
+              uint32_t z[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) z[i] = 0u;
+              ptx::tmem_st16(tS + (uint32_t)(16 * qd), z);
+            }
+          }
+        }
         const float alpha = rescale ? ex2(m_run * c - mc) : 1.f;  // 0 when m_run == -inf
         if (rescale) {
           l_run *= alpha;
