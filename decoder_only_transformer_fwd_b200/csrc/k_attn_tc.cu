@@ -71,6 +71,7 @@ static_assert(2 * 128 * kRegsHigh<true> + 128 * kRegsLow<true> <= kThreads * 168
 struct AttnArgs {
   int B, T, H, Hkv, window;
   int ldo;
+  int o_v8;  // o is 32-byte aligned and ldo a multiple of 16: 32-byte stores
   int n_qblocks, n_pairs, n_items;
   float scale_log2;  // softmax_scale * log2(e)
   bf16* o;
@@ -562,12 +563,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) ptx::mbar_arrive(bar(B_OE + g));
         }
         if (qi < a.T) {
+          // each thread writes its own row: whole 32-byte sectors when the
+          // layout allows, else 16-byte halves
+          if (a.o_v8) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            d4[4 * cc + q] = make_uint4(pack_bf16(__uint_as_float(u[8 * q + 0]) * inv, __uint_as_float(u[8 * q + 1]) * inv),
-                                        pack_bf16(__uint_as_float(u[8 * q + 2]) * inv, __uint_as_float(u[8 * q + 3]) * inv),
-                                        pack_bf16(__uint_as_float(u[8 * q + 4]) * inv, __uint_as_float(u[8 * q + 5]) * inv),
-                                        pack_bf16(__uint_as_float(u[8 * q + 6]) * inv, __uint_as_float(u[8 * q + 7]) * inv));
+            for (int hh = 0; hh < 2; ++hh) {
+              uint32_t wv[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                wv[e] = pack_bf16(__uint_as_float(u[16 * hh + 2 * e]) * inv, __uint_as_float(u[16 * hh + 2 * e + 1]) * inv);
+              ptx::st_global_v8(d4 + 4 * cc + 2 * hh, wv);
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              d4[4 * cc + q] = make_uint4(pack_bf16(__uint_as_float(u[8 * q + 0]) * inv, __uint_as_float(u[8 * q + 1]) * inv),
+                                          pack_bf16(__uint_as_float(u[8 * q + 2]) * inv, __uint_as_float(u[8 * q + 3]) * inv),
+                                          pack_bf16(__uint_as_float(u[8 * q + 4]) * inv, __uint_as_float(u[8 * q + 5]) * inv),
+                                          pack_bf16(__uint_as_float(u[8 * q + 6]) * inv, __uint_as_float(u[8 * q + 7]) * inv));
+          }
         }
       }
     }
@@ -602,6 +616,7 @@ bool launch_attn_common(const bf16* q, const bf16* k, const bf16* v, const bf16*
   a.Hkv = Hkv;
   a.window = (window <= 0 || window > T) ? T : window;
   a.ldo = ldo;
+  a.o_v8 = (reinterpret_cast<uintptr_t>(o) % 32 == 0) && (ldo % 16 == 0);
   a.n_qblocks = (T + kQ - 1) / kQ;
   a.n_pairs = route ? a.n_qblocks : (a.n_qblocks + 1) / 2;
   a.n_items = a.n_pairs * B * H;
