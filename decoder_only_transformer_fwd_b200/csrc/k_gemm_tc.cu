@@ -423,6 +423,9 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
   if (col0 < ep.qk_cols) {
     const int t_lane = (m0 + lane) % ep.T;
     const int fp = lane & 7, rsub = lane >> 3;  // lane -> (frequency pair, row within a group of 4)
+    // the warp's 32 rows are 32 consecutive positions of one sequence
+    const bool lin = (m0 % ep.T) + 31 < ep.T;
+    const int t_first = (m0 % ep.T) + rsub;
     // RoPE pairs (j, j + 64) preserve each pair's sum of squares, so the RMS
     // comes from the raw accumulator in a first pass
     float ssa = 0.f, ssb = 0.f;
@@ -464,17 +467,13 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
       // hardware sine / cosine within [-pi, pi])
       const float fh0 = __ldg(ep.rope_fsplit + f0), fh1 = __ldg(ep.rope_fsplit + f0 + 1);
       const float fl0 = __ldg(ep.rope_fsplit + 64 + f0), fl1 = __ldg(ep.rope_fsplit + 64 + f0 + 1);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int rr = 4 * i + rsub;
-        const float rs = __shfl_sync(0xffffffffu, rs_lane, rr);
-        const float tf = (float)__shfl_sync(0xffffffffu, t_lane, rr);
-        float p0 = tf * fh0, p1 = tf * fh1;  // exact
-        p0 = fmaf(tf, fl0, p0 - floorf(p0));
-        p1 = fmaf(tf, fl1, p1 - floorf(p1));
-        p0 = (p0 - rintf(p0)) * 6.2831853071795865f;
-        p1 = (p1 - rintf(p1)) * 6.2831853071795865f;
-        const float c0 = __cosf(p0), s0 = __sinf(p0), c1 = __cosf(p1), s1 = __sinf(p1);
+      // angle 2 pi (t f mod 1) of position t, |angle| <= pi
+      auto angle = [&](float tf, float fh, float fl) {
+        float ph = tf * fh;  // exact
+        ph = fmaf(tf, fl, ph - floorf(ph));
+        return (ph - rintf(ph)) * 6.2831853071795865f;
+      };
+      auto rotate_store = [&](int rr, float rs, float c0, float s0, float c1, float s1) {
         const float a1x = stage[rr * 33 + 2 * fp], a1y = stage[rr * 33 + 2 * fp + 1];
         const float a2x = stage[rr * 33 + 16 + 2 * fp], a2y = stage[rr * 33 + 16 + 2 * fp + 1];
         if (m0 + rr < a.M) {
@@ -483,6 +482,36 @@ __device__ __forceinline__ void epi_qkv_head(const EpiParams& ep, const TcArgs& 
                                                                         (a1y * c1 + a2y * s1) * rs);
           *reinterpret_cast<__nv_bfloat162*>(o + 64) = __floats2bfloat162_rn((-a1x * s0 + a2x * c0) * rs,
                                                                              (-a1y * s1 + a2y * c1) * rs);
+        }
+      };
+      if (lin) {
+        // this lane's rows 4 i + rsub sit at positions t_first + 4 i: one
+        // angle from the hardware sine / cosine, then exact-angle steps of
+        // 4 f by rotation (7 steps add ~1e-6 to the ~4e-7 of the first angle)
+        const float tf = (float)t_first;
+        const float q0 = angle(tf, fh0, fl0), q1 = angle(tf, fh1, fl1);
+        const float d0 = angle(4.0f, fh0, fl0), d1 = angle(4.0f, fh1, fl1);
+        float c0 = __cosf(q0), s0 = __sinf(q0), c1 = __cosf(q1), s1 = __sinf(q1);
+        const float dc0 = __cosf(d0), ds0 = __sinf(d0), dc1 = __cosf(d1), ds1 = __sinf(d1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + rsub;
+          rotate_store(rr, __shfl_sync(0xffffffffu, rs_lane, rr), c0, s0, c1, s1);
+          const float c0n = fmaf(c0, dc0, -s0 * ds0), s0n = fmaf(s0, dc0, c0 * ds0);
+          const float c1n = fmaf(c1, dc1, -s1 * ds1), s1n = fmaf(s1, dc1, c1 * ds1);
+          c0 = c0n;
+          s0 = s0n;
+          c1 = c1n;
+          s1 = s1n;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + rsub;
+          const float rs = __shfl_sync(0xffffffffu, rs_lane, rr);
+          const float tf = (float)__shfl_sync(0xffffffffu, t_lane, rr);
+          const float p0 = angle(tf, fh0, fl0), p1 = angle(tf, fh1, fl1);
+          rotate_store(rr, rs, __cosf(p0), __sinf(p0), __cosf(p1), __sinf(p1));
         }
       }
       __syncwarp();

@@ -44,3 +44,35 @@ def test_rope_phase_split_is_exact_enough():
             err = np.abs(((got - exact) + 0.5) % 1.0 - 0.5)
             worst = max(worst, err.max())
         assert worst < 2e-7, (T, worst)
+
+
+def _f32_fma(a, b, c):
+    """fma in float32: one rounding of the exact a * b + c."""
+    return F32(np.float64(a) * np.float64(b) + np.float64(c))
+
+
+def test_rope_angle_steps_by_rotation():
+    """Where a warp's 32 rows are 32 consecutive positions, the QKV epilogue
+    takes each lane's first angle (rows 4 i + r, i = 0..7) from the phase
+    above and reaches the next seven by rotating with cos / sin of the exact
+    step 4 f (two fmas per component).  Modelled here with float32 products
+    and float32 fmas, cosine / sine of the float32 angles in float64 (the
+    hardware adds ~4e-7 to each); the seven steps must stay within 2e-6 of the
+    exact cos / sin of 2 pi t f, far below bf16's 2^-9."""
+    worst = 0.0
+    for T in (2048, 8192):
+        tbits = int(np.ceil(np.log2(T)))
+        f, fh, fl = split_freqs(1e5, 128, tbits)
+        for t0 in (0, 4, T // 2 + 1, T - 32):
+            q = (phase_turns(t0, fh, fl) * F32(2 * np.pi)).astype(F32)
+            d = (phase_turns(4, fh, fl) * F32(2 * np.pi)).astype(F32)
+            c, s = np.cos(q.astype(np.float64)).astype(F32), np.sin(q.astype(np.float64)).astype(F32)
+            dc, ds = np.cos(d.astype(np.float64)).astype(F32), np.sin(d.astype(np.float64)).astype(F32)
+            for i in range(8):
+                t = t0 + 4 * i
+                ang = 2 * np.pi * ((t * f) % 1.0)
+                worst = max(worst, np.abs(c - np.cos(ang)).max(), np.abs(s - np.sin(ang)).max())
+                cn = np.array([_f32_fma(a, b, -F32(x * y)) for a, b, x, y in zip(c, dc, s, ds)], dtype=F32)
+                sn = np.array([_f32_fma(a, b, F32(x * y)) for a, b, x, y in zip(s, dc, c, ds)], dtype=F32)
+                c, s = cn, sn
+    assert worst < 2e-6, worst
