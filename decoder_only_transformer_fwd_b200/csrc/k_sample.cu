@@ -52,12 +52,15 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   return d;
 }
 
-// k_last_logits: warps 0..15 multiply (two groups of 8 that take alternate
-// stages), warp 16 streams W_U into the ring
-constexpr int kLastGroupWarps = 8;
+// k_last_logits: warps 0..7 multiply (two groups of 4 that take alternate
+// stages), warp 8 streams W_U into the ring.  Each consumer warp multiplies
+// four vocabulary rows together, so every staged x value read from shared
+// memory serves four rows (shared-memory traffic, not HBM, bounded the
+// two-row form).
+constexpr int kLastGroupWarps = 4;
 constexpr int kLastConsumers = 2 * kLastGroupWarps;
 constexpr int kLastThreads = 32 * (kLastConsumers + 1);
-constexpr int kLastR = 2;  // vocabulary rows a consumer warp multiplies together
+constexpr int kLastR = 4;  // vocabulary rows a consumer warp multiplies together
 
 // The ring geometry for rows of `row_bytes`: kLastGroupWarps * kLastR rows
 // per stage, 4 or 2 stages, as fit next to the staged x rows (fp32).
@@ -119,7 +122,8 @@ k_last_logits(const float* __restrict__ x, int ldx, int T, int b0, const TW* __r
   constexpr int kN = Chunk<TW>::kN;  // elements of a 16-byte chunk of W_U
   constexpr int kH = kN / 4;         // float4s of x per chunk
   constexpr int kNV = NB <= 4 ? 4 : 8;
-  constexpr int kK = NB <= 4 ? 3 : 4;  // log2(kLastR * kNV)
+  constexpr int kK = NB <= 4 ? 4 : 5;  // log2(kLastR * kNV)
+  static_assert((1 << kK) == kLastR * kNV, "one value per (row, x row) slot");
   constexpr int rows = kLastGroupWarps * kLastR;
   extern __shared__ __align__(16) unsigned char sh_raw[];
   const size_t row_bytes = (size_t)C * sizeof(TW);
@@ -199,9 +203,11 @@ k_last_logits(const float* __restrict__ x, int ldx, int T, int b0, const TW* __r
     const int r0 = blk * rows;
     const int nr = V - r0 < rows ? V - r0 : rows;
     if (r < nr) {
-      const bool two = r + 1 < nr;
-      const uint4* w0 = reinterpret_cast<const uint4*>(ring + s * stage_bytes + (size_t)r * row_bytes);
-      const uint4* w1 = reinterpret_cast<const uint4*>(ring + s * stage_bytes + (size_t)(two ? r + 1 : r) * row_bytes);
+      const int nq = nr - r < kLastR ? nr - r : kLastR;  // rows of this warp inside the block
+      const uint4* wr[kLastR];
+#pragma unroll
+      for (int q = 0; q < kLastR; ++q)  // rows past the block's end repeat row r (their sums are dropped)
+        wr[q] = reinterpret_cast<const uint4*>(ring + s * stage_bytes + (size_t)(r + (q < nq ? q : 0)) * row_bytes);
       float2 acc[kLastR][NB];
 #pragma unroll
       for (int q = 0; q < kLastR; ++q)
@@ -210,8 +216,8 @@ k_last_logits(const float* __restrict__ x, int ldx, int T, int b0, const TW* __r
 #pragma unroll 2
       for (int ci = lane; ci < nchunks; ci += 32) {
         float2 wf[kLastR][kN / 2];
-        Chunk<TW>::unpack(w0[ci], wf[0]);
-        Chunk<TW>::unpack(w1[ci], wf[1]);
+#pragma unroll
+        for (int q = 0; q < kLastR; ++q) Chunk<TW>::unpack(wr[q][ci], wf[q]);
 #pragma unroll
         for (int j = 0; j < NB; ++j) {
 #pragma unroll
@@ -237,7 +243,7 @@ k_last_logits(const float* __restrict__ x, int ldx, int T, int b0, const TW* __r
       for (int rr = 0; rr < kK; ++rr) vi |= ((lane >> (4 - rr)) & 1) << (kK - 1 - rr);
       const int q = vi / kNV, j = vi % kNV;
       const bool writer = (lane & ((1 << (5 - kK)) - 1)) == 0;
-      if (writer && j < NB && (q == 0 || two))
+      if (writer && j < NB && q < nq)
         out[(size_t)(b0 + j) * ldo + r0 + r + q] = cap * tanhf(tot * rs[j] / cap);
     }
     __syncwarp();
