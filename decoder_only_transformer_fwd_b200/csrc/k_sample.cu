@@ -112,7 +112,7 @@ __device__ __forceinline__ float warp_reduce_many(float (&a)[1 << K], int lane) 
 // consecutive vocabulary rows c, c + G, c + 2G, ...  One thread copies each
 // block (contiguous in W_U) into a ring of shared-memory stages with a bulk
 // copy; the two groups of consumer warps take alternate blocks, each warp
-// multiplies two rows against the staged x rows, and the group releases the
+// multiplies four rows against the staged x rows, and the group releases the
 // stage.
 template <typename TW, int NB>
 __global__ void __launch_bounds__(kLastThreads, 1)
