@@ -300,6 +300,60 @@ def routing_sweep(args, dev, stream, peaks):
     return out
 
 
+def nested_step(args, dev, stream, peaks):
+    """The StairFormer nesting pieces at the README's d24 widths (384 + 1152,
+    C = 1536) over M = 8192 rows: PrefixRMSNorm (bytes: x read, bf16 out
+    written), the block lower triangular linear map C -> C (algorithmic FLOPs
+    of the live blocks only: 2 M sum_a w_a C_a) and the prefix cross-entropy
+    of both submodels at V = 32768 (2 M V (C_1 + C_2) FLOPs)."""
+    import numpy as np
+    import torch
+
+    from decoder_only_transformer_fwd_b200 import nc, synth
+    widths, M, V = [384, 1152], 8192, 32768
+    Cw = sum(widths)
+    x, w, w_u, y = synth.nested_inputs(synth.SEED_BASE + 90, M, Cw, Cw, V, V)
+    ends = np.cumsum(widths)
+    for a in range(len(widths)):  # dead blocks of the BTL weight are zero
+        w[ends[a] - widths[a]:ends[a], ends[a]:] = 0.0
+    xd = torch.from_numpy(x).to(dev)
+    xb = xd.to(torch.bfloat16)
+    wd = torch.from_numpy(w).to(dev).to(torch.bfloat16)
+    wud = torch.from_numpy(w_u).to(dev).to(torch.bfloat16)
+    yd = torch.from_numpy(y).to(dev)
+    xn = torch.empty(M, Cw, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(M, Cw, dtype=torch.float32, device=dev)
+    loss = torch.empty(len(widths), M, dtype=torch.float32, device=dev)
+    ws = torch.empty(int(nc.lib().nc_prefix_ce_workspace_bytes(M, Cw, V)), dtype=torch.uint8, device=dev)
+    res = {"workload": "StairFormer nesting pieces, widths 384 + 1152 (C = 1536), M = 8192, V = 32768"}
+
+    def timed(call):
+        for _ in range(3):
+            call()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(args.steps):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return 1e3 * e0.elapsed_time(e1) / args.steps  # microseconds per call
+
+    us = timed(lambda: nc.nc_prefix_rmsnorm(xd, widths, xn, stream=stream))
+    nbytes = M * Cw * (4 + 2)
+    res["prefix_rmsnorm"] = {"us": us, "bytes": nbytes, "achieved_gbs": nbytes / (us * 1e-6) / 1e9,
+                             "frac": nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"]}
+    us = timed(lambda: nc.nc_btl_linear(xb, wd, out, widths, widths, stream=stream))
+    f = 2.0 * M * sum(int(wa) * int(ea) for wa, ea in zip(widths, ends))
+    res["btl_linear"] = {"us": us, "gflop": f / 1e9, "tflops": f / (us * 1e-6) / 1e12,
+                         "dense_gflop": 2.0 * M * Cw * Cw / 1e9}
+    us = timed(lambda: nc.nc_prefix_ce(xd, wud, yd, loss, V, widths, workspace=ws, stream=stream))
+    f = 2.0 * M * V * float(sum(ends))
+    res["prefix_ce"] = {"us": us, "gflop": f / 1e9, "tflops": f / (us * 1e-6) / 1e12,
+                        "pct_bf16_peak": 100.0 * f / (us * 1e-6) / 1e12 / peaks["bf16_tflops"]}
+    return res
+
+
 def generation_step(args, model, cfg, tok, B, T, stream, peaks):
     """One generation step at the bench workload's sizes (nc_generate_next):
     the forward over [B, T], the last-position logits, one token per row drawn
@@ -448,10 +502,11 @@ def run_ours(args):
     gen = None
     if not args.no_generation:
         gen = generation_step(args, model, cfg, tok, B, T, stream, load_peaks()[0])
-    bwd = route = None
+    bwd = route = nest = None
     if not args.no_variants:
         bwd = head_backward_step(args, model, cfg, tok, tgt, M, stream, load_peaks()[0])
         route = routing_sweep(args, dev, stream, load_peaks()[0])
+        nest = nested_step(args, dev, stream, load_peaks()[0])
     clk = clocks.stop()
     rc, bits = nc.nc_get_status(stream)
     if rc != 0:
@@ -545,6 +600,7 @@ def run_ours(args):
             "generation": gen,
             "head_backward": bwd,
             "routing_attention": route,
+            "nested": nest,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -70,7 +70,26 @@ struct TcArgs {
   unsigned sk_gen;
   unsigned sk_expect;
   unsigned long long sk_wait_ns;
+  // pair kernel, block lower triangular B (kl_k > 0): output columns below
+  // kl_out_end[a] read only the first kl_in_end[a] elements of K, so a column
+  // tile's contraction stops after the K prefix its last column reads
+  int kl_k;
+  int kl_out_end[kMaxPrefixBlocks];
+  int kl_in_end[kMaxPrefixBlocks];
 };
+
+// The k-blocks a pair column tile nb (width bn) contracts over: all of K, or
+// with a block lower triangular B the prefix its last column reads.
+__device__ __forceinline__ int tile_kb_end(const TcArgs& a, int nb, int bn, int nk) {
+  if (a.kl_k <= 0) return nk;
+  const int lc = min(a.N, (nb + 1) * bn) - 1;
+  int kend = a.K;
+#pragma unroll
+  for (int i = kMaxPrefixBlocks - 1; i >= 0; --i)
+    if (i < a.kl_k && a.kl_out_end[i] > lc) kend = a.kl_in_end[i];
+  const int kb = (kend + kBK - 1) / kBK;
+  return kb < nk ? kb : nk;
+}
 
 // Pair tile pt -> (row-pair block, column tile).  Column-fastest order keeps
 // the A rows that the CTAs of one wave share few enough to stay in L2 (for
@@ -1088,6 +1107,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         job_at(sched, j, pt, kb_lo, kb_hi, kind);
         int mbp, nb;
         pair_tile(a, pt, tiles_mp, mbp, nb);
+        kb_hi = min(kb_hi, tile_kb_end(a, nb, BN, nk));
         bool ok = true;
         for (int kb = kb_lo; kb < kb_hi; ++kb) {
           if (*abort_flag || !ptx::mbar_wait_cluster(empty(stage), ph ^ 1, a.status)) {
@@ -1121,6 +1141,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       for (int j = 0; j < sched.njobs; ++j) {
         int pt, kb_lo, kb_hi, kind;
         job_at(sched, j, pt, kb_lo, kb_hi, kind);
+        {
+          int mbp, nb;
+          pair_tile(a, pt, tiles_mp, mbp, nb);
+          kb_hi = min(kb_hi, tile_kb_end(a, nb, BN, nk));
+        }
         if (*abort_flag || !ptx::mbar_wait_cluster(tempty(acc), aph ^ 1, a.status)) {
           *abort_flag = 1;
           break;
@@ -1325,6 +1350,7 @@ bool launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const TcArgs& a, 
     case EPI_BLOCK_END: return launch_pair_mode<EPI_BLOCK_END>(ta, tb, a, ep, nclusters, st);
     case EPI_CE: return launch_pair_mode<EPI_CE>(ta, tb, a, ep, nclusters, st);
     case EPI_QKV: return launch_pair_mode<EPI_QKV>(ta, tb, a, ep, nclusters, st);
+    case EPI_F32: return launch_pair_mode<EPI_F32>(ta, tb, a, ep, nclusters, st);
     default: return false;
   }
 }
@@ -1403,7 +1429,7 @@ bool launch_gemm_tc_layout(const bf16* A, int lda, int a_mn, const bf16* Bm, int
 
 bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int N, int K,
                     const EpiParams& ep, int* status, int num_sms, cudaStream_t st, bool pair,
-                    const StreamK* sk) {
+                    const StreamK* sk, const GemmKLimit* kl) {
   const int BN = gemm_tc_bn(N);
   if (pair && BN == 256 && num_sms >= 2) {
     // CTA pairs: each CTA loads 128 rows of A and 128 rows of B per k-slice.
@@ -1416,6 +1442,7 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
     if (!make_tmap_2d(&ta, A, M, K, lda, kBM, kBK)) return false;
     if (!make_tmap_2d(&tb, Bm, N, K, ldb, bnp / 2, kBK)) return false;
     TcArgs a;
+    memset(&a, 0, sizeof(a));
     a.M = M;
     a.N = N;
     a.K = K;
@@ -1447,6 +1474,14 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
       flag_wait_test(&a.sk_wait_ns, &skew);
       a.sk_expect = sk->gen + skew;
     }
+    a.kl_k = 0;
+    if (kl != nullptr && !a.streamk) {
+      a.kl_k = kl->out.k;
+      for (int i = 0; i < kMaxPrefixBlocks; ++i) {
+        a.kl_out_end[i] = i < kl->out.k ? kl->out.end[i] : 0;
+        a.kl_in_end[i] = i < kl->in.k ? kl->in.end[i] : 0;
+      }
+    }
     LaunchScope scope_(KK_GEMM_TC, st);
     return launch_pair(ta, tb, a, ep, ncl, st, bnp);
   }
@@ -1454,6 +1489,7 @@ bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int 
   if (!make_tmap_2d(&ta, A, M, K, lda, kBM, kBK)) return false;
   if (!make_tmap_2d(&tb, Bm, N, K, ldb, BN, kBK)) return false;
   TcArgs a;
+  memset(&a, 0, sizeof(a));
   a.M = M;
   a.N = N;
   a.K = K;

@@ -579,6 +579,57 @@ __global__ void k_rmsnorm_bwd(const float* __restrict__ x, const float* __restri
   }
 }
 
+// PrefixRMSNorm ("Fully Nested Transformers" README: normalisation that does
+// not leak information backward down the hierarchy): block a of row m, the
+// columns [end[a-1], end[a]), is divided by the RMS of the row's prefix
+// [0, end[a]).  One warp per row: the prefix sums of squares first (16-byte
+// loads, one warp reduction per block), then every block scaled and stored.
+template <typename TO>
+__global__ void k_prefix_rmsnorm(const float* __restrict__ x, int M, int C, PrefixBlocks pb, float eps,
+                                 TO* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (m >= M) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)m * C);
+  float inv[kMaxPrefixBlocks];
+  float cum = 0.f;
+  int c0 = 0;
+#pragma unroll
+  for (int a = 0; a < kMaxPrefixBlocks; ++a) {
+    if (a < pb.k) {
+      float ss = 0.f;
+      for (int i = c0 / 4 + lane; i < pb.end[a] / 4; i += 32) {
+        const float4 v = xr[i];
+        ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+      }
+      cum += warp_sum(ss);
+      inv[a] = rsqrtf(cum / (float)pb.end[a] + eps);
+      c0 = pb.end[a];
+    }
+  }
+  c0 = 0;
+#pragma unroll
+  for (int a = 0; a < kMaxPrefixBlocks; ++a) {
+    if (a < pb.k) {
+      const float r = inv[a];
+      for (int i = c0 / 4 + lane; i < pb.end[a] / 4; i += 32) {
+        const float4 v = xr[i];
+        const float4 y = make_float4(v.x * r, v.y * r, v.z * r, v.w * r);
+        if constexpr (sizeof(TO) == 2) {
+          const __nv_bfloat162 b0 = __floats2bfloat162_rn(y.x, y.y), b1 = __floats2bfloat162_rn(y.z, y.w);
+          reinterpret_cast<uint2*>(out + (size_t)m * C)[i] =
+              make_uint2(*reinterpret_cast<const uint32_t*>(&b0), *reinterpret_cast<const uint32_t*>(&b1));
+        } else {
+          reinterpret_cast<float4*>(out + (size_t)m * C)[i] = y;
+        }
+      }
+      c0 = pb.end[a];
+    }
+  }
+}
+
 // Mean of loss over valid targets, fixed reduction order (deterministic).
 __global__ void k_loss_mean(const float* loss, const int32_t* targets, int n, float* out) {
   pdl_launch_dependents();
@@ -738,6 +789,17 @@ void launch_rmsnorm_bwd(const float* x, const float* g, float* dx, int M, int C,
   LaunchScope scope_(KK_HEAD_BWD_ROWS, st);
   const int wpb = 8;
   launch_pdl(k_rmsnorm_bwd, dim3((M + wpb - 1) / wpb), dim3(wpb * 32), 0, st, 1, x, g, dx, M, C, eps);
+}
+
+void launch_prefix_rmsnorm(const float* x, int M, int C, const PrefixBlocks& pb, float eps, void* out, int out_bf16,
+                           cudaStream_t st) {
+  LaunchScope scope_(KK_PREFIX_NORM, st);
+  constexpr int wpb = 8;
+  const dim3 grid((M + wpb - 1) / wpb), block(wpb * 32);
+  if (out_bf16)
+    launch_pdl(k_prefix_rmsnorm<bf16>, grid, block, 0, st, 1, x, M, C, pb, eps, static_cast<bf16*>(out));
+  else
+    launch_pdl(k_prefix_rmsnorm<float>, grid, block, 0, st, 1, x, M, C, pb, eps, static_cast<float*>(out));
 }
 
 void launch_loss_mean(const float* loss, const int32_t* targets, int n, float* out, cudaStream_t st) {

@@ -745,6 +745,112 @@ int nc_routing_attention(const void* q2, const void* k2, const void* v2, const v
   return check_launch("nc_routing_attention");
 }
 
+}  // extern "C"
+
+namespace {
+
+// Nested block widths -> cumulative ends; false unless 1 <= k <= 8, every
+// width a positive multiple of 64 and their sum C.
+bool prefix_blocks(const int* widths, int k, int C, PrefixBlocks* pb) {
+  if (widths == nullptr || k < 1 || k > kMaxPrefixBlocks) return false;
+  memset(pb, 0, sizeof(*pb));
+  pb->k = k;
+  int e = 0;
+  for (int a = 0; a < k; ++a) {
+    if (widths[a] <= 0 || widths[a] % 64 != 0) return false;
+    e += widths[a];
+    pb->end[a] = e;
+  }
+  return e == C;
+}
+
+}  // namespace
+
+extern "C" {
+
+int nc_prefix_rmsnorm(const float* x, int M, int C, const int* widths, int k, float eps, void* out, int out_bf16,
+                      void* stream) {
+  t_launches = 0;
+  if (x == nullptr || out == nullptr || !(eps >= 0.f)) return NC_ERR_ARG;
+  PrefixBlocks pb;
+  if (M < 0 || C <= 0 || !prefix_blocks(widths, k, C, &pb)) return NC_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(out)) return NC_ERR_ALIGN;
+  if (M == 0) return NC_OK;
+  launch_prefix_rmsnorm(x, M, C, pb, eps, out, out_bf16, static_cast<cudaStream_t>(stream));
+  return check_launch("nc_prefix_rmsnorm");
+}
+
+int nc_btl_linear(const void* x, const void* w, float* y, int M, int C_in, int C_out, const int* in_widths,
+                  const int* out_widths, int k, void* stream) {
+  t_launches = 0;
+  if (x == nullptr || w == nullptr || y == nullptr) return NC_ERR_ARG;
+  GemmKLimit kl;
+  if (M < 0 || C_in <= 0 || C_out <= 0 || C_out % 256 != 0 || !prefix_blocks(in_widths, k, C_in, &kl.in) ||
+      !prefix_blocks(out_widths, k, C_out, &kl.out))
+    return NC_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return NC_ERR_ALIGN;
+  if (M == 0) return NC_OK;
+  DevInfo d;
+  if (!dev_info(&d)) return NC_ERR_CUDA;
+  EpiParams e;
+  memset(&e, 0, sizeof(e));
+  e.mode = EPI_F32;
+  e.out = y;
+  e.ldo = C_out;
+  if (!launch_gemm_tc(static_cast<const bf16*>(x), C_in, static_cast<const bf16*>(w), C_in, M, C_out, C_in, e,
+                      d.status, d.num_sms, static_cast<cudaStream_t>(stream), true, nullptr, &kl))
+    return NC_ERR_CUDA;
+  return check_launch("nc_btl_linear");
+}
+
+size_t nc_prefix_ce_workspace_bytes(int M, int C, int V_pad) {
+  if (M <= 0 || C <= 0 || V_pad <= 0) return 0;
+  const size_t tiles = 2 * ((size_t)V_pad / 128);
+  return align256((size_t)M * C * 2) + align256((size_t)M * tiles * 4) + 2 * align256((size_t)M * 4);
+}
+
+int nc_prefix_ce(const float* x, const void* w_u, const int32_t* targets, float* out_loss, int M, int C, int V,
+                 int V_pad, const int* widths, int k, float eps, float cap, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+  t_launches = 0;
+  if (x == nullptr || w_u == nullptr || targets == nullptr || out_loss == nullptr) return NC_ERR_ARG;
+  if (!(eps >= 0.f) || !(cap > 0.f)) return NC_ERR_ARG;
+  PrefixBlocks pb;
+  if (M <= 0 || C <= 0 || V <= 0 || V_pad < V || V_pad % 256 != 0 || !prefix_blocks(widths, k, C, &pb))
+    return NC_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(w_u) || !aligned16(targets) || !aligned16(out_loss) || !aligned16(workspace))
+    return NC_ERR_ALIGN;
+  if (workspace == nullptr || workspace_bytes < nc_prefix_ce_workspace_bytes(M, C, V_pad)) return NC_ERR_WORKSPACE;
+  DevInfo d;
+  if (!dev_info(&d)) return NC_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  bf16* xn = reinterpret_cast<bf16*>(ws);
+  const int tiles = 2 * (V_pad / 256);  // partial sums per row: (256-column pair tile, column half)
+  float* ce_sum = reinterpret_cast<float*>(ws + align256((size_t)M * C * 2));
+  float* ce_tgt = reinterpret_cast<float*>(ws + align256((size_t)M * C * 2) + align256((size_t)M * (2 * (V_pad / 128)) * 4));
+  float* lse = ce_tgt + align256((size_t)M * 4) / 4;
+  // the normalised prefix of every submodel at once (block a scaled by the
+  // RMS of the prefix up to it), bf16 as the head GEMM's A operand
+  launch_prefix_rmsnorm(x, M, C, pb, eps, xn, 1, st);
+  for (int j = 0; j < k; ++j) {
+    // submodel j + 1: the first C_j columns of x_n and of W_U
+    EpiParams e;
+    memset(&e, 0, sizeof(e));
+    e.mode = EPI_CE;
+    e.cap = cap;
+    e.vocab = V;
+    e.targets = targets;
+    e.ce_sum = ce_sum;
+    e.ce_tgt = ce_tgt;
+    e.ce_tiles = tiles;
+    if (!launch_gemm_tc(xn, C, static_cast<const bf16*>(w_u), C, M, V_pad, pb.end[j], e, d.status, d.num_sms, st, true))
+      return NC_ERR_CUDA;
+    launch_ce_combine(ce_sum, ce_tgt, tiles, cap, targets, M, V, out_loss + (size_t)j * M, lse, d.status, st);
+  }
+  return check_launch("nc_prefix_ce");
+}
+
 int nc_get_status(void* stream, int* out_bits) {
   DevInfo d;
   if (!dev_info(&d)) return NC_ERR_CUDA;
@@ -805,7 +911,7 @@ const char* nc_kernel_name(int kind) {
   static const char* names[KK_COUNT] = {
       "embed_norm_smear", "rmsnorm", "rope_table", "rope_qknorm", "gemm_tcgen05", "gemm_cuda_core",
       "attention_tcgen05", "attention_cuda_core", "ce_combine", "ce_rows", "loss_mean", "last_logits",
-      "sample", "gemm_tcgen05_bwd", "head_bwd_rows"};
+      "sample", "gemm_tcgen05_bwd", "head_bwd_rows", "prefix_rmsnorm"};
   return (kind >= 0 && kind < KK_COUNT) ? names[kind] : "unknown";
 }
 

@@ -148,6 +148,15 @@ void launch_inv_count(const int32_t* targets, int n, float* inv_count, cudaStrea
 // out = bf16(g * in), n a multiple of 8 elements, 16-byte aligned buffers
 void launch_scale_bf16(const bf16* in, bf16* out, long long n, float g, int num_sms, cudaStream_t st);
 void launch_rmsnorm_bwd(const float* x, const float* g, float* dx, int M, int C, float eps, cudaStream_t st);
+// Nested blocks of a width: block a is [end[a-1], end[a]) (end[-1] = 0).
+constexpr int kMaxPrefixBlocks = 8;
+struct PrefixBlocks {
+  int k;
+  int end[kMaxPrefixBlocks];
+};
+// PrefixRMSNorm of x [M, C] fp32 into out (bf16 when out_bf16, else fp32).
+void launch_prefix_rmsnorm(const float* x, int M, int C, const PrefixBlocks& pb, float eps, void* out, int out_bf16,
+                           cudaStream_t st);
 void launch_loss_mean(const float* loss, const int32_t* targets, int n, float* out, cudaStream_t st);
 // generation: softcapped logits of the last position of each of B rows
 // (x: the final fp32 residual [B T, ldx]; W: lm_head [V_padded, C], bf16 or
@@ -178,9 +187,14 @@ struct StreamK {
   unsigned gen;
   int max_pairs;
 };
+// Block lower triangular B (pair kernel): output columns below out.end[a]
+// read only K elements below in.end[a] (the rest of B must be zero there).
+struct GemmKLimit {
+  PrefixBlocks out, in;
+};
 bool launch_gemm_tc(const bf16* A, int lda, const bf16* Bm, int ldb, int M, int N, int K,
                     const EpiParams& ep, int* status, int num_sms, cudaStream_t st, bool pair,
-                    const StreamK* sk = nullptr);
+                    const StreamK* sk = nullptr, const GemmKLimit* kl = nullptr);
 // tcgen05 GEMM with operands in either layout, single-CTA kernel (bf16):
 // C[M, N] = A[M, K] B[N, K]^T where A is stored row-major [M, lda] when
 // a_mn == 0 (K contiguous) or as its transpose [K, lda] when a_mn == 1 (M
@@ -224,7 +238,7 @@ int check_launch(const char* what);
 enum KernelKind : int {
   KK_EMBED = 0, KK_RMSNORM, KK_ROPE_TABLE, KK_ROPE_QKNORM, KK_GEMM_TC, KK_GEMM_SIMT, KK_ATTN_TC,
   KK_ATTN_SIMT, KK_CE_COMBINE, KK_CE_ROWS, KK_LOSS_MEAN, KK_LAST_LOGITS, KK_SAMPLE, KK_GEMM_TC_BWD,
-  KK_HEAD_BWD_ROWS, KK_COUNT
+  KK_HEAD_BWD_ROWS, KK_PREFIX_NORM, KK_COUNT
 };
 // Every launcher holds one of these around its kernel launch: it counts the
 // launch (per host thread) and, when the caller enabled timing for this kind,

@@ -83,6 +83,12 @@ _SIGS = {
                                        C.c_float, C.c_int, C.c_void_p]),
     "nc_attention_noalloc_max_bytes": (C.c_size_t, []),
     "nc_set_flag_wait_test": (C.c_int, [C.c_int, C.c_double]),
+    "nc_prefix_rmsnorm": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_int, C.c_float, C.c_void_p,
+                                    C.c_int, C.c_void_p]),
+    "nc_btl_linear": (C.c_int, [C.c_void_p] * 3 + [C.c_int] * 3 + [C.c_void_p, C.c_void_p, C.c_int, C.c_void_p]),
+    "nc_prefix_ce_workspace_bytes": (C.c_size_t, [C.c_int] * 3),
+    "nc_prefix_ce": (C.c_int, [C.c_void_p] * 4 + [C.c_int] * 4 + [C.c_void_p, C.c_int, C.c_float, C.c_float,
+                                                                 C.c_void_p, C.c_size_t, C.c_void_p]),
     "nc_routing_attention_workspace_bytes": (C.c_size_t, [C.c_int] * 4),
     "nc_routing_attention": (C.c_int, [C.c_void_p] * 6 + [C.c_int] * 6 + [C.c_float, C.c_float, C.c_void_p,
                                                                          C.c_size_t, C.c_void_p]),
@@ -93,7 +99,7 @@ _SIGS = {
 
 KERNEL_KINDS = ["embed_norm_smear", "rmsnorm", "rope_table", "rope_qknorm", "gemm_tcgen05",
                 "gemm_cuda_core", "attention_tcgen05", "attention_cuda_core", "ce_combine", "ce_rows",
-                "loss_mean", "last_logits", "sample", "gemm_tcgen05_bwd", "head_bwd_rows"]
+                "loss_mean", "last_logits", "sample", "gemm_tcgen05_bwd", "head_bwd_rows", "prefix_rmsnorm"]
 
 
 class LaunchTimer:
@@ -276,6 +282,47 @@ def nc_routing_attention(q2, k2, v2, q1, k1, out, window: int, gate_logit: float
     _check(lib().nc_routing_attention(_ptr(q2), _ptr(k2), _ptr(v2), _ptr(q1), _ptr(k1), _ptr(out), B, T, H, Hkv, D,
                                       window, gate_logit, scale, _ptr(workspace), nbytes, _stream(stream)),
            "nc_routing_attention")
+
+
+def _widths(widths):
+    arr = (C.c_int * len(widths))(*[int(w) for w in widths])
+    return arr, len(widths)
+
+
+def nc_prefix_rmsnorm(x, widths, out, eps: float = 1e-6, stream=None):
+    """PrefixRMSNorm of x [M, C] fp32 into out [M, C] (bf16 or fp32), nested block widths `widths`."""
+    import torch
+    M, Cw = x.shape
+    w, k = _widths(widths)
+    _check(lib().nc_prefix_rmsnorm(_ptr(x), M, Cw, w, k, eps, _ptr(out), int(out.dtype == torch.bfloat16),
+                                   _stream(stream)), "nc_prefix_rmsnorm")
+
+
+def nc_btl_linear(x, w, y, in_widths, out_widths, stream=None):
+    """y [M, C_out] fp32 = x [M, C_in] bf16 @ W^T with W [C_out, C_in] bf16 block lower triangular."""
+    M, C_in = x.shape
+    C_out = w.shape[0]
+    wi, k = _widths(in_widths)
+    wo, k2 = _widths(out_widths)
+    if k2 != k:
+        raise NcError("nc_btl_linear: in_widths and out_widths differ in length")
+    _check(lib().nc_btl_linear(_ptr(x), _ptr(w), _ptr(y), M, C_in, C_out, wi, wo, k, _stream(stream)),
+           "nc_btl_linear")
+
+
+def nc_prefix_ce(x, w_u, targets, out_loss, vocab: int, widths, eps: float = 1e-6, cap: float = 15.0,
+                 workspace=None, stream=None):
+    """Per-token softcapped CE of every j-front submodel: out_loss [k, M] fp32."""
+    import torch
+    M, Cw = x.shape
+    V_pad = w_u.shape[0]
+    wd, k = _widths(widths)
+    if workspace is None:
+        workspace = torch.empty(int(lib().nc_prefix_ce_workspace_bytes(M, Cw, V_pad)), dtype=torch.uint8,
+                                device=x.device)
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().nc_prefix_ce(_ptr(x), _ptr(w_u), _ptr(targets), _ptr(out_loss), M, Cw, vocab, V_pad, wd, k, eps,
+                              cap, _ptr(workspace), nbytes, _stream(stream)), "nc_prefix_ce")
 
 
 def nc_get_status(stream=None) -> tuple[int, int]:

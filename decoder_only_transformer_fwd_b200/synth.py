@@ -30,6 +30,7 @@ SEED_BASE = 20260  # seed of workload i is SEED_BASE + i
 _ID_TOKENS, _ID_TARGETS, _ID_WTE, _ID_HEAD, _ID_SMEAR = 1, 2, 3, 4, 5
 _ID_Q, _ID_K, _ID_V = 11, 12, 13
 _ID_UNIFORM, _ID_LOGITS = 21, 22
+_ID_NEST_X, _ID_NEST_W, _ID_NEST_WU, _ID_NEST_Y = 31, 32, 33, 34
 _LAYER_BASE = 1000  # layer l uses ids _LAYER_BASE + 16*l + j
 
 
@@ -167,6 +168,18 @@ def attention_inputs(seed: int, B: int, T: int, H: int, D: int, Hkv: int | None 
     k = rnd(normal(seed, _ID_K, (B, T, Hkv, D), 1.0))
     v = rnd(normal(seed, _ID_V, (B, T, Hkv, D), 1.0))
     return q, k, v
+
+
+def nested_inputs(seed: int, M: int, C_in: int, C_out: int, V: int, V_pad: int):
+    """Inputs of the nesting pieces: a residual x [M, C_in] ~ N(0, 1) (fp32),
+    a dense weight W [C_out, C_in] ~ N(0, 1/C_in) and a head W_U [V_pad, C_in]
+    ~ N(0, 1/C_in) (both bf16 values held as float32), targets [M] uniform in
+    [0, V).  Zeroing the weight's dead blocks is left to the caller."""
+    x = normal(seed, _ID_NEST_X, (M, C_in), 1.0)
+    w = round_bf16(normal(seed, _ID_NEST_W, (C_out, C_in), C_in ** -0.5))
+    w_u = round_bf16(normal(seed, _ID_NEST_WU, (V_pad, C_in), C_in ** -0.5))
+    y = _gen(seed, _ID_NEST_Y).integers(0, V, size=M, dtype=np.int64).astype(np.int32)
+    return x, w, w_u, y
 
 
 # Workload shapes (model depth, batch, sequence length, short window, dtype).

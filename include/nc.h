@@ -283,6 +283,49 @@ int nc_routing_attention(const void* q2, const void* k2, const void* v2, const v
                          int B, int T, int H, int Hkv, int D, int window, float gate_logit, float softmax_scale,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* StairFormer nesting pieces ("Fully Nested Transformers" README: block
+ * lower triangular weights keep the residual stream of smaller models a
+ * prefix of larger models', and PrefixRMSNorm keeps normalisation from
+ * leaking information backward down the hierarchy).  A width C is cut into k
+ * nested blocks, `widths` (host array of k ints, 1 <= k <= 8, each a positive
+ * multiple of 64, summing to C); C_a = widths[0] + ... + widths[a].  The
+ * j-front submodel is the first j blocks.  NC_ERR_SHAPE on other widths.
+ *
+ * nc_prefix_rmsnorm: block a of the output is block a of x divided by the RMS
+ * of x's prefix up to C_a:
+ *   out[m, c] = x[m, c] / sqrt(mean(x[m, :C_a]^2) + eps),  C_{a-1} <= c < C_a.
+ * x [M, C] fp32, out [M, C] bf16 (out_bf16 != 0) or fp32, row-major, 16-byte
+ * aligned device pointers (NC_ERR_ALIGN).  With one block it is RMSNorm. */
+int nc_prefix_rmsnorm(const float* x, int M, int C, const int* widths, int k, float eps, void* out, int out_bf16,
+                      void* stream);
+
+/* nc_btl_linear: y = x W^T with W [C_out, C_in] block lower triangular:
+ * output block a (columns below C_out_a) reads input blocks b <= a only
+ * (elements below C_in_a).  W is stored dense, row-major, and its dead blocks
+ * must hold zeros: each 256-column output tile contracts over the input prefix
+ * its last column reads, so dead blocks beyond it are never loaded, and those
+ * inside it are multiplied as the zeros they are.  x [M, C_in] bf16, W bf16,
+ * y [M, C_out] fp32; in_widths and out_widths: k block widths each.  C_out must
+ * be a multiple of 256 (NC_ERR_SHAPE); 16-byte aligned pointers. */
+int nc_btl_linear(const void* x, const void* w, float* y, int M, int C_in, int C_out, const int* in_widths,
+                  const int* out_widths, int k, void* stream);
+
+/* nc_prefix_ce: per-token softcapped cross-entropy of every j-front
+ * submodel, j = 1..k: its logits use the first C_j columns of the head on the
+ * normalised prefix,
+ *   z_j = PrefixRMSNorm(x)[:, :C_j] W_U[:, :C_j]^T,  zhat_j = cap tanh(z_j / cap),
+ *   out_loss[(j - 1) M + m] = logsumexp_v zhat_j[m, v] - zhat_j[m, y_m]
+ * over v < V (0 where y_m = -1; out-of-range targets are flagged as in
+ * nc_forward).  x [M, C] fp32; w_u [V_pad, C] bf16 (rows V.. V_pad - 1 are
+ * read but excluded from the sums); targets [M] int32; out_loss [k, M] fp32.
+ * PrefixRMSNorm(x) is held in bf16 (the head GEMM's operand) in `workspace`
+ * (>= nc_prefix_ce_workspace_bytes).  V_pad a multiple of 256 (NC_ERR_SHAPE);
+ * 16-byte aligned pointers. */
+size_t nc_prefix_ce_workspace_bytes(int M, int C, int V_pad);
+int nc_prefix_ce(const float* x, const void* w_u, const int32_t* targets, float* out_loss, int M, int C, int V,
+                 int V_pad, const int* widths, int k, float eps, float cap, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
 /* Synchronise `stream`, read the device status word (an OR of
  * 1 << NC_ERR_DATA and 1 << NC_ERR_TIMEOUT bits set by kernels since the last
  * read), clear it, and return NC_OK, NC_ERR_DATA or NC_ERR_TIMEOUT (timeout
@@ -320,7 +363,8 @@ int nc_set_flag_wait_test(int skew, double wait_limit_ms);
  * ... up to capacity.  Calling again (or with events == NULL, which disables
  * it) restarts the count.  Kinds: 0 embed_norm_smear, 1 rmsnorm, 2 rope_table,
  * 3 rope_qknorm, 4 gemm_tcgen05, 5 gemm_cuda_core, 6 attention_tcgen05,
- * 7 attention_cuda_core, 8 ce_combine, 9 ce_rows, 10 loss_mean.
+ * 7 attention_cuda_core, 8 ce_combine, 9 ce_rows, 10 loss_mean, 11 last_logits,
+ * 12 sample, 13 gemm_tcgen05_bwd, 14 head_bwd_rows, 15 prefix_rmsnorm.
  * Returns NC_ERR_ARG if events != NULL with kinds == NULL or capacity <= 0. */
 int nc_set_launch_timing(void** events, int* kinds, int capacity, unsigned kind_mask);
 

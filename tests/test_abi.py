@@ -260,3 +260,43 @@ def test_head_backward_rejects_bad_arguments_without_launching():
     assert lib.nc_params_init(C.byref(p), C.byref(cfg32)) == 0
     p.max_tokens = 8
     assert call() == SHAPE                      # bf16 mode only
+
+
+def test_stairformer_entry_points_reject_bad_arguments():
+    """Nested block widths must be 1..8 positive multiples of 64 summing to the
+    width; BTL outputs a multiple of 256 wide; the prefix CE's padded vocabulary
+    a multiple of 256 and its workspace large enough.  All rejected before any
+    launch."""
+    lib = nc.lib()
+    buf = (C.c_byte * 4096)()
+    a16 = C.c_void_p((C.addressof(buf) + 15) & ~15)
+    mis = C.c_void_p(a16.value + 4)
+    ARG, SHAPE = nc.STATUS_CODES["NC_ERR_ARG"], nc.STATUS_CODES["NC_ERR_SHAPE"]
+    ALIGN, WS = nc.STATUS_CODES["NC_ERR_ALIGN"], nc.STATUS_CODES["NC_ERR_WORKSPACE"]
+
+    def w(*v):
+        return (C.c_int * len(v))(*v)
+
+    ok = w(384, 1152)
+    # nc_prefix_rmsnorm(x, M, C, widths, k, eps, out, out_bf16, stream)
+    assert lib.nc_prefix_rmsnorm(None, 4, 1536, ok, 2, 1e-6, a16, 1, None) == ARG
+    assert lib.nc_prefix_rmsnorm(a16, 4, 1536, ok, 2, -1.0, a16, 1, None) == ARG
+    assert lib.nc_prefix_rmsnorm(a16, 4, 1536, w(384, 1088), 2, 1e-6, a16, 1, None) == SHAPE  # sum != C
+    assert lib.nc_prefix_rmsnorm(a16, 4, 1536, w(400, 1136), 2, 1e-6, a16, 1, None) == SHAPE  # not x64
+    assert lib.nc_prefix_rmsnorm(a16, 4, 1536, ok, 0, 1e-6, a16, 1, None) == SHAPE
+    assert lib.nc_prefix_rmsnorm(a16, 4, 576, w(*([64] * 9)), 9, 1e-6, a16, 1, None) == SHAPE  # k > 8
+    assert lib.nc_prefix_rmsnorm(a16, 4, 1536, ok, 2, 1e-6, mis, 1, None) == ALIGN
+    assert lib.nc_prefix_rmsnorm(a16, 0, 1536, ok, 2, 1e-6, a16, 1, None) == 0  # nothing to do
+    # nc_btl_linear(x, w, y, M, C_in, C_out, in_widths, out_widths, k, stream)
+    assert lib.nc_btl_linear(a16, None, a16, 8, 1536, 1536, ok, ok, 2, None) == ARG
+    assert lib.nc_btl_linear(a16, a16, a16, 8, 1536, 1152, ok, w(384, 768), 2, None) == SHAPE  # C_out % 256
+    assert lib.nc_btl_linear(a16, a16, a16, 8, 1536, 1536, ok, w(512, 1024), 1, None) == SHAPE  # k mismatch
+    assert lib.nc_btl_linear(mis, a16, a16, 8, 1536, 1536, ok, ok, 2, None) == ALIGN
+    # nc_prefix_ce(x, w_u, targets, out_loss, M, C, V, V_pad, widths, k, eps, cap, ws, ws_bytes, stream)
+    assert lib.nc_prefix_ce(a16, a16, None, a16, 8, 1536, 1000, 1024, ok, 2, 1e-6, 15.0, a16, 1 << 30, None) == ARG
+    assert lib.nc_prefix_ce(a16, a16, a16, a16, 8, 1536, 1000, 1024, ok, 2, 1e-6, 0.0, a16, 1 << 30, None) == ARG
+    assert lib.nc_prefix_ce(a16, a16, a16, a16, 8, 1536, 1000, 1000, ok, 2, 1e-6, 15.0, a16, 1 << 30, None) == SHAPE
+    assert lib.nc_prefix_ce(a16, a16, a16, a16, 8, 1536, 1100, 1024, ok, 2, 1e-6, 15.0, a16, 1 << 30, None) == SHAPE
+    need = nc.lib().nc_prefix_ce_workspace_bytes(8, 1536, 1024)
+    assert need >= 8 * 1536 * 2
+    assert lib.nc_prefix_ce(a16, a16, a16, a16, 8, 1536, 1000, 1024, ok, 2, 1e-6, 15.0, a16, need - 1, None) == WS

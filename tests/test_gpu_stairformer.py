@@ -1,0 +1,133 @@
+"""GPU parity of the StairFormer nesting pieces ("Fully Nested Transformers"
+README) against oracle/stairformer.py: PrefixRMSNorm (nc_prefix_rmsnorm),
+the block lower triangular linear map (nc_btl_linear) and the prefix
+cross-entropy of the j-front submodels (nc_prefix_ce).
+
+Tolerances, from the arithmetic:
+  * PrefixRMSNorm in fp32: every element within 2e-6 relative (fp32 sums of
+    squares and rsqrt); with bf16 output within the bf16 rounding bound (half
+    a unit in the 8th significant bit: 2^-8 relative) plus that;
+  * BTL: bf16 x bf16 products are exact in fp32 and summed in fp32 over
+    K <= 1536 terms: every element within 1e-4 of the output's largest
+    magnitude; and output block a does not move, bit for bit, when input
+    blocks past a change (the dead blocks are skipped or multiplied as zeros);
+  * prefix CE: the normalised prefix is rounded to bf16 once (the head GEMM's
+    operand), a relative error of rms 2^-8 / sqrt(3) per element.  Through a
+    logit over C_j weights of variance 1 / C that is an error of rms
+    2^-8 / sqrt(3) * sqrt(C_j / C) (about 2.3e-3 at C_j = C), which the loss
+    carries through its target logit.  Per-token loss within 1e-2 (the
+    forward's tolerance), rms within 1.5 times that estimate, mean within
+    1e-3, and 0 for ignored targets."""
+import numpy as np
+import pytest
+
+from decoder_only_transformer_fwd_b200 import nc, synth
+from oracle import stairformer as S
+
+pytestmark = pytest.mark.gpu
+
+D24_WIDTHS = [384, 1152]  # the README's d24 run: 6 + 18 heads of 64
+
+
+def _dev(a, dtype=None):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    return t.to(dtype) if dtype is not None else t
+
+
+def _zero_dead_blocks(w, out_widths, in_widths):
+    """W [C_out, C_in] with the blocks that output block a may not read (input
+    blocks b > a) set to zero, as the kernel's dense storage requires."""
+    w = w.copy()
+    oe, ie = np.cumsum(out_widths), np.cumsum(in_widths)
+    for a in range(len(out_widths)):
+        w[oe[a] - out_widths[a]:oe[a], ie[a]:] = 0.0
+    return w
+
+
+@pytest.mark.parametrize("M,widths", [(37, D24_WIDTHS), (256, [256, 512, 768]), (5, [1536])])
+@pytest.mark.parametrize("out_dtype", ["fp32", "bf16"])
+def test_prefix_rmsnorm(M, widths, out_dtype):
+    import torch
+    C = sum(widths)
+    x, _, _, _ = synth.nested_inputs(synth.SEED_BASE + 50 + M, M, C, 256, 8, 256)
+    x *= np.linspace(0.2, 3.0, C, dtype=np.float32)  # blocks of different scales
+    dt = torch.float32 if out_dtype == "fp32" else torch.bfloat16
+    out = torch.empty(M, C, dtype=dt, device="cuda")
+    nc.nc_prefix_rmsnorm(_dev(x), widths, out, eps=1e-6)
+    got = out.float().cpu().numpy().astype(np.float64)
+    ref = S.prefix_rmsnorm(x, widths, eps=1e-6)
+    rel = 2e-6 + (2.0 ** -8 if out_dtype == "bf16" else 0.0)
+    assert np.all(np.abs(got - ref) <= rel * np.abs(ref) + 1e-30), float(np.max(np.abs(got - ref) / np.abs(ref)))
+
+
+@pytest.mark.parametrize("M,in_widths,out_widths", [(300, D24_WIDTHS, D24_WIDTHS),
+                                                    (128, D24_WIDTHS, [1536, 4608]),
+                                                    (77, [256, 256, 1024], [256, 256, 1024])])
+def test_btl_linear(M, in_widths, out_widths):
+    import torch
+    C_in, C_out = sum(in_widths), sum(out_widths)
+    x, w, _, _ = synth.nested_inputs(synth.SEED_BASE + 60 + M, M, C_in, C_out, 8, 256)
+    x = synth.round_bf16(x)
+    w = _zero_dead_blocks(w, out_widths, in_widths)
+    y = torch.empty(M, C_out, dtype=torch.float32, device="cuda")
+    xd = _dev(x, torch.bfloat16)
+    nc.nc_btl_linear(xd, _dev(w, torch.bfloat16), y, in_widths, out_widths)
+    got = y.cpu().numpy().astype(np.float64)
+    ref = S.btl_linear(x, w, out_widths, in_widths)
+    assert float(np.max(np.abs(got - ref))) <= 1e-4 * float(np.max(np.abs(ref)))
+    # filtration: change every input block past the first; output block 0 stays bit-identical
+    x2 = x.copy()
+    x2[:, in_widths[0]:] = synth.round_bf16(x2[:, in_widths[0]:] * 3.0 + 1.0)
+    y2 = torch.empty_like(y)
+    nc.nc_btl_linear(_dev(x2, torch.bfloat16), _dev(w, torch.bfloat16), y2, in_widths, out_widths)
+    assert torch.equal(y2[:, :out_widths[0]], y[:, :out_widths[0]])
+    assert not torch.equal(y2[:, out_widths[0]:], y[:, out_widths[0]:])
+    rc, bits = nc.nc_get_status()
+    assert rc == 0, bits
+
+
+def _check_prefix_ce(got, ref, valid, cj, c):
+    d = np.abs(got - ref)
+    rms_bound = 1.5 * 2.0 ** -8 / np.sqrt(3.0) * np.sqrt(cj / c)
+    print(f"prefix CE (C_j = {cj}): max err {d.max():.3e}, rms {np.sqrt(np.mean(d ** 2)):.3e} (bound {rms_bound:.2e})")
+    assert d.max() <= 1e-2
+    assert np.sqrt(np.mean(d ** 2)) <= rms_bound
+    assert abs(float(got[valid].mean() - ref[valid].mean())) <= 1e-3
+    assert np.all(got[~valid] == 0.0)
+
+
+@pytest.mark.parametrize("M,widths,V,V_pad", [(300, D24_WIDTHS, 1000, 1024), (64, [256, 512, 768], 4000, 4096)])
+def test_prefix_ce(M, widths, V, V_pad):
+    import torch
+    C = sum(widths)
+    x, _, w_u, y = synth.nested_inputs(synth.SEED_BASE + 70 + M, M, C, 256, V, V_pad)
+    y[::7] = -1
+    loss = torch.full((len(widths), M), float("nan"), dtype=torch.float32, device="cuda")
+    nc.nc_prefix_ce(_dev(x), _dev(w_u, torch.bfloat16), _dev(y), loss, V, widths)
+    rc, bits = nc.nc_get_status()
+    assert rc == 0, bits
+    got = loss.cpu().numpy().astype(np.float64)
+    ref = S.prefix_ce(x, w_u[:V], y, widths)
+    for j in range(len(widths)):
+        _check_prefix_ce(got[j], ref[j], y != -1, sum(widths[:j + 1]), C)
+    # the larger submodel sees more: its loss differs from the smaller one's
+    assert not np.allclose(got[0], got[-1])
+
+
+def test_prefix_ce_d24_sampled_rows():
+    """The README's d24 widths at full vocabulary, B*T = 8192 rows on the GPU,
+    checked on a sample of rows (rows are independent)."""
+    import torch
+    M, V = 8192, 32768
+    C = sum(D24_WIDTHS)
+    x, _, w_u, y = synth.nested_inputs(synth.SEED_BASE + 80, M, C, 256, V, V)
+    loss = torch.empty((2, M), dtype=torch.float32, device="cuda")
+    nc.nc_prefix_ce(_dev(x), _dev(w_u, torch.bfloat16), _dev(y), loss, V, D24_WIDTHS)
+    rc, bits = nc.nc_get_status()
+    assert rc == 0, bits
+    got = loss.cpu().numpy().astype(np.float64)
+    rows = np.array([0, 1, 2047, 4096, 8191] + list(range(100, 8192, 811)))
+    ref = S.prefix_ce(x[rows], w_u, y[rows], D24_WIDTHS)
+    for j in range(2):
+        _check_prefix_ce(got[j][rows], ref[j], np.ones(len(rows), bool), sum(D24_WIDTHS[:j + 1]), C)
