@@ -131,3 +131,36 @@ def test_prefix_ce_d24_sampled_rows():
     ref = S.prefix_ce(x[rows], w_u, y[rows], D24_WIDTHS)
     for j in range(2):
         _check_prefix_ce(got[j][rows], ref[j], np.ones(len(rows), bool), sum(D24_WIDTHS[:j + 1]), C)
+
+
+def test_edge_cases():
+    """One row and eight 64-wide blocks (PrefixRMSNorm); a 256-column output
+    tile that straddles two block boundaries (BTL: its columns of blocks 0 and
+    1 are multiplied by dead zeros of the wider prefix, and must still match);
+    three submodels over a single 256-column vocabulary tile (prefix CE)."""
+    import torch
+    x, _, _, _ = synth.nested_inputs(synth.SEED_BASE + 95, 1, 512, 256, 8, 256)
+    out = torch.empty(1, 512, dtype=torch.float32, device="cuda")
+    nc.nc_prefix_rmsnorm(_dev(x), [64] * 8, out)
+    ref = S.prefix_rmsnorm(x, [64] * 8)
+    assert np.all(np.abs(out.cpu().numpy() - ref) <= 2e-6 * np.abs(ref) + 1e-30)
+
+    in_w, out_w = [128, 128, 256], [64, 128, 320]
+    x, w, _, _ = synth.nested_inputs(synth.SEED_BASE + 96, 130, 512, 512, 8, 256)
+    x = synth.round_bf16(x)
+    w = _zero_dead_blocks(w, out_w, in_w)
+    y = torch.empty(130, 512, dtype=torch.float32, device="cuda")
+    nc.nc_btl_linear(_dev(x, torch.bfloat16), _dev(w, torch.bfloat16), y, in_w, out_w)
+    ref = S.btl_linear(x, w, out_w, in_w)
+    assert float(np.max(np.abs(y.cpu().numpy() - ref))) <= 1e-4 * float(np.max(np.abs(ref)))
+
+    widths = [64, 128, 320]
+    x, _, w_u, t = synth.nested_inputs(synth.SEED_BASE + 97, 19, 512, 256, 200, 256)
+    loss = torch.empty(3, 19, dtype=torch.float32, device="cuda")
+    nc.nc_prefix_ce(_dev(x), _dev(w_u, torch.bfloat16), _dev(t), loss, 200, widths)
+    rc, bits = nc.nc_get_status()
+    assert rc == 0, bits
+    ref = S.prefix_ce(x, w_u[:200], t, widths)
+    got = loss.cpu().numpy().astype(np.float64)
+    for j in range(3):
+        _check_prefix_ce(got[j], ref[j], np.ones(19, bool), sum(widths[:j + 1]), 512)
