@@ -496,7 +496,11 @@ def run_ours(args):
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     for _ in range(args.steps):
+        # each step copies its inputs in and its per-token loss out; the calls
+        # are asynchronous, so the host enqueues the next step while the GPU
+        # runs this one, and the clock stops once the last loss is on the host
         nc.nc_forward_host(model.params, h_tok, h_tgt, h_loss, stream)
+    torch.cuda.synchronize()
     e2e_s = max_over_ranks(time.perf_counter() - t0)
     attn = None if args.no_attention_sweep else attention_sweep(args, dev, stream)
     gen = None

@@ -578,7 +578,6 @@ int nc_forward_host(const nc_params* p, const int32_t* h_tokens, const int32_t* 
   const int rc = nc_forward(p, dtok, dtgt, B, T, dloss, nullptr, stream);
   if (rc != NC_OK) return rc;
   e = cudaMemcpyAsync(h_out_loss, dloss, n * 4, cudaMemcpyDeviceToHost, st);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) {
     set_err("nc_forward_host D2H", e);
     return NC_ERR_CUDA;

@@ -224,7 +224,8 @@ def nc_generate_next(params: nc_params, tokens, temperature: float, top_k: int, 
 
 def nc_forward_host(params: nc_params, tokens: np.ndarray, targets: np.ndarray, out_loss: np.ndarray,
                     stream=None):
-    """tokens/targets/out_loss are host arrays (pinned torch tensors or numpy)."""
+    """tokens/targets/out_loss are host arrays (pinned torch tensors or numpy).
+    Asynchronous on `stream`: out_loss is valid after the stream synchronises."""
     B, T = tokens.shape
     ptr = lambda a: C.c_void_p(a.data_ptr() if hasattr(a, "data_ptr") else a.ctypes.data)
     _check(lib().nc_forward_host(C.byref(params), ptr(tokens), ptr(targets), B, T, ptr(out_loss),

@@ -139,8 +139,12 @@ int nc_forward(const nc_params* p, const int32_t* tokens, const int32_t* targets
 
 /* The same pass from HOST buffers: copies h_tokens/h_targets ([B, T] int32,
  * host) into the workspace, runs nc_forward() and copies the per-token loss
- * back into h_out_loss ([B*T] fp32, host).  Synchronous: returns after the
- * loss is on the host.  Pinned host memory gives asynchronous-capable copies. */
+ * back into h_out_loss ([B*T] fp32, host).  Asynchronous on `stream` like every
+ * call: h_out_loss holds the loss once the stream has been synchronised, and
+ * the host buffers must stay valid until then.  With pinned host memory the
+ * copies overlap other work on the GPU (consecutive calls on one stream
+ * pipeline); with pageable memory the runtime may complete them before it
+ * returns. */
 int nc_forward_host(const nc_params* p, const int32_t* h_tokens, const int32_t* h_targets, int B,
                     int T, float* h_out_loss, void* stream);
 

@@ -157,8 +157,16 @@ def test_loss_mean_and_host_entry_point():
     assert abs(out.item() - loss[valid].mean()) < 1e-5
     # host buffers in, host loss out: same numbers as the device entry point
     h_loss = torch.empty(tok.size, dtype=torch.float32).pin_memory()
-    nc.nc_forward_host(model.params, torch.from_numpy(tok).pin_memory(),
-                       torch.from_numpy(tgt).pin_memory(), h_loss)
+    h_tok, h_tgt = torch.from_numpy(tok).pin_memory(), torch.from_numpy(tgt).pin_memory()
+    nc.nc_forward_host(model.params, h_tok, h_tgt, h_loss)
+    torch.cuda.synchronize()  # the call is asynchronous: the loss is on the host after a sync
+    assert np.array_equal(h_loss.numpy().reshape(tok.shape), loss)
+    # consecutive calls on one stream pipeline; each one's loss lands in its own buffer
+    h_loss2 = torch.full((tok.size,), float("nan"), dtype=torch.float32).pin_memory()
+    for buf in (h_loss2, h_loss, h_loss2):
+        nc.nc_forward_host(model.params, h_tok, h_tgt, buf)
+    torch.cuda.synchronize()
+    assert np.array_equal(h_loss2.numpy().reshape(tok.shape), loss)
     assert np.array_equal(h_loss.numpy().reshape(tok.shape), loss)
     # all targets ignored: the mean is NaN
     none = torch.full((8,), -1, dtype=torch.int32, device="cuda")
