@@ -373,10 +373,13 @@ int forward_impl(const nc_params* p, const int32_t* tokens, const int32_t* targe
   // tensor-core path: RMSNorm is fused into the GEMMs (producers write bf16(x)
   // and per-row sums of squares, consumers scale their rows by 1 / rms)
   const bool tc = bf && c.gemm_impl == 0;
-  // stream-K flags start at 0 each forward; every GEMM launch of the forward
-  // gets its own generation number
+  // stream-K flags (split-tail schedule, gemm_pair == 2 only) start at 0 each
+  // forward; every GEMM launch of the forward gets its own generation number.
+  // Other schedules skip the memset, which would break the programmatic
+  // dependent launch between the previous forward's last kernel and this one's
+  // first.
   StreamK sk{nullptr, nullptr, 0u, kStreamKPairs};
-  if (tc) {
+  if (tc && c.gemm_pair == 2) {
     sk.ws = at<float>(ws, Lw.skws);
     sk.flags = at<unsigned>(ws, Lw.skflags);
     if (cudaMemsetAsync(sk.flags, 0, (size_t)kStreamKPairs * 2 * 4, st) != cudaSuccess) return NC_ERR_CUDA;
