@@ -711,9 +711,9 @@ void launch_rmsnorm(const float* x, void* xn, int M, int C, float eps, int act_b
 void launch_rope_table(float* cos_t, float* sin_t, int T, int D, float base, cudaStream_t st, float* fsplit,
                        int tbits) {
   LaunchScope scope_(KK_ROPE_TABLE, st);
-  const int n = T * (D / 2);
-  launch_pdl(k_rope_table, dim3((n + 255) / 256), dim3(256), 0, st, 1, cos_t, sin_t, T, D, (double)base, fsplit,
-             tbits);
+  const int n = T * (D / 2);  // T = 0: the split frequencies only
+  launch_pdl(k_rope_table, dim3(n > 0 ? (n + 255) / 256 : 1), dim3(256), 0, st, 1, cos_t, sin_t, T, D, (double)base,
+             fsplit, tbits);
 }
 
 void launch_rope_qknorm_ve(void* qkv, int ld, int B, int T, int H, int Hkv, int D,

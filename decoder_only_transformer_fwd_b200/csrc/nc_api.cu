@@ -391,7 +391,9 @@ int forward_impl(const nc_params* p, const int32_t* tokens, const int32_t* targe
   };
   int tbits = 1;
   while ((1 << tbits) < T) ++tbits;
-  launch_rope_table(rcos, rsin, T, D, c.rope_base, st, rfreq, tbits);
+  // the tensor-core QKV epilogue computes cos / sin from the split
+  // frequencies alone; the positional table serves the CUDA-core path
+  launch_rope_table(rcos, rsin, tc ? 0 : T, D, c.rope_base, st, rfreq, tbits);
   float* ss = at<float>(ws, Lw.ss);
   const int ss_parts = C / (gemm_tc_bn(C) / 2);  // per-row sums of squares, one slot per epilogue warp's columns
   bf16* xb = tc ? static_cast<bf16*>(xn) : nullptr;
@@ -427,8 +429,6 @@ int forward_impl(const nc_params* p, const int32_t* tokens, const int32_t* targe
       norm_in(e);
       e.T = T;
       e.qk_cols = (H + Hkv) * D;
-      e.rope_cos = rcos;
-      e.rope_sin = rsin;
       e.rope_fsplit = rfreq;
       e.qk_alpha = c.qk_alpha;
       e.tokens = tokens;

@@ -84,8 +84,6 @@ struct EpiParams {
   // EPI_QKV (out/ldo as for EPI_STORE)
   int T;              // positions per row (position = m % T)
   int qk_cols;        // (H + H_kv) * D: columns below this are q and k heads
-  const float* rope_cos;  // [T, D/2]
-  const float* rope_sin;
   const float* rope_fsplit;  // [2, D/2]: per-frequency cycles per position, split hi | lo (see k_rope_table)
   float qk_alpha, eps;
   const int32_t* tokens;  // [M]
