@@ -657,7 +657,7 @@ __device__ __forceinline__ RowPre epilogue_pre(const EpiParams& ep, const TcArgs
   return p;
 }
 
-// Pull into L2 the rows of x (and x0 / x_bo) that the residual epilogue of
+// Pull into L2 the rows of x that the O-projection's residual epilogue of
 // tile (mb, nb) will read: called one tile ahead, so the reads hit L2.
 template <int BN, int MODE>
 __device__ __forceinline__ void epilogue_prefetch(const EpiParams& ep, const TcArgs& a, int mb, int nb, int g,
@@ -665,23 +665,17 @@ __device__ __forceinline__ void epilogue_prefetch(const EpiParams& ep, const TcA
   const int m = mb * kBM + g * 32 + lane;
   const int n_lo = nb * BN + c_lo;
   if (m >= a.M) return;
-  if constexpr (MODE == EPI_RESID || MODE == EPI_BLOCK_END) {
-    // this thread's row of the warp's columns of x (and x0 / x_bo)
+  // (EPI_BLOCK_END, the MLP down-projection, is left out: its K = 4C
+  // mainloop is so long that lines pulled in a tile ahead leave L2 again
+  // before they are read, and would be fetched twice)
+  if constexpr (MODE == EPI_RESID) {
+    // this thread's row of the warp's columns of x
     const int nc = min(c_cnt, a.N - n_lo);
     if (nc > 0) {
       const char* xr = reinterpret_cast<const char*>(ep.x + (size_t)m * ep.ldx + n_lo);
 #pragma unroll
       for (int o = 0; o < (BN / 2) * 4; o += 128)
         if (o < nc * 4) ptx::prefetch_l2(xr + o);
-      if (MODE == EPI_BLOCK_END) {
-        const float* z = ep.end_kind == 1 ? ep.x0 : ((ep.end_kind == 2 && !ep.capture_bo) ? ep.xbo : nullptr);
-        if (z != nullptr) {
-          const char* zr = reinterpret_cast<const char*>(z + (size_t)m * ep.ldx + n_lo);
-#pragma unroll
-          for (int o = 0; o < (BN / 2) * 4; o += 128)
-            if (o < nc * 4) ptx::prefetch_l2(zr + o);
-        }
-      }
     }
   }
 }
