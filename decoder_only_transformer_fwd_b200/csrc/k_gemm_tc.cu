@@ -657,45 +657,6 @@ __device__ __forceinline__ RowPre epilogue_pre(const EpiParams& ep, const TcArgs
   return p;
 }
 
-// Pull into L2 the rows of x that the O-projection's residual epilogue of
-// tile (mb, nb) will read: called one tile ahead, so the reads hit L2.
-template <int BN, int MODE>
-__device__ __forceinline__ void epilogue_prefetch(const EpiParams& ep, const TcArgs& a, int mb, int nb, int g,
-                                                  int c_lo, int c_cnt, int lane) {
-  const int m = mb * kBM + g * 32 + lane;
-  const int n_lo = nb * BN + c_lo;
-  if (m >= a.M) return;
-  // (EPI_BLOCK_END, the MLP down-projection, is left out: its K = 4C
-  // mainloop is so long that lines pulled in a tile ahead leave L2 again
-  // before they are read, and would be fetched twice)
-  if constexpr (MODE == EPI_RESID) {
-    // this thread's row of the warp's columns of x
-    const int nc = min(c_cnt, a.N - n_lo);
-    if (nc > 0) {
-      const char* xr = reinterpret_cast<const char*>(ep.x + (size_t)m * ep.ldx + n_lo);
-#pragma unroll
-      for (int o = 0; o < (BN / 2) * 4; o += 128)
-        if (o < nc * 4) ptx::prefetch_l2(xr + o);
-    }
-  }
-}
-
-// Before the first tile: touch (prefetch into L2) one line of each output
-// row this thread will write first, so that the address translations and L2
-// lines of the output region are in place when the first accumulator is ready.
-template <int BN, int MODE>
-__device__ __forceinline__ void epilogue_touch_outputs(const EpiParams& ep, const TcArgs& a, int mb, int nb, int g,
-                                                       int c_lo, int lane) {
-  const int m = mb * kBM + g * 32 + lane;
-  const int n_lo = nb * BN + c_lo;
-  if (m >= a.M || n_lo >= a.N) return;
-  if constexpr (MODE == EPI_STORE || MODE == EPI_RELU2 || MODE == EPI_QKV) {
-    ptx::prefetch_l2(reinterpret_cast<const bf16*>(ep.out) + (size_t)m * ep.ldo + n_lo);
-  } else if constexpr (MODE == EPI_RESID || MODE == EPI_BLOCK_END) {
-    if (ep.xb_out != nullptr) ptx::prefetch_l2(ep.xb_out + (size_t)m * ep.ldxb + n_lo);
-  }
-}
-
 // Epilogue work of one warp on one tile: rows g*32 .. g*32+31 of the tile
 // (its TMEM lane quarter) and the columns [c_lo, c_lo + c_cnt) (a multiple
 // of 32; the two warps of a lane quarter split the tile's columns).
@@ -963,16 +924,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* stage = epi_stage + ew * Cf::STAGE_FLOATS;
     int acc = 0;
     uint32_t aph = 0;
-    if (blockIdx.x < a.num_tiles) {
-      epilogue_prefetch<BN, MODE>(ep, a, blockIdx.x % a.tiles_m, blockIdx.x / a.tiles_m, g, c_lo, c_cnt, lane);
-      epilogue_touch_outputs<BN, MODE>(ep, a, blockIdx.x % a.tiles_m, blockIdx.x / a.tiles_m, g, c_lo, lane);
-    }
     for (int tile = blockIdx.x; tile < a.num_tiles; tile += gridDim.x) {
       const int mb = tile % a.tiles_m, nb = tile / a.tiles_m;
       const RowPre pre = epilogue_pre<BN, MODE>(ep, a, mb, nb, g, c_lo, lane);
-      const int nxt = tile + gridDim.x;
-      if (nxt < a.num_tiles)
-        epilogue_prefetch<BN, MODE>(ep, a, nxt % a.tiles_m, nxt / a.tiles_m, g, c_lo, c_cnt, lane);
       if (*abort_flag || !ptx::mbar_wait(tfull(acc), aph, a.status)) {
         *abort_flag = 1;
         break;
@@ -1189,15 +1143,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     float* stage = epi_stage + ew * Cf::STAGE_FLOATS;
     int acc = 0;
     uint32_t aph = 0;
-    if (sched.njobs > 0) {
-      int pt, kb_lo, kb_hi, kind;
-      job_at(sched, 0, pt, kb_lo, kb_hi, kind);
-      int mbp, nb, c_lo, c_cnt;
-      pair_tile(a, pt, tiles_mp, mbp, nb);
-      cols(0, c_lo, c_cnt);
-      epilogue_prefetch<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, c_lo, c_cnt, lane);
-      epilogue_touch_outputs<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, c_lo, lane);
-    }
     for (int j = 0; j < sched.njobs; ++j) {
       int pt, kb_lo, kb_hi, kind;
       job_at(sched, j, pt, kb_lo, kb_hi, kind);
@@ -1207,14 +1152,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       pair_tile(a, pt, tiles_mp, mbp, nb);
       cols(j, c_lo, c_cnt);
       const RowPre pre = epilogue_pre<BN, MODE>(ep, a, mbp * 2 + (int)rank, nb, g, c_lo, lane);
-      if (j + 1 < sched.njobs) {
-        int ptn, kln, khn, kn, cln, ccn;
-        job_at(sched, j + 1, ptn, kln, khn, kn);
-        int mbn, nbn;
-        pair_tile(a, ptn, tiles_mp, mbn, nbn);
-        cols(j + 1, cln, ccn);
-        epilogue_prefetch<BN, MODE>(ep, a, mbn * 2 + (int)rank, nbn, g, cln, ccn, lane);
-      }
       if (*abort_flag || !ptx::mbar_wait_cluster(tfull(acc), aph, a.status)) {
         *abort_flag = 1;
         break;
