@@ -15,6 +15,9 @@
 
 namespace nc {
 
+bool make_tmap_2d(CUtensorMap* map, const void* ptr, int rows, int cols, int ld, int box_rows,
+                  int box_cols);
+
 namespace {
 
 constexpr int kLastRows = 8;  // rows of one k_last_logits launch
@@ -248,6 +251,228 @@ k_last_logits(const float* __restrict__ x, int ldx, int T, int b0, const TW* __r
     }
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(empty(s));
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Last-position logits on the tensor cores (bf16 W_U, C a multiple of 64)
+// ---------------------------------------------------------------------------
+// The same product as k_last_logits, logits^T = W_U x^T, as an MMA with the
+// vocabulary rows as M and the (at most 16) x rows as N:
+//   * x^T is staged once per CTA in shared memory as the B operand (bf16,
+//     K-major, 128-byte swizzle: for each 64-wide k block, 16 rows of 128 B);
+//   * W_U streams through a ring of 32 KB stages by TMA, one 32-row x 64-k box
+//     per 32-row unit (128-byte swizzle); a stage holds up to 8 units, i.e.
+//     two M = 128 tiles;
+//   * one thread issues tcgen05.mma (M = 128, N = 16, K = 16) into TMEM; four
+//     epilogue warps read D (lane = vocabulary row, column = x row), apply
+//     the RMSNorm scale and the softcap and store one row of each x row per
+//     lane, so a warp's stores are 128 contiguous bytes.
+// Each CTA owns a contiguous run of units (the units spread evenly over the
+// grid), taken in passes of at most 8 units with two TMEM buffers.  Every
+// wait is bounded; on a timeout the CTA records NC_ERR_TIMEOUT and returns
+// once its copies and MMAs have landed.
+constexpr int kLtUnit = 32;                                 // vocabulary rows per TMA box
+constexpr int kLtUnitsMax = 8;                              // units per pass (two M = 128 tiles)
+constexpr int kLtN = 16;                                    // MMA N: x rows of one launch
+constexpr int kLtBoxBytes = kLtUnit * 128;                  // 4 KB: 32 rows x 64 bf16
+constexpr int kLtStageBytes = kLtUnitsMax * kLtBoxBytes;    // 32 KB
+constexpr int kLtMaxStages = 5;
+constexpr int kLtThreads = 192;                             // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr uint32_t kLtTmemCols = 64;                        // 2 buffers x 2 tiles x 16 columns
+
+struct LtGeom {
+  int stages;
+  size_t xt_bytes, smem;
+};
+inline LtGeom lt_geom(int C) {
+  LtGeom g;
+  g.xt_bytes = (size_t)kLtN * C * 2;
+  const size_t limit = 220 * 1024, fixed = 1024 + 256;
+  const size_t avail = limit > fixed + g.xt_bytes ? limit - fixed - g.xt_bytes : 0;
+  g.stages = (int)(avail / kLtStageBytes);
+  if (g.stages > kLtMaxStages) g.stages = kLtMaxStages;
+  g.smem = fixed + g.xt_bytes + (size_t)g.stages * kLtStageBytes;
+  return g;
+}
+
+__global__ void __launch_bounds__(kLtThreads, 1)
+k_last_logits_tc(const __grid_constant__ CUtensorMap tmW, const float* __restrict__ x, int ldx, int T, int b0, int nb,
+                 int V, int C, float cap, float eps, float* __restrict__ out, int ldo, int stages, int* status) {
+  pdl_launch_dependents();
+  extern __shared__ uint8_t lt_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lt_raw) + 1023) & ~uintptr_t(1023));
+  const int nkb = C / 64;
+  uint8_t* xt = smem;                                   // nkb blocks of 2 KB
+  uint8_t* ring = smem + (size_t)kLtN * C * 2;          // a multiple of 2 KB past a 1 KB boundary
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + (size_t)stages * kLtStageBytes);
+  // full[kLtMaxStages] | empty[kLtMaxStages] | tfull[2] | tempty[2] | done
+  const uint32_t bar0 = ptx::smem_u32(bars);
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (kLtMaxStages + s); };
+  auto tfull = [&](int b) { return bar0 + 8u * (2 * kLtMaxStages + b); };
+  auto tempty = [&](int b) { return bar0 + 8u * (2 * kLtMaxStages + 2 + b); };
+  const uint32_t done = bar0 + 8u * (2 * kLtMaxStages + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kLtMaxStages + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  __shared__ float rs[kLtN];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) {
+      ptx::mbar_init(full(s), 1);
+      ptx::mbar_init(empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(tfull(b), 1);
+      ptx::mbar_init(tempty(b), 4);
+    }
+    ptx::mbar_init(done, 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tmW);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kLtTmemCols);
+    ptx::tmem_relinquish();
+    ptx::tc_fence_before();
+  }
+  // this CTA's units [u_lo, u_hi) of 32 vocabulary rows
+  const int nunits = (V + kLtUnit - 1) / kLtUnit;
+  const int u_lo = (int)((long long)blockIdx.x * nunits / gridDim.x);
+  const int u_hi = (int)((long long)(blockIdx.x + 1) * nunits / gridDim.x);
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // x comes from the previous kernel
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (ptx::elect_one()) {
+      int k = 0;
+      bool ok = true;
+      for (int ub = u_lo; ub < u_hi && ok; ub += kLtUnitsMax) {
+        const int nu = min(kLtUnitsMax, u_hi - ub);
+        for (int kb = 0; kb < nkb; ++kb, ++k) {
+          const int s = k % stages;
+          if (*abort_flag || !ptx::mbar_wait(empty(s), ((uint32_t)(k / stages) & 1u) ^ 1u, status)) {
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(full(s), (uint32_t)(nu * kLtBoxBytes));
+          const uint32_t dst = ptx::smem_u32(ring + (size_t)s * kLtStageBytes);
+          for (int i = 0; i < nu; ++i)
+            ptx::tma_load_2d(dst + (uint32_t)(i * kLtBoxBytes), &tmW, full(s), kb * 64, (ub + i) * kLtUnit);
+        }
+      }
+      if (!ok) *abort_flag = 1;
+      // every issued copy has landed before the CTA may exit
+      for (int q = k - stages > 0 ? k - stages : 0; q < k; ++q)
+        ptx::mbar_wait(full(q % stages), (uint32_t)(q / stages) & 1u, status);
+    }
+  } else {
+    // ---------------- stage x^T (warps 1..5) ----------------
+    // warp w takes x rows j = w - 1, w + 4, ...; lane c handles the 16-byte
+    // chunks c, c + 32, ... (8 consecutive k) of the row
+    for (int j = warp - 1; j < kLtN; j += 5) {
+      const bool live = j < nb;
+      const float* xr = x + ((size_t)(b0 + (live ? j : 0)) * T + (T - 1)) * ldx;
+      float sq = 0.f;
+      for (int ci = lane; ci < C / 8; ci += 32) {
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (live) {
+          const float4 a = *reinterpret_cast<const float4*>(xr + 8 * ci);
+          const float4 b = *reinterpret_cast<const float4*>(xr + 8 * ci + 4);
+          sq += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w + b.x * b.x + b.y * b.y + b.z * b.z + b.w * b.w;
+          const __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w);
+          const __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
+          w = make_uint4(*reinterpret_cast<const uint32_t*>(&p0), *reinterpret_cast<const uint32_t*>(&p1),
+                         *reinterpret_cast<const uint32_t*>(&p2), *reinterpret_cast<const uint32_t*>(&p3));
+        }
+        const int kb = ci >> 3, chunk = ci & 7;
+        *reinterpret_cast<uint4*>(xt + (size_t)kb * 2048 + j * 128 + ((chunk ^ (j & 7)) << 4)) = w;
+      }
+      sq = warp_sum(sq);
+      if (lane == 0) rs[j] = live ? rsqrtf(sq / (float)C + eps) : 0.f;
+    }
+    ptx::fence_proxy_async_smem();  // the tensor core reads x^T through the async proxy
+    asm volatile("bar.sync 1, %0;" ::"r"(32 * 5));
+
+    if (warp == 1) {
+      // ---------------- MMA issuer ----------------
+      if (ptx::elect_one()) {
+        constexpr uint32_t idesc = ptx::idesc_bf16(128, kLtN);
+        const uint32_t xt0 = ptx::smem_u32(xt);
+        int k = 0, pass = 0;
+        bool ok = true;
+        for (int ub = u_lo; ub < u_hi && ok; ub += kLtUnitsMax, ++pass) {
+          const int nu = min(kLtUnitsMax, u_hi - ub);
+          const int buf = pass & 1;
+          if (*abort_flag || !ptx::mbar_wait(tempty(buf), ((uint32_t)(pass >> 1) & 1u) ^ 1u, status)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t d = tmem + (uint32_t)(buf * 2 * kLtN);
+          for (int kb = 0; kb < nkb; ++kb, ++k) {
+            const int s = k % stages;
+            if (*abort_flag || !ptx::mbar_wait(full(s), (uint32_t)(k / stages) & 1u, status)) {
+              ok = false;
+              break;
+            }
+            ptx::tc_fence_after();
+            const uint32_t a0 = ptx::smem_u32(ring + (size_t)s * kLtStageBytes);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t bd = ptx::desc_kmajor_sw128(xt0 + (uint32_t)(kb * 2048 + kk * 32));
+              const uint32_t acc = (kb | kk) != 0;
+              ptx::mma_bf16_ss(d, ptx::desc_kmajor_sw128(a0 + (uint32_t)(kk * 32)), bd, idesc, acc);
+              if (nu > 4)
+                ptx::mma_bf16_ss(d + kLtN, ptx::desc_kmajor_sw128(a0 + 16384u + (uint32_t)(kk * 32)), bd, idesc, acc);
+            }
+            ptx::mma_commit(empty(s));
+          }
+          if (ok) ptx::mma_commit(tfull(buf));
+        }
+        if (!ok) *abort_flag = 1;
+        // every issued MMA has completed before TMEM is released
+        ptx::mma_commit(done);
+        ptx::mbar_wait(done, 0, status);
+      }
+    } else {
+      // ---------------- epilogue (warps 2..5) ----------------
+      const int q = warp & 3;  // TMEM lane quarter this warp may access
+      int pass = 0;
+      for (int ub = u_lo; ub < u_hi; ub += kLtUnitsMax, ++pass) {
+        const int nu = min(kLtUnitsMax, u_hi - ub);
+        const int buf = pass & 1;
+        if (*abort_flag || !ptx::mbar_wait(tfull(buf), (uint32_t)(pass >> 1) & 1u, status)) {
+          *abort_flag = 1;
+          break;
+        }
+        ptx::tc_fence_after();
+        const int row_end = min((ub + nu) * kLtUnit, V);
+        for (int t = 0; t < (nu > 4 ? 2 : 1); ++t) {
+          uint32_t r[16];
+          ptx::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 2 * kLtN + t * kLtN), r);
+          ptx::tmem_ld_wait();
+          const int row = ub * kLtUnit + t * 128 + q * 32 + lane;
+          if (row < row_end) {
+#pragma unroll
+            for (int j = 0; j < kLtN; ++j)
+              if (j < nb) out[(size_t)(b0 + j) * ldo + row] = cap * tanhf(__uint_as_float(r[j]) * rs[j] / cap);
+          }
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(tempty(buf));
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kLtTmemCols);
   }
 }
 
@@ -548,8 +773,31 @@ void launch_last_logits_t(const float* x, int ldx, int B, int T, const TW* W, in
 
 }  // namespace
 
+// The tensor-core form: bf16 W_U with C a multiple of 64 and room for two
+// ring stages next to x^T.  False when it does not apply or its tensor map
+// cannot be made (the CUDA-core form then runs).
+static bool launch_last_logits_tc(const float* x, int ldx, int B, int T, const bf16* W, int V, int C, float cap, float eps,
+                           float* out, int ldo, int num_sms, int* status, cudaStream_t st) {
+  if (C % 64 != 0 || V <= 0 || ldx % 4 != 0) return false;
+  const LtGeom g = lt_geom(C);
+  if (g.stages < 2) return false;
+  CUtensorMap tm;
+  if (!make_tmap_2d(&tm, W, V, C, C, kLtUnit, 64)) return false;
+  if (!smem_optin(k_last_logits_tc, 220 * 1024)) return false;
+  for (int b0 = 0; b0 < B; b0 += kLtN) {
+    const int nb = B - b0 < kLtN ? B - b0 : kLtN;
+    LaunchScope scope_(KK_LAST_LOGITS, st);
+    launch_pdl(k_last_logits_tc, dim3(num_sms), dim3(kLtThreads), g.smem, st, 1, tm, x, ldx, T, b0, nb, V, C, cap, eps,
+               out, ldo, g.stages, status);
+  }
+  return true;
+}
+
 void launch_last_logits(const float* x, int ldx, int B, int T, const void* W, int V, int C, bool bf, float cap,
                         float eps, float* out, int ldo, int num_sms, int* status, cudaStream_t st) {
+  if (bf && launch_last_logits_tc(x, ldx, B, T, static_cast<const bf16*>(W), V, C, cap, eps, out, ldo, num_sms,
+                                  status, st))
+    return;
   if (bf)
     launch_last_logits_t(x, ldx, B, T, static_cast<const bf16*>(W), V, C, cap, eps, out, ldo, num_sms, status, st);
   else

@@ -14,7 +14,7 @@
 
 #include <atomic>
 #include <mutex>
-#include <set>
+#include <map>
 #include <utility>
 
 #include "nc_internal.cuh"
@@ -86,7 +86,7 @@ void flag_wait_test(unsigned long long* limit_ns, unsigned* skew) {
 
 namespace {
 std::mutex g_optin_mu;
-std::set<std::pair<const void*, int>> g_optin_done;  // (kernel, device) pairs already raised
+std::map<std::pair<const void*, int>, int> g_optin_done;  // (kernel, device) -> dynamic shared memory limit set
 }  // namespace
 
 bool smem_optin(const void* kernel, int bytes) {
@@ -98,13 +98,14 @@ bool smem_optin(const void* kernel, int bytes) {
   }
   std::lock_guard<std::mutex> lk(g_optin_mu);
   const std::pair<const void*, int> key(kernel, dev);
-  if (g_optin_done.count(key)) return true;
+  const auto it = g_optin_done.find(key);
+  if (it != g_optin_done.end() && it->second >= bytes) return true;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) {
     set_err("cudaFuncSetAttribute", e);
     return false;
   }
-  g_optin_done.insert(key);
+  g_optin_done[key] = bytes;
   return true;
 }
 

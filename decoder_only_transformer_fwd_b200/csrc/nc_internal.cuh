@@ -211,9 +211,9 @@ bool launch_attn_tc(const bf16* q, const bf16* k, const bf16* v, int ldq, int ld
                     int num_sms, cudaStream_t st);
 
 // Raise `kernel`'s dynamic shared-memory limit to `bytes` on the current
-// device.  The attribute belongs to the device's context, so it is set once
-// per (kernel, device): a process that drives several devices sets it on
-// each.  Returns false, with the CUDA error recorded for nc_last_error(),
+// device.  The attribute belongs to the device's context, so it is set per
+// (kernel, device): a process that drives several devices sets it on each,
+// and a later request for more bytes than the last one raises it again.  Returns false, with the CUDA error recorded for nc_last_error(),
 // when the device cannot be queried or the attribute cannot be set.
 bool smem_optin(const void* kernel, int bytes);
 template <typename... KArgs>

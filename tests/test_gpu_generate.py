@@ -153,11 +153,35 @@ def _last_logits(cfg, p, tok):
 @pytest.mark.parametrize("depth,B,T,short,dtype", [
     (4, 2, 300, 128, "bf16"), (4, 9, 64, 32, "bf16"), (1, 3, 77, 77, "fp32"), (12, 1, 200, 64, "bf16")])
 def test_last_logits_match_oracle(depth, B, T, short, dtype):
-    """B = 9 spans two launches of eight rows."""
+    """bf16 runs the tensor-core form (up to 16 rows per launch, so B = 9 is
+    one launch); fp32 runs the CUDA-core form (eight rows per launch)."""
     cfg, ocfg, p, tok, _ = make_case(depth, B, T, short, dtype, 600 + B * T)
     z, rc, _ = _last_logits(cfg, p, tok)
     assert rc == 0
     _check_last_logits(ocfg, p, tok, z, dtype)
+
+
+@pytest.mark.parametrize("V,B", [(1000, 3), (50000, 17)])
+def test_last_logits_vocab_shapes(V, B):
+    """Vocabularies that are not a multiple of the 32-row unit the tensor-core
+    head streams W_U in: V = 1000 (fewer units than SMs, a partial last unit)
+    and V = 50000 (more than eight units per CTA, so the CTAs take two passes
+    through their two TMEM buffers); B = 17 spans two launches of 16 rows."""
+    import torch
+    depth, T, short = 2, 48, 32
+    cfg = nc.nc_init_config(depth, T, "bf16", "SSSL", short, -1)
+    cfg.vocab = V
+    cfg.vocab_padded = O.padded_vocab(V)
+    ocfg = O.make_config(depth, T, short, vocab=V)
+    seed = 900 + V + B
+    p = synth.params(seed, n_layer=cfg.n_layer, n_embd=cfg.n_embd, n_head=cfg.n_head, n_kv_head=cfg.n_kv_head,
+                     head_dim=cfg.head_dim, vocab=V, vocab_padded=cfg.vocab_padded, ve_layers=ocfg["ve_layers"],
+                     bf16=True)
+    tok = synth.tokens(seed, B, T, V)
+    z, rc, _ = _last_logits(cfg, p, tok)
+    assert rc == 0
+    assert z.shape == (B, V)
+    _check_last_logits(ocfg, p, tok, z, "bf16")
 
 
 def test_last_logits_equal_full_forward_last_position():
