@@ -261,51 +261,66 @@ k_last_logits(const float* __restrict__ x, int ldx, int T, int b0, const TW* __r
 // vocabulary rows as M and the (at most 16) x rows as N:
 //   * x^T is staged once per CTA in shared memory as the B operand (bf16,
 //     K-major, 128-byte swizzle: for each 64-wide k block, 16 rows of 128 B);
-//   * W_U streams through a ring of 32 KB stages by TMA, one 32-row x 64-k box
-//     per 32-row unit (128-byte swizzle); a stage holds up to 8 units, i.e.
-//     two M = 128 tiles;
+//   * W_U streams through a ring of stages by TMA, one 32-row x 64-k box per
+//     32-row unit (128-byte swizzle); a stage holds the 4 to 8 units a CTA
+//     takes per pass, covered by one or two M = 128 tiles (the second one
+//     ends at the last unit, overlapping the first);
 //   * one thread issues tcgen05.mma (M = 128, N = 16, K = 16) into TMEM; four
 //     epilogue warps read D (lane = vocabulary row, column = x row), apply
 //     the RMSNorm scale and the softcap and store one row of each x row per
 //     lane, so a warp's stores are 128 contiguous bytes.
 // Each CTA owns a contiguous run of units (the units spread evenly over the
-// grid), taken in passes of at most 8 units with two TMEM buffers.  Every
+// grid), taken in passes of at most 8 units with two TMEM buffers.  W_U does
+// not depend on the previous kernel, so the copy thread issues the first
+// three stages before the programmatic-dependency wait clears; it issues the
+// rest once the staging threads have sent out their x loads, so that those
+// do not queue behind a full ring of W_U copies (the first MMA needs x^T).  Every
 // wait is bounded; on a timeout the CTA records NC_ERR_TIMEOUT and returns
 // once its copies and MMAs have landed.
 constexpr int kLtUnit = 32;                                 // vocabulary rows per TMA box
 constexpr int kLtUnitsMax = 8;                              // units per pass (two M = 128 tiles)
 constexpr int kLtN = 16;                                    // MMA N: x rows of one launch
 constexpr int kLtBoxBytes = kLtUnit * 128;                  // 4 KB: 32 rows x 64 bf16
-constexpr int kLtStageBytes = kLtUnitsMax * kLtBoxBytes;    // 32 KB
-constexpr int kLtMaxStages = 5;
+constexpr int kLtMaxStages = 8;
 constexpr int kLtThreads = 192;                             // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr uint32_t kLtTmemCols = 64;                        // 2 buffers x 2 tiles x 16 columns
 
+constexpr int kLtSmemLimit = 227 * 1024;
+
+// su: units per pass (and per stage), from the units a CTA of the grid takes,
+// at least 4 (one full M = 128 tile) and at most 8; stages: as many as fit.
 struct LtGeom {
-  int stages;
-  size_t xt_bytes, smem;
+  int su, stages;
+  size_t xt_bytes, stage_bytes, smem;
 };
-inline LtGeom lt_geom(int C) {
+inline LtGeom lt_geom(int C, int V, int grid) {
   LtGeom g;
+  const int nunits = (V + kLtUnit - 1) / kLtUnit;
+  const int per_cta = grid > 0 ? (nunits + grid - 1) / grid : kLtUnitsMax;
+  g.su = per_cta < 4 ? 4 : (per_cta > kLtUnitsMax ? kLtUnitsMax : per_cta);
   g.xt_bytes = (size_t)kLtN * C * 2;
-  const size_t limit = 220 * 1024, fixed = 1024 + 256;
+  g.stage_bytes = (size_t)g.su * kLtBoxBytes;
+  // (256 bytes of the limit are left to the kernel's static shared memory)
+  const size_t limit = kLtSmemLimit - 256, fixed = 1024 + 256;
   const size_t avail = limit > fixed + g.xt_bytes ? limit - fixed - g.xt_bytes : 0;
-  g.stages = (int)(avail / kLtStageBytes);
+  g.stages = (int)(avail / g.stage_bytes);
   if (g.stages > kLtMaxStages) g.stages = kLtMaxStages;
-  g.smem = fixed + g.xt_bytes + (size_t)g.stages * kLtStageBytes;
+  g.smem = fixed + g.xt_bytes + (size_t)g.stages * g.stage_bytes;
   return g;
 }
 
 __global__ void __launch_bounds__(kLtThreads, 1)
 k_last_logits_tc(const __grid_constant__ CUtensorMap tmW, const float* __restrict__ x, int ldx, int T, int b0, int nb,
-                 int V, int C, float cap, float eps, float* __restrict__ out, int ldo, int stages, int* status) {
+                 int V, int C, float cap, float eps, float* __restrict__ out, int ldo, int su, int stages,
+                 int* status) {
   pdl_launch_dependents();
   extern __shared__ uint8_t lt_raw[];
+  const size_t stage_bytes = (size_t)su * kLtBoxBytes;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lt_raw) + 1023) & ~uintptr_t(1023));
   const int nkb = C / 64;
   uint8_t* xt = smem;                                   // nkb blocks of 2 KB
   uint8_t* ring = smem + (size_t)kLtN * C * 2;          // a multiple of 2 KB past a 1 KB boundary
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + (size_t)stages * kLtStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + (size_t)stages * stage_bytes);
   // full[kLtMaxStages] | empty[kLtMaxStages] | tfull[2] | tempty[2] | done
   const uint32_t bar0 = ptx::smem_u32(bars);
   auto full = [&](int s) { return bar0 + 8u * s; };
@@ -313,11 +328,13 @@ k_last_logits_tc(const __grid_constant__ CUtensorMap tmW, const float* __restric
   auto tfull = [&](int b) { return bar0 + 8u * (2 * kLtMaxStages + b); };
   auto tempty = [&](int b) { return bar0 + 8u * (2 * kLtMaxStages + 2 + b); };
   const uint32_t done = bar0 + 8u * (2 * kLtMaxStages + 4);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kLtMaxStages + 5);
+  const uint32_t xbar = bar0 + 8u * (2 * kLtMaxStages + 5);  // the staging threads' x loads are issued
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kLtMaxStages + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  __shared__ float rs[kLtN];
+  __shared__ float ssq[kLtN];  // sum of squares of each x row
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  if (threadIdx.x < kLtN) ssq[threadIdx.x] = 0.f;
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
       ptx::mbar_init(full(s), 1);
@@ -328,6 +345,7 @@ k_last_logits_tc(const __grid_constant__ CUtensorMap tmW, const float* __restric
       ptx::mbar_init(tempty(b), 4);
     }
     ptx::mbar_init(done, 1);
+    ptx::mbar_init(xbar, 32 * 5);
     *abort_flag = 0;
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tmW);
@@ -344,23 +362,27 @@ k_last_logits_tc(const __grid_constant__ CUtensorMap tmW, const float* __restric
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_wait();  // x comes from the previous kernel
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (reads only W_U: no dependency wait) ----------------
     if (ptx::elect_one()) {
       int k = 0;
       bool ok = true;
-      for (int ub = u_lo; ub < u_hi && ok; ub += kLtUnitsMax) {
-        const int nu = min(kLtUnitsMax, u_hi - ub);
+      const int early = min(3, stages);  // stages issued before the x loads
+      for (int ub = u_lo; ub < u_hi && ok; ub += su) {
+        const int nu = min(su, u_hi - ub);
         for (int kb = 0; kb < nkb; ++kb, ++k) {
           const int s = k % stages;
+          if (k == early && !ptx::mbar_wait(xbar, 0, status)) {
+            ok = false;
+            break;
+          }
           if (*abort_flag || !ptx::mbar_wait(empty(s), ((uint32_t)(k / stages) & 1u) ^ 1u, status)) {
             ok = false;
             break;
           }
           ptx::mbar_arrive_expect_tx(full(s), (uint32_t)(nu * kLtBoxBytes));
-          const uint32_t dst = ptx::smem_u32(ring + (size_t)s * kLtStageBytes);
+          const uint32_t dst = ptx::smem_u32(ring + (size_t)s * stage_bytes);
           for (int i = 0; i < nu; ++i)
             ptx::tma_load_2d(dst + (uint32_t)(i * kLtBoxBytes), &tmW, full(s), kb * 64, (ub + i) * kLtUnit);
         }
@@ -371,29 +393,55 @@ k_last_logits_tc(const __grid_constant__ CUtensorMap tmW, const float* __restric
         ptx::mbar_wait(full(q % stages), (uint32_t)(q / stages) & 1u, status);
     }
   } else {
+    pdl_wait();  // x comes from the previous kernel
     // ---------------- stage x^T (warps 1..5) ----------------
-    // warp w takes x rows j = w - 1, w + 4, ...; lane c handles the 16-byte
-    // chunks c, c + 32, ... (8 consecutive k) of the row
-    for (int j = warp - 1; j < kLtN; j += 5) {
-      const bool live = j < nb;
-      const float* xr = x + ((size_t)(b0 + (live ? j : 0)) * T + (T - 1)) * ldx;
-      float sq = 0.f;
-      for (int ci = lane; ci < C / 8; ci += 32) {
-        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    // The chunks (8 consecutive k, 16 bytes of bf16) of all rows are spread
+    // over the 160 threads; each thread issues the loads of up to five
+    // chunks before it uses any of them, so the staging costs about one
+    // memory round trip per round rather than one per chunk.
+    const int tid = threadIdx.x - 32, nth = 32 * 5;
+    const int cpr = C / 8;
+    auto chunk_at = [&](int j, int ci) {
+      return reinterpret_cast<uint4*>(xt + (size_t)(ci >> 3) * 2048 + j * 128 + (((ci & 7) ^ (j & 7)) << 4));
+    };
+    for (int t = tid; t < (kLtN - nb) * cpr; t += nth) *chunk_at(nb + t / cpr, t % cpr) = make_uint4(0u, 0u, 0u, 0u);
+    constexpr int U = 5;  // d24 widths, four rows: 768 chunks, one round over 160 threads
+    for (int t0 = tid, round = 0; t0 < nb * cpr || round == 0; t0 += U * nth, ++round) {
+      float4 va[U], vb[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int t = t0 + u * nth;
+        va[u] = vb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (t < nb * cpr) {
+          const float* xr = x + ((size_t)(b0 + t / cpr) * T + (T - 1)) * ldx + 8 * (t % cpr);
+          va[u] = *reinterpret_cast<const float4*>(xr);
+          vb[u] = *reinterpret_cast<const float4*>(xr + 4);
+        }
+      }
+      if (round == 0) ptx::mbar_arrive_relaxed(xbar);  // every staging thread, once
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int t = t0 + u * nth;
+        const bool live = t < nb * cpr;
+        float sq = 0.f;
         if (live) {
-          const float4 a = *reinterpret_cast<const float4*>(xr + 8 * ci);
-          const float4 b = *reinterpret_cast<const float4*>(xr + 8 * ci + 4);
-          sq += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w + b.x * b.x + b.y * b.y + b.z * b.z + b.w * b.w;
+          const float4 a = va[u], b = vb[u];
+          sq = a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w + b.x * b.x + b.y * b.y + b.z * b.z + b.w * b.w;
           const __nv_bfloat162 p0 = __floats2bfloat162_rn(a.x, a.y), p1 = __floats2bfloat162_rn(a.z, a.w);
           const __nv_bfloat162 p2 = __floats2bfloat162_rn(b.x, b.y), p3 = __floats2bfloat162_rn(b.z, b.w);
-          w = make_uint4(*reinterpret_cast<const uint32_t*>(&p0), *reinterpret_cast<const uint32_t*>(&p1),
+          *chunk_at(t / cpr, t % cpr) =
+              make_uint4(*reinterpret_cast<const uint32_t*>(&p0), *reinterpret_cast<const uint32_t*>(&p1),
                          *reinterpret_cast<const uint32_t*>(&p2), *reinterpret_cast<const uint32_t*>(&p3));
         }
-        const int kb = ci >> 3, chunk = ci & 7;
-        *reinterpret_cast<uint4*>(xt + (size_t)kb * 2048 + j * 128 + ((chunk ^ (j & 7)) << 4)) = w;
+        if (cpr % 32 == 0) {
+          // a warp's 32 consecutive chunks lie in one row and are all live
+          // or all not: one shared-memory atomic per warp, not 32 on one word
+          sq = warp_sum(sq);
+          if (lane == 0 && live) atomicAdd(&ssq[t / cpr], sq);
+        } else if (live) {
+          atomicAdd(&ssq[t / cpr], sq);
+        }
       }
-      sq = warp_sum(sq);
-      if (lane == 0) rs[j] = live ? rsqrtf(sq / (float)C + eps) : 0.f;
     }
     ptx::fence_proxy_async_smem();  // the tensor core reads x^T through the async proxy
     asm volatile("bar.sync 1, %0;" ::"r"(32 * 5));
@@ -405,8 +453,8 @@ k_last_logits_tc(const __grid_constant__ CUtensorMap tmW, const float* __restric
         const uint32_t xt0 = ptx::smem_u32(xt);
         int k = 0, pass = 0;
         bool ok = true;
-        for (int ub = u_lo; ub < u_hi && ok; ub += kLtUnitsMax, ++pass) {
-          const int nu = min(kLtUnitsMax, u_hi - ub);
+        for (int ub = u_lo; ub < u_hi && ok; ub += su, ++pass) {
+          const int nu = min(su, u_hi - ub);
           const int buf = pass & 1;
           if (*abort_flag || !ptx::mbar_wait(tempty(buf), ((uint32_t)(pass >> 1) & 1u) ^ 1u, status)) {
             ok = false;
@@ -421,14 +469,16 @@ k_last_logits_tc(const __grid_constant__ CUtensorMap tmW, const float* __restric
               break;
             }
             ptx::tc_fence_after();
-            const uint32_t a0 = ptx::smem_u32(ring + (size_t)s * kLtStageBytes);
+            const uint32_t a0 = ptx::smem_u32(ring + (size_t)s * stage_bytes);
+            // the second tile covers the pass's last 128 rows (units nu - 4 .. nu - 1)
+            const uint32_t a1 = a0 + (uint32_t)((nu - 4) * kLtBoxBytes);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t bd = ptx::desc_kmajor_sw128(xt0 + (uint32_t)(kb * 2048 + kk * 32));
               const uint32_t acc = (kb | kk) != 0;
               ptx::mma_bf16_ss(d, ptx::desc_kmajor_sw128(a0 + (uint32_t)(kk * 32)), bd, idesc, acc);
               if (nu > 4)
-                ptx::mma_bf16_ss(d + kLtN, ptx::desc_kmajor_sw128(a0 + 16384u + (uint32_t)(kk * 32)), bd, idesc, acc);
+                ptx::mma_bf16_ss(d + kLtN, ptx::desc_kmajor_sw128(a1 + (uint32_t)(kk * 32)), bd, idesc, acc);
             }
             ptx::mma_commit(empty(s));
           }
@@ -442,9 +492,12 @@ k_last_logits_tc(const __grid_constant__ CUtensorMap tmW, const float* __restric
     } else {
       // ---------------- epilogue (warps 2..5) ----------------
       const int q = warp & 3;  // TMEM lane quarter this warp may access
+      float rs[kLtN];          // 1 / rms of each x row
+#pragma unroll
+      for (int j = 0; j < kLtN; ++j) rs[j] = rsqrtf(ssq[j] / (float)C + eps);
       int pass = 0;
-      for (int ub = u_lo; ub < u_hi; ub += kLtUnitsMax, ++pass) {
-        const int nu = min(kLtUnitsMax, u_hi - ub);
+      for (int ub = u_lo; ub < u_hi; ub += su, ++pass) {
+        const int nu = min(su, u_hi - ub);
         const int buf = pass & 1;
         if (*abort_flag || !ptx::mbar_wait(tfull(buf), (uint32_t)(pass >> 1) & 1u, status)) {
           *abort_flag = 1;
@@ -456,11 +509,15 @@ k_last_logits_tc(const __grid_constant__ CUtensorMap tmW, const float* __restric
           uint32_t r[16];
           ptx::tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 2 * kLtN + t * kLtN), r);
           ptx::tmem_ld_wait();
-          const int row = ub * kLtUnit + t * 128 + q * 32 + lane;
-          if (row < row_end) {
+          // row of the pass: tile 0 holds rows 0..127, tile 1 rows (nu - 4) * 32 .. nu * 32 - 1,
+          // of which it stores those past 127
+          const int rp = (t == 0 ? 0 : (nu - 4) * kLtUnit) + q * 32 + lane;
+          const int row = ub * kLtUnit + rp;
+          if (row < row_end && (t == 0 || rp >= 128)) {
 #pragma unroll
             for (int j = 0; j < kLtN; ++j)
-              if (j < nb) out[(size_t)(b0 + j) * ldo + row] = cap * tanhf(__uint_as_float(r[j]) * rs[j] / cap);
+              if (j < nb)
+                out[(size_t)(b0 + j) * ldo + row] = cap * tanhf(__uint_as_float(r[j]) * rs[j] / cap);
           }
         }
         ptx::tc_fence_before();
@@ -779,16 +836,16 @@ void launch_last_logits_t(const float* x, int ldx, int B, int T, const TW* W, in
 static bool launch_last_logits_tc(const float* x, int ldx, int B, int T, const bf16* W, int V, int C, float cap, float eps,
                            float* out, int ldo, int num_sms, int* status, cudaStream_t st) {
   if (C % 64 != 0 || V <= 0 || ldx % 4 != 0) return false;
-  const LtGeom g = lt_geom(C);
+  const LtGeom g = lt_geom(C, V, num_sms);
   if (g.stages < 2) return false;
   CUtensorMap tm;
   if (!make_tmap_2d(&tm, W, V, C, C, kLtUnit, 64)) return false;
-  if (!smem_optin(k_last_logits_tc, 220 * 1024)) return false;
+  if (!smem_optin(k_last_logits_tc, (int)g.smem)) return false;
   for (int b0 = 0; b0 < B; b0 += kLtN) {
     const int nb = B - b0 < kLtN ? B - b0 : kLtN;
     LaunchScope scope_(KK_LAST_LOGITS, st);
     launch_pdl(k_last_logits_tc, dim3(num_sms), dim3(kLtThreads), g.smem, st, 1, tm, x, ldx, T, b0, nb, V, C, cap, eps,
-               out, ldo, g.stages, status);
+               out, ldo, g.su, g.stages, status);
   }
   return true;
 }
