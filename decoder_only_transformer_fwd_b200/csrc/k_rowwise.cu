@@ -93,8 +93,9 @@ __global__ void k_embed(const T* __restrict__ wte, const int32_t* __restrict__ t
   }
 }
 
-// bf16 tables, C = 32 * EPL: one warp walks a run of `run` consecutive
-// positions of one row.  Lane l holds elements [4 (k * 32 + l), + 4) of every
+// bf16 tables, C = 32 * EPL: one warp walks a run of `run` (<= 32)
+// consecutive positions of one row; lane i loads the run's i-th token id up
+// front, so no row load waits for its id.  Lane l holds elements [4 (k * 32 + l), + 4) of every
 // row for k < EPL / 4, so each warp-wide access is contiguous: 256 bytes of a
 // bf16 row, 512 bytes of an fp32 row.  The next position's embedding row is
 // requested before the current one is normalised and stored, so a warp keeps
@@ -140,14 +141,15 @@ __global__ void __launch_bounds__(64) k_embed_vec(
 #pragma unroll
     for (int i = 0; i < EPL; ++i) v[i] *= r;
   };
-  auto token = [&](int t) {
-    int tok = tokens[(size_t)b * T_ + t];
-    if (tok < 0 || tok >= V) {
-      if (lane == 0) atomicOr(status, kStatusData);
-      tok = min(max(tok, 0), V - 1);
+  int my_tok = 0;  // lane i: the id at position t0 + i, clamped
+  if (lane < t1 - t0) {
+    my_tok = tokens[(size_t)b * T_ + t0 + lane];
+    if (my_tok < 0 || my_tok >= V) {
+      atomicOr(status, kStatusData);
+      my_tok = min(max(my_tok, 0), V - 1);
     }
-    return tok;
-  };
+  }
+  auto token = [&](int t) { return __shfl_sync(0xffffffffu, my_tok, t - t0); };
   float prev[EPL];
   uint2 raw[NCH], nxt[NCH];
   if (smear && t0 > 0) {
@@ -511,6 +513,7 @@ __global__ void k_ce_combine(const float* ce_sum, const float* ce_tgt, int n_til
   if ((n_tiles & 3) == 0) {
     // 16-byte loads: a row of 2 V_pad / 128 partial sums is 2 KB at V = 32768
     const float4* p4 = reinterpret_cast<const float4*>(ps);
+#pragma unroll 4
     for (int i = lane; i < n_tiles / 4; i += 32) {
       const float4 v = p4[i];
       s += (v.x + v.y) + (v.z + v.w);
