@@ -25,7 +25,8 @@ from __future__ import annotations
 
 import numpy as np
 
-NORTH_STAR = {"loss": 1e-2, "logits": 3e-2}
+# the stated bf16 tolerances: per-token loss and softcapped logits, absolute
+STATED_TOL = {"loss": 1e-2, "logits": 3e-2}
 
 
 def _stats(err, tol):
@@ -37,7 +38,7 @@ def _stats(err, tol):
 def check(kind, gpu, ref, emu):
     """Assert the rules above for one kind of output ('loss' or 'logits');
     returns the GPU's and the emulation's statistics."""
-    tol = NORTH_STAR[kind]
+    tol = STATED_TOL[kind]
     assert np.all(np.isfinite(gpu)), f"{kind}: non-finite values"
     g = _stats(np.asarray(gpu, np.float64) - ref, tol)
     e = _stats(np.asarray(emu, np.float64) - ref, tol)
