@@ -543,6 +543,11 @@ def run_ours(args):
                         "24 O, 24 FC1, 23 FC2 + 1 last-block FC2, 1 head per 97 launches)",
         "launches": n_gemm, "avg_launch_us": 1e3 * gemm_ms / max(n_gemm, 1),
         "share_of_step": gemm_ms / ms_total if ms_total > 0 else None,
+        "instrumented_ms_per_step": ms_step_b,
+        "timing_note": "avg_launch_us and achieved come from CUDA events recorded around every launch; those "
+                       "events cut the programmatic-dependent-launch overlap between kernels, so the step with "
+                       "them (instrumented_ms_per_step) runs longer than without (ms_per_step) and the per-launch "
+                       "times are upper bounds",
     }
 
     # the embedding kernel is HBM-bound: per launch it gathers M rows of W_E
