@@ -862,7 +862,10 @@ void launch_last_logits(const float* x, int ldx, int B, int T, const void* W, in
 }
 
 bool last_logits_supported(int C, bool bf) {
-  // at least two ring stages next to eight staged rows of x
+  // bf16 with C a multiple of 64: the tensor-core form, whose stages hold at
+  // most 8 units (its geometry for a grid that gives each CTA 8 units or more)
+  if (bf && C > 0 && C % 64 == 0 && lt_geom(C, kLtUnitsMax * kLtUnit, 1).stages >= 2) return true;
+  // otherwise the CUDA-core form: two ring stages next to eight staged rows of x
   return C > 0 && last_geom(C, bf ? 2 : 4, kLastRows).stages >= 2;
 }
 

@@ -176,12 +176,15 @@ def test_generation_entry_points_reject_bad_arguments():
     assert lib.nc_generate_next(C.byref(p), a16, 1, 8, -1.0, 0, a16, a16, a16, None) == SHAPE
 
 
-@pytest.mark.parametrize("dtype,C_ok,C_bad", [("bf16", 2304, 2432), ("fp32", 1280, 1408)])
+@pytest.mark.parametrize("dtype,C_ok,C_bad", [("bf16", 5120, 5248), ("fp32", 1280, 1408)])
 def test_last_logits_width_limit(dtype, C_ok, C_bad):
-    """The last-position head stages eight rows of x next to two stages of 16
-    W_U rows in 220 KB of shared memory: C <= 2304 in bf16, <= 1280 in fp32.
-    Past the limit the call is rejected before any launch; at the limit it
-    gets as far as the (missing) workspace."""
+    """The last-position head keeps the x rows in shared memory next to at
+    least two stages of W_U: in bf16 (tensor-core form, C a multiple of 64)
+    16 rows of x^T at 2 C bytes each and two 32 KB stages within 227 KB, so
+    C <= 5168; in fp32 (CUDA-core form) eight fp32 rows next to two stages of
+    16 W_U rows within 220 KB, so C <= 1280.  Past the limit the call is
+    rejected before any launch; at the limit it gets as far as the (missing)
+    workspace."""
     lib = nc.lib()
     buf = (C.c_byte * 4096)()
     a16 = C.c_void_p((C.addressof(buf) + 15) & ~15)
