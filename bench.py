@@ -157,12 +157,13 @@ def run_reference(args):
                           vocab_padded=ocfg["vocab_padded"], ve_layers=ocfg["ve_layers"], bf16=True)
     tok = synth.tokens(seed, w["B"], w["T"], ocfg["vocab"])
     tgt = synth.targets(seed, w["B"], w["T"], ocfg["vocab"])
+    ntok = min(args.ref_tokens, w["T"])
     for _ in range(args.warmup):
-        cpu_oracle_run(ocfg, params, tok, tgt, CPU_SAMPLE_TOKENS)
-    times = [cpu_oracle_run(ocfg, params, tok, tgt, CPU_SAMPLE_TOKENS) for _ in range(args.steps)]
+        cpu_oracle_run(ocfg, params, tok, tgt, ntok)
+    times = [cpu_oracle_run(ocfg, params, tok, tgt, ntok) for _ in range(args.steps)]
     total = sum(times)
-    value = CPU_SAMPLE_TOKENS * args.steps / total
-    sample = (f"first {CPU_SAMPLE_TOKENS} positions of row 0 of the d24 batch per step "
+    value = ntok * args.steps / total
+    sample = (f"first {ntok} positions of row 0 of the d24 batch per step "
               f"(causal prefix: exact per-token losses), fp64 numpy oracle")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -625,6 +626,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tokens", type=int, default=1024)
+    ap.add_argument("--ref-tokens", type=int, default=CPU_SAMPLE_TOKENS,
+                    help="--impl reference: positions of row 0 the oracle runs per step")
     ap.add_argument("--rows", type=int, default=0, help="rows per step (default: the workload's B = 4)")
     ap.add_argument("--no-attention-sweep", action="store_true")
     ap.add_argument("--no-generation", action="store_true", help="skip the generation-step measurement")
@@ -637,6 +640,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if not 0 <= args.layers <= 24:
         ap.error("--layers must be in 0..24 (0: all 24 blocks)")
+    if args.ref_tokens < 1:
+        ap.error("--ref-tokens must be >= 1")
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
