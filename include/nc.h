@@ -154,8 +154,10 @@ int nc_forward_host(const nc_params* p, const int32_t* h_tokens, const int32_t* 
  *   out_logits [B, V] fp32 (device), out_logits[b] = 15 tanh(z/15) with
  *   z = RMSNorm(x_L[b, T-1]) W_U^T (in bf16 mode the normalised row is
  *   rounded to bf16 before the product, as in nc_forward).
- * Same requirements as nc_forward, plus C <= 2304 in bf16 mode (<= 1280 in
- * fp32 mode); no targets, no loss.
+ * Same requirements as nc_forward, plus a width the head supports: in bf16
+ * mode C a multiple of 64 up to 5168 (the tensor-core form) or C <= 2304,
+ * in fp32 mode C <= 1280 (NC_ERR_SHAPE otherwise, before any launch); no
+ * targets, no loss.
  * Status codes as nc_forward (NC_ERR_ARG for a NULL tokens/out_logits). */
 int nc_last_logits(const nc_params* p, const int32_t* tokens, int B, int T, float* out_logits,
                    void* stream);
