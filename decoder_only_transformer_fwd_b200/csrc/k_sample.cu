@@ -267,16 +267,17 @@ k_last_logits(const float* __restrict__ x, int ldx, int T, int b0, const TW* __r
 //     ends at the last unit, overlapping the first);
 //   * one thread issues tcgen05.mma (M = 128, N = 16, K = 16) into TMEM; four
 //     epilogue warps read D (lane = vocabulary row, column = x row), apply
-//     the RMSNorm scale and the softcap and store one row of each x row per
-//     lane, so a warp's stores are 128 contiguous bytes.
+//     the RMSNorm scale and the softcap, and each lane stores its vocabulary
+//     row's logit for every x row, so a warp's stores for one x row are 128
+//     contiguous bytes.
 // Each CTA owns a contiguous run of units (the units spread evenly over the
-// grid), taken in passes of at most 8 units with two TMEM buffers.  W_U does
-// not depend on the previous kernel, so the copy thread issues the first
-// three stages before the programmatic-dependency wait clears; it issues the
-// rest once the staging threads have sent out their x loads, so that those
-// do not queue behind a full ring of W_U copies (the first MMA needs x^T).  Every
-// wait is bounded; on a timeout the CTA records NC_ERR_TIMEOUT and returns
-// once its copies and MMAs have landed.
+// grid), taken in passes of 4 to 8 units (the stage size) with two TMEM
+// buffers.  W_U does not depend on the previous kernel, so the copy thread
+// issues the first three stages before the programmatic-dependency wait
+// clears; it issues the rest once the staging threads have sent out their x
+// loads, so that those do not queue behind a full ring of W_U copies (the
+// first MMA needs x^T).  Every wait is bounded; on a timeout the CTA records
+// NC_ERR_TIMEOUT and returns once its copies and MMAs have landed.
 constexpr int kLtUnit = 32;                                 // vocabulary rows per TMA box
 constexpr int kLtUnitsMax = 8;                              // units per pass (two M = 128 tiles)
 constexpr int kLtN = 16;                                    // MMA N: x rows of one launch
